@@ -1,0 +1,187 @@
+/*
+ * palu.h — C ABI of libpalu.so: Palu's decode step read straight from a
+ * low-rank latent KV cache, on NVIDIA B200 (sm_100a).
+ *
+ * The method (cited by page title and section):
+ *   "PALU 论文低秩投影分解：从数学结构到工程落地，一次讲透" (palu-low-rank explainer)
+ *     §低秩投影分解: K = x W_k ≈ x A_k B_k, V ≈ x A_v B_v with A ∈ R^{d_model×r},
+ *       B ∈ R^{r×d}; the cache holds z_k = x A_k and z_v = x A_v instead of K, V.
+ *     §把它放进一次真实推理流程里看 (Prefill 阶段 / Decode 阶段): prefill computes and
+ *       caches z; decode reads z and rebuilds K/V through B, or fuses that into the
+ *       attention kernel without materialising K/V.
+ *   "Palu: Compressing KV-Cache with Low-Rank Projection" (arXiv 2407.21118 v2
+ *     abstract): medium-grained (group-head) decomposition, RoPE-based attention,
+ *     quantisation compatibility, fused GPU kernels.
+ *
+ * Conventions shared by every entry point
+ *   - Heads are grouped consecutively: head h belongs to group h / group_size
+ *     and uses columns [(h % group_size)·head_dim, +head_dim) of its group's B.
+ *     G = num_heads / group_size groups, group width W = group_size·head_dim.
+ *   - All tensors are dense, row-major, in DEVICE memory owned by the caller.
+ *     The library allocates nothing, keeps no per-call state, and never frees
+ *     what it is given.  It caches CUDA tensor-map descriptors keyed by pointer
+ *     and shape; that cache is thread-safe.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream).  Argument checks are synchronous and return a status
+ *     before anything is launched.  Faults found by the kernels themselves
+ *     (a page index past the pool, a bounded wait that ran out) are recorded
+ *     in a status word at the start of the workspace, read back with
+ *     palu_get_device_status(); the kernels skip the bad access instead of
+ *     faulting.
+ *   - No exception, abort or trap crosses this ABI.
+ *
+ * Latent-cache layout (the "cache manager" side; paged by sequence):
+ *   K pool  [num_pages][G][page_size][row_k]    row_k = rank_k elements of the
+ *   V pool  [num_pages][G][page_size][row_v]    latent dtype (int4: rank/2 bytes)
+ *   int4 scale pools [num_pages][G][page_size][srow]   srow = 16-byte padded
+ *           rank/32 fp16 scales (one per 32 consecutive latent entries)
+ *   pos pool [num_pages][page_size] int32 (optional)
+ *   A token lives at slot = page·page_size + offset.  Rows are token-major and
+ *   16-byte aligned, so one page of one group is a 2-D tile a TMA box can move.
+ */
+#ifndef PALU_H_
+#define PALU_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* palu_stream_t; /* same handle as cudaStream_t */
+
+typedef enum palu_status {
+  PALU_OK = 0,
+  PALU_ERR_INVALID_ARG = 1,    /* NULL pointer, negative size, inconsistent shape */
+  PALU_ERR_UNSUPPORTED = 2,    /* a valid shape/dtype this build has no kernel for */
+  PALU_ERR_ALIGNMENT = 3,      /* a pointer or row stride not 16-byte aligned */
+  PALU_ERR_WORKSPACE = 4,      /* workspace NULL or smaller than the size query */
+  PALU_ERR_CUDA = 5,           /* a CUDA runtime/launch error (see palu_last_cuda_error) */
+  PALU_ERR_DEVICE_TIMEOUT = 6, /* a kernel's bounded wait ran out (device status) */
+  PALU_ERR_DEVICE_BOUNDS = 7   /* a kernel found a page/slot index out of range */
+} palu_status;
+
+typedef enum palu_dtype {
+  PALU_F32 = 0,
+  PALU_F16 = 1,
+  PALU_BF16 = 2,
+  PALU_INT4 = 3 /* latent dtype only */
+} palu_dtype;
+
+typedef struct palu_config {
+  int32_t num_heads;    /* H query heads (= KV heads) */
+  int32_t head_dim;     /* d_h, even */
+  int32_t group_size;   /* g heads share one latent (medium-grained decomposition) */
+  int32_t rank_k;       /* r_k latent width per group for keys */
+  int32_t rank_v;       /* r_v latent width per group for values */
+  int32_t page_size;    /* tokens per cache page */
+  float rope_base;      /* RoPE base (10000); 0 turns RoPE off */
+  int32_t act_dtype;    /* palu_dtype of q, x, A, B and out: F32 | F16 | BF16 */
+  int32_t latent_dtype; /* palu_dtype of the cache: act_dtype, or INT4 with F16/BF16 act */
+} palu_config;
+
+/* Bytes of one page of each pool for `cfg` (scale pages are 0 unless INT4).
+ * Returns PALU_ERR_INVALID_ARG / PALU_ERR_UNSUPPORTED for a bad config. */
+palu_status palu_cache_strides(const palu_config* cfg, size_t* k_page_bytes, size_t* v_page_bytes,
+                               size_t* k_scale_page_bytes, size_t* v_scale_page_bytes);
+
+/* Workspace bytes palu_compress_append needs for n_tokens rows (status word +
+ * any partial sums).  Always >= 256. */
+palu_status palu_compress_workspace_size(const palu_config* cfg, int n_tokens, int d_model,
+                                         size_t* bytes);
+
+/* Compress / append — the prefill (and per-step append) projection.
+ * "PALU 论文低秩投影分解" §低秩投影分解 (z_k = x A_k, z_v = x A_v) and
+ * §把它放进一次真实推理流程里看, Prefill 阶段 (compute z and cache it).
+ *
+ *   x        [n_tokens][d_model]        act dtype
+ *   A_k      [d_model][G·rank_k]        act dtype (group g = columns [g·r_k, +r_k))
+ *   A_v      [d_model][G·rank_v]        act dtype
+ *   slot_mapping [n_tokens] int32       destination slot page·page_size + offset;
+ *                                       a negative slot skips that row
+ *   positions [n_tokens] int32 or NULL  written to pos_pool[slot] when both are
+ *                                       non-NULL
+ *   zk_pool, zv_pool, zk_scales, zv_scales, pos_pool: the cache (layout above);
+ *            scales are used only for INT4 latents (else may be NULL)
+ *   num_pages  pool capacity in pages (slots >= num_pages·page_size are
+ *            skipped and reported as PALU_ERR_DEVICE_BOUNDS)
+ *
+ * Each latent row is z = x·A accumulated in float32 and rounded to nearest even
+ * into the latent dtype; INT4 rows are quantised per 32 entries with a
+ * symmetric fp16 scale s = fp16(max|z|/7) and codes clamp(rint(z/s), -7, 7),
+ * two's-complement nibbles, even entry in the low nibble.
+ * d_model must be a multiple of 64; every pointer 16-byte aligned.
+ */
+palu_status palu_compress_append(const palu_config* cfg, int n_tokens, int d_model,
+                                 const void* x, const void* A_k, const void* A_v,
+                                 const int32_t* slot_mapping, const int32_t* positions,
+                                 void* zk_pool, void* zv_pool, void* zk_scales, void* zv_scales,
+                                 int32_t* pos_pool, int num_pages,
+                                 void* workspace, size_t workspace_bytes, palu_stream_t stream);
+
+/* The split count palu_decode_attn uses when asked for num_splits = 0. */
+palu_status palu_decode_num_splits(const palu_config* cfg, int batch, int max_pages,
+                                   int* num_splits);
+
+/* Workspace bytes palu_decode_attn needs (status word + per-split partials
+ * (m, l, a[rank_v]) in float32 for every (sequence, head, split)). */
+palu_status palu_decode_workspace_size(const palu_config* cfg, int batch, int max_pages,
+                                       int num_splits, size_t* bytes);
+
+/* One decode step of attention over the latent cache.
+ * "PALU 论文低秩投影分解" §把它放进一次真实推理流程里看, Decode 阶段: read z, rebuild
+ * keys through B_k on the fly (K = z_k B_k, rotated by RoPE at each token's
+ * position), softmax(q'K'^T/sqrt(d_h)) over the cached tokens, and reduce values
+ * in latent space, out_h = (p · z_v) · B_v — V is never materialised.  The
+ * context is split into num_splits page ranges per sequence whose partials are
+ * merged by a log-sum-exp combine.
+ *
+ *   q          [batch][H][head_dim]   act dtype, before RoPE
+ *   q_pos      [batch] int32          the query's position
+ *   zk_pool ... pos_pool              the cache; pos_pool NULL => a token's
+ *                                     position is its index in the sequence
+ *   page_table [batch][max_pages] int32 physical page of each logical page
+ *   seq_lens   [batch] int32          cached tokens per sequence (0 allowed)
+ *   num_pages  pool capacity in pages (checked on the device)
+ *   B_k        [G][rank_k][W]         act dtype
+ *   B_v        [G][rank_v][W]         act dtype
+ *   out        [batch][H][head_dim]   act dtype (written)
+ *   lse        [batch][H] float32 or NULL: m + ln(sum), -inf for an empty sequence
+ *   workspace  >= palu_decode_workspace_size bytes, 256-byte aligned
+ *   num_splits 0 = automatic
+ * Attends over all seq_lens[b] tokens (the caller appends the current token
+ * first); an empty sequence gives out = 0.
+ */
+palu_status palu_decode_attn(const palu_config* cfg, int batch, const void* q, const int32_t* q_pos,
+                             const void* zk_pool, const void* zv_pool, const void* zk_scales,
+                             const void* zv_scales, const int32_t* pos_pool,
+                             const int32_t* page_table, int max_pages, const int32_t* seq_lens,
+                             int num_pages, const void* B_k, const void* B_v, void* out, float* lse,
+                             void* workspace, size_t workspace_bytes, int num_splits,
+                             palu_stream_t stream);
+
+/* Synchronises `stream`, then reads and clears the device status word at the
+ * start of `workspace`.  Returns PALU_OK, PALU_ERR_DEVICE_TIMEOUT or
+ * PALU_ERR_DEVICE_BOUNDS; *detail (optional) receives the kernel's detail code. */
+palu_status palu_get_device_status(void* workspace, palu_stream_t stream, int32_t* detail);
+
+/* Static description of a status code. */
+const char* palu_status_string(palu_status status);
+
+/* The last CUDA error string seen by this thread's calls ("" if none). */
+const char* palu_last_cuda_error(void);
+
+/* Which kernel family a decode call with this config would launch:
+ * 0 = none (unsupported), 1 = CUDA-core kernels, 2 = tcgen05/TMA kernels. */
+int palu_decode_kernel_kind(const palu_config* cfg);
+
+/* Number of CUDA kernels this library has launched in this process (all
+ * entry points, all devices).  A monotone counter for instrumentation. */
+uint64_t palu_kernel_launches(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PALU_H_ */

@@ -1,0 +1,301 @@
+// C-ABI layer of libpalu.so: argument checks, workspace layout, kernel choice.
+// Every entry point validates synchronously and returns a palu_status; nothing
+// throws or aborts across the ABI.
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <atomic>
+
+#include "palu_common.cuh"
+#include "palu_internal.h"
+#include "palu_tc.h"
+
+namespace palu {
+static std::atomic<unsigned long long> g_launches{0};
+void count_launch(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
+}  // namespace palu
+
+namespace {
+
+thread_local char g_cuda_err[256] = "";
+
+palu_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return PALU_OK;
+  snprintf(g_cuda_err, sizeof(g_cuda_err), "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
+  return PALU_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+palu_status check_config(const palu_config* c) {
+  if (c == nullptr) return PALU_ERR_INVALID_ARG;
+  if (c->num_heads <= 0 || c->head_dim <= 0 || c->group_size <= 0 || c->rank_k <= 0 ||
+      c->rank_v <= 0 || c->page_size <= 0)
+    return PALU_ERR_INVALID_ARG;
+  if (c->num_heads % c->group_size != 0) return PALU_ERR_INVALID_ARG;
+  if (c->head_dim % 2 != 0) return PALU_ERR_INVALID_ARG;
+  if (!(c->rope_base >= 0.f) || isinf(c->rope_base)) return PALU_ERR_INVALID_ARG;
+  if (c->act_dtype < PALU_F32 || c->act_dtype > PALU_BF16) return PALU_ERR_INVALID_ARG;
+  if (c->latent_dtype < PALU_F32 || c->latent_dtype > PALU_INT4) return PALU_ERR_INVALID_ARG;
+  // supported pairs: latent == act, or int4 latents with a 16-bit compute dtype
+  const bool pair_ok = (c->latent_dtype == c->act_dtype) ||
+                       (c->latent_dtype == PALU_INT4 && c->act_dtype != PALU_F32);
+  if (!pair_ok) return PALU_ERR_UNSUPPORTED;
+  if (c->head_dim > 2 * palu::kMaxHalfDim) return PALU_ERR_UNSUPPORTED;
+  if (c->rank_k > 512 || c->rank_v > 512) return PALU_ERR_UNSUPPORTED;
+  // 16-byte latent rows (TMA rows, vector stores); int4 needs whole 32-entry blocks
+  const int mult = c->latent_dtype == PALU_INT4 ? 32 : (c->latent_dtype == PALU_F32 ? 4 : 8);
+  if (c->rank_k % mult != 0 || c->rank_v % mult != 0) return PALU_ERR_ALIGNMENT;
+  return PALU_OK;
+}
+
+void fill_omega(const palu_config* c, uint64_t* omega) {
+  const int half = c->head_dim / 2;
+  const long double two_pi = 6.283185307179586476925286766559005768L;
+  for (int i = 0; i < palu::kMaxHalfDim; ++i) {
+    if (i >= half || c->rope_base == 0.f) {
+      omega[i] = 0;
+      continue;
+    }
+    const long double theta = powl((long double)c->rope_base, -2.0L * i / c->head_dim);
+    const long double turns = theta / two_pi;  // < 1
+    omega[i] = (uint64_t)llroundl(ldexpl(turns, 64));  // 64-bit fixed-point fraction (< 2^62)
+  }
+}
+
+constexpr size_t kStatusBytes = sizeof(palu::DevStatus);
+
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+int auto_splits(const palu_config* c, int batch, int max_pages, int kind) {
+  const int sms = 148;
+  const long long units = kind == 2 ? (long long)batch * (c->num_heads / c->group_size) *
+                                          palu::tc_head_blocks(c)
+                                    : (long long)batch * c->num_heads;
+  // enough CTAs for ~4 waves of one CTA per SM, but never more splits than pages
+  long long S = (4LL * sms + units - 1) / units;
+  if (kind == 2) {
+    // whole waves: round the CTA count up to a multiple of the SM count when cheap
+    S = (S < 1) ? 1 : S;
+  }
+  if (S > max_pages) S = max_pages;
+  if (S < 1) S = 1;
+  if (S > 256) S = 256;
+  return (int)S;
+}
+
+int kernel_kind(const palu_config* c) {
+  if (check_config(c) != PALU_OK) return 0;
+  if (palu::tc_decode_supported(c)) return 2;
+  return 1;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* palu_status_string(palu_status s) {
+  switch (s) {
+    case PALU_OK: return "ok";
+    case PALU_ERR_INVALID_ARG: return "invalid argument";
+    case PALU_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case PALU_ERR_ALIGNMENT: return "pointer or row not 16-byte aligned";
+    case PALU_ERR_WORKSPACE: return "workspace missing or too small";
+    case PALU_ERR_CUDA: return "CUDA error";
+    case PALU_ERR_DEVICE_TIMEOUT: return "a kernel's bounded wait timed out";
+    case PALU_ERR_DEVICE_BOUNDS: return "a kernel found an index out of range";
+  }
+  return "unknown status";
+}
+
+const char* palu_last_cuda_error(void) { return g_cuda_err; }
+
+int palu_decode_kernel_kind(const palu_config* cfg) { return kernel_kind(cfg); }
+
+uint64_t palu_kernel_launches(void) { return palu::g_launches.load(std::memory_order_relaxed); }
+
+palu_status palu_cache_strides(const palu_config* cfg, size_t* k_page_bytes, size_t* v_page_bytes,
+                               size_t* k_scale_page_bytes, size_t* v_scale_page_bytes) {
+  palu_status s = check_config(cfg);
+  if (s != PALU_OK) return s;
+  const int G = cfg->num_heads / cfg->group_size;
+  const size_t per = (size_t)G * cfg->page_size;
+  if (k_page_bytes) *k_page_bytes = per * palu::latent_row_bytes(cfg->latent_dtype, cfg->rank_k);
+  if (v_page_bytes) *v_page_bytes = per * palu::latent_row_bytes(cfg->latent_dtype, cfg->rank_v);
+  if (k_scale_page_bytes) *k_scale_page_bytes = per * palu::scale_row_bytes(cfg->latent_dtype, cfg->rank_k);
+  if (v_scale_page_bytes) *v_scale_page_bytes = per * palu::scale_row_bytes(cfg->latent_dtype, cfg->rank_v);
+  return PALU_OK;
+}
+
+palu_status palu_compress_workspace_size(const palu_config* cfg, int n_tokens, int d_model,
+                                         size_t* bytes) {
+  palu_status s = check_config(cfg);
+  if (s != PALU_OK) return s;
+  if (bytes == nullptr || n_tokens < 0 || d_model <= 0) return PALU_ERR_INVALID_ARG;
+  *bytes = kStatusBytes + palu::tc_compress_scratch_bytes(cfg, n_tokens, d_model);
+  return PALU_OK;
+}
+
+palu_status palu_compress_append(const palu_config* cfg, int n_tokens, int d_model, const void* x,
+                                 const void* A_k, const void* A_v, const int32_t* slot_mapping,
+                                 const int32_t* positions, void* zk_pool, void* zv_pool,
+                                 void* zk_scales, void* zv_scales, int32_t* pos_pool, int num_pages,
+                                 void* workspace, size_t workspace_bytes, palu_stream_t stream) {
+  palu_status s = check_config(cfg);
+  if (s != PALU_OK) return s;
+  if (n_tokens < 0 || d_model <= 0 || num_pages < 0) return PALU_ERR_INVALID_ARG;
+  if (d_model % 64 != 0) return PALU_ERR_UNSUPPORTED;
+  size_t need = 0;
+  palu_compress_workspace_size(cfg, n_tokens, d_model, &need);
+  if (workspace == nullptr || workspace_bytes < need) return PALU_ERR_WORKSPACE;
+  if (n_tokens == 0) return PALU_OK;
+  if (!x || !A_k || !A_v || !slot_mapping || !zk_pool || !zv_pool) return PALU_ERR_INVALID_ARG;
+  const bool int4 = cfg->latent_dtype == PALU_INT4;
+  if (int4 && (!zk_scales || !zv_scales)) return PALU_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(A_k) || !aligned16(A_v) || !aligned16(zk_pool) ||
+      !aligned16(zv_pool) || (int4 && (!aligned16(zk_scales) || !aligned16(zv_scales))) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return PALU_ERR_ALIGNMENT;
+
+  palu::CompressArgs a{};
+  a.n = n_tokens;
+  a.d_model = d_model;
+  a.G = cfg->num_heads / cfg->group_size;
+  a.r_k = cfg->rank_k;
+  a.r_v = cfg->rank_v;
+  a.P = cfg->page_size;
+  a.num_pages = num_pages;
+  a.act = cfg->act_dtype;
+  a.lat = cfg->latent_dtype;
+  a.x = x;
+  a.Ak = A_k;
+  a.Av = A_v;
+  a.slots = slot_mapping;
+  a.positions = positions;
+  a.zk = zk_pool;
+  a.zv = zv_pool;
+  a.zks = zk_scales;
+  a.zvs = zv_scales;
+  a.pos_pool = pos_pool;
+  a.status = workspace;
+  a.scratch = reinterpret_cast<float*>(static_cast<char*>(workspace) + kStatusBytes);
+  a.scratch_bytes = workspace_bytes - kStatusBytes;
+  a.k_row = palu::latent_row_bytes(a.lat, a.r_k);
+  a.v_row = palu::latent_row_bytes(a.lat, a.r_v);
+  a.ks_row = palu::scale_row_bytes(a.lat, a.r_k);
+  a.vs_row = palu::scale_row_bytes(a.lat, a.r_v);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (palu::tc_compress_supported(cfg, n_tokens, d_model))
+    e = palu::launch_compress_tc(a, st);
+  else
+    e = palu::launch_compress_simt(a, st);
+  return cuda_status(e);
+}
+
+palu_status palu_decode_num_splits(const palu_config* cfg, int batch, int max_pages, int* num_splits) {
+  palu_status s = check_config(cfg);
+  if (s != PALU_OK) return s;
+  if (num_splits == nullptr || batch < 0 || max_pages <= 0) return PALU_ERR_INVALID_ARG;
+  *num_splits = auto_splits(cfg, batch, max_pages, kernel_kind(cfg));
+  return PALU_OK;
+}
+
+palu_status palu_decode_workspace_size(const palu_config* cfg, int batch, int max_pages,
+                                       int num_splits, size_t* bytes) {
+  palu_status s = check_config(cfg);
+  if (s != PALU_OK) return s;
+  if (bytes == nullptr || batch < 0 || max_pages <= 0 || num_splits < 0) return PALU_ERR_INVALID_ARG;
+  const int S = num_splits == 0 ? auto_splits(cfg, batch, max_pages, kernel_kind(cfg)) : num_splits;
+  const size_t part = (size_t)batch * cfg->num_heads * S * (cfg->rank_v + 2) * sizeof(float);
+  *bytes = kStatusBytes + align256(part);
+  return PALU_OK;
+}
+
+palu_status palu_decode_attn(const palu_config* cfg, int batch, const void* q, const int32_t* q_pos,
+                             const void* zk_pool, const void* zv_pool, const void* zk_scales,
+                             const void* zv_scales, const int32_t* pos_pool,
+                             const int32_t* page_table, int max_pages, const int32_t* seq_lens,
+                             int num_pages, const void* B_k, const void* B_v, void* out, float* lse,
+                             void* workspace, size_t workspace_bytes, int num_splits,
+                             palu_stream_t stream) {
+  palu_status s = check_config(cfg);
+  if (s != PALU_OK) return s;
+  if (batch < 0 || max_pages <= 0 || num_pages < 0 || num_splits < 0) return PALU_ERR_INVALID_ARG;
+  const int kind = kernel_kind(cfg);
+  const int S = num_splits == 0 ? auto_splits(cfg, batch, max_pages, kind) : num_splits;
+  if (S > max_pages) return PALU_ERR_INVALID_ARG;
+  size_t need = 0;
+  palu_decode_workspace_size(cfg, batch, max_pages, S, &need);
+  if (workspace == nullptr || workspace_bytes < need) return PALU_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return PALU_ERR_ALIGNMENT;
+  if (batch == 0) return PALU_OK;
+  if (!q || !q_pos || !zk_pool || !zv_pool || !page_table || !seq_lens || !B_k || !B_v || !out)
+    return PALU_ERR_INVALID_ARG;
+  const bool int4 = cfg->latent_dtype == PALU_INT4;
+  if (int4 && (!zk_scales || !zv_scales)) return PALU_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(zk_pool) || !aligned16(zv_pool) || !aligned16(B_k) ||
+      !aligned16(B_v) || (int4 && (!aligned16(zk_scales) || !aligned16(zv_scales))))
+    return PALU_ERR_ALIGNMENT;
+
+  palu::DecodeArgs a{};
+  a.H = cfg->num_heads;
+  a.d_h = cfg->head_dim;
+  a.gs = cfg->group_size;
+  a.G = cfg->num_heads / cfg->group_size;
+  a.W = cfg->group_size * cfg->head_dim;
+  a.r_k = cfg->rank_k;
+  a.r_v = cfg->rank_v;
+  a.P = cfg->page_size;
+  a.batch = batch;
+  a.max_pages = max_pages;
+  a.num_pages = num_pages;
+  a.S = S;
+  a.act = cfg->act_dtype;
+  a.lat = cfg->latent_dtype;
+  a.rope = cfg->rope_base != 0.f;
+  a.sm_scale = (float)(1.0 / sqrt((double)cfg->head_dim));
+  a.q = q;
+  a.q_pos = q_pos;
+  a.zk = zk_pool;
+  a.zv = zv_pool;
+  a.zks = zk_scales;
+  a.zvs = zv_scales;
+  a.pos_pool = pos_pool;
+  a.page_table = page_table;
+  a.seq_lens = seq_lens;
+  a.Bk = B_k;
+  a.Bv = B_v;
+  a.out = out;
+  a.lse = lse;
+  a.status = workspace;
+  a.part = reinterpret_cast<float*>(static_cast<char*>(workspace) + kStatusBytes);
+  a.k_row = palu::latent_row_bytes(a.lat, a.r_k);
+  a.v_row = palu::latent_row_bytes(a.lat, a.r_v);
+  a.ks_row = palu::scale_row_bytes(a.lat, a.r_k);
+  a.vs_row = palu::scale_row_bytes(a.lat, a.r_v);
+  fill_omega(cfg, a.omega);
+
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = (kind == 2) ? palu::launch_decode_tc(a, st) : palu::launch_decode_simt(a, st);
+  if (e != cudaSuccess) return cuda_status(e);
+  return cuda_status(palu::launch_combine(a, st));
+}
+
+palu_status palu_get_device_status(void* workspace, palu_stream_t stream, int32_t* detail) {
+  if (workspace == nullptr) return PALU_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  palu::DevStatus host{};
+  cudaError_t e = cudaMemcpyAsync(&host, workspace, 8, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(workspace, 0, 8, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_status(e);
+  if (detail) *detail = host.detail;
+  if (host.code == PALU_ERR_DEVICE_TIMEOUT) return PALU_ERR_DEVICE_TIMEOUT;
+  if (host.code != 0) return PALU_ERR_DEVICE_BOUNDS;
+  return PALU_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,84 @@
+// Internal interface between the C-ABI layer (palu_abi.cu) and the kernel
+// launchers.  Host-side only; not part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/palu.h"
+
+namespace palu {
+
+constexpr int kMaxHalfDim = 64;  // head_dim <= 128
+
+// Everything a decode launch needs, already validated.
+struct DecodeArgs {
+  int H, d_h, gs, G, W, r_k, r_v, P;
+  int batch, max_pages, num_pages, S;
+  int act, lat;        // palu_dtype values
+  int rope;            // 0: RoPE off
+  float sm_scale;      // 1/sqrt(d_h)
+  const void* q;
+  const int32_t* q_pos;
+  const void* zk;
+  const void* zv;
+  const void* zks;
+  const void* zvs;
+  const int32_t* pos_pool;
+  const int32_t* page_table;
+  const int32_t* seq_lens;
+  const void* Bk;
+  const void* Bv;
+  void* out;
+  float* lse;
+  float* part;         // [batch][H][S][r_v + 2] float32
+  void* status;        // DevStatus*
+  long long k_row, v_row, ks_row, vs_row;  // bytes per latent / scale row
+  uint64_t omega[kMaxHalfDim];             // RoPE frequencies as 64-bit fixed-point turns
+};
+
+struct CompressArgs {
+  int n, d_model, G, r_k, r_v, P, num_pages;
+  int act, lat;
+  const void* x;
+  const void* Ak;
+  const void* Av;
+  const int32_t* slots;
+  const int32_t* positions;
+  void* zk;
+  void* zv;
+  void* zks;
+  void* zvs;
+  int32_t* pos_pool;
+  void* status;
+  float* scratch;  // workspace past the status header
+  size_t scratch_bytes;
+  long long k_row, v_row, ks_row, vs_row;
+};
+
+// CUDA-core kernels (any supported dtype; the only path for float32).
+cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t st);
+cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t st);
+cudaError_t launch_compress_simt(const CompressArgs& a, cudaStream_t st);
+
+// Counts kernel launches (palu_kernel_launches); call once per launch.
+void count_launch(int n = 1);
+
+// Row bytes of the pools for a config.
+inline long long latent_row_bytes(int lat, int r) {
+  switch (lat) {
+    case PALU_F32: return 4LL * r;
+    case PALU_F16:
+    case PALU_BF16: return 2LL * r;
+    case PALU_INT4: return r / 2;
+  }
+  return 0;
+}
+inline long long scale_row_bytes(int lat, int r) {
+  if (lat != PALU_INT4) return 0;
+  long long b = 2LL * (r / 32);
+  return (b + 15) / 16 * 16;
+}
+
+}  // namespace palu

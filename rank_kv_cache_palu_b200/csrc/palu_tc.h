@@ -1,0 +1,21 @@
+// Host-side interface of the tcgen05/TMA (sm_100a) kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "palu_internal.h"
+
+namespace palu {
+
+// Decode: shapes the tensor-core split kernel takes.
+bool tc_decode_supported(const palu_config* c);
+// Head blocks per group the split kernel's grid uses (heads per CTA = 2).
+int tc_head_blocks(const palu_config* c);
+cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st);
+
+// Compress: shapes the tensor-core GEMM takes, and the scratch it needs.
+bool tc_compress_supported(const palu_config* c, int n_tokens, int d_model);
+size_t tc_compress_scratch_bytes(const palu_config* c, int n_tokens, int d_model);
+cudaError_t launch_compress_tc(const CompressArgs& a, cudaStream_t st);
+
+}  // namespace palu

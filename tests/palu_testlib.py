@@ -1,0 +1,185 @@
+"""Test infrastructure shared by the parity tests: build seeded decode cases,
+lay logical latents out in the paged pool, run the oracle, compare.
+
+Nothing here computes the method: the oracle does that, from the same host
+tensors the GPU receives.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+from oracle import palu_oracle as O
+from rank_kv_cache_palu_b200 import api as P
+from rank_kv_cache_palu_b200.synth import TORCH_DTYPE, Workload, normal, normal_tensor, page_permutation
+
+TOL = {"f32": 1e-4, "f16": 1e-2, "bf16": 1e-2}
+
+
+def rel_err(gpu: np.ndarray, ref: np.ndarray) -> float:
+    """max |gpu - ref| / max |ref| over the whole tensor (the stated parity metric)."""
+    den = float(np.max(np.abs(ref)))
+    return float(np.max(np.abs(gpu - ref))) / (den if den > 0 else 1.0)
+
+
+@dataclass
+class DecodeCase:
+    w: Workload
+    seq_lens: list[int]
+    q: torch.Tensor              # [b, H, d_h] act dtype (CPU)
+    q_pos: np.ndarray            # [b]
+    B_k: torch.Tensor            # [G, r_k, W]
+    B_v: torch.Tensor            # [G, r_v, W]
+    zk: list                     # per b: storage tensor [G, T, r_k] (int4: packed uint8 [G, T, r/2])
+    zv: list
+    zks: list | None             # int4: per b fp16 scales [G, T, r/32]
+    zvs: list | None
+    pos: list                    # per b: int32 positions [T] or None (index)
+    page_table: np.ndarray       # [b, max_pages]
+    num_pages: int
+
+    @property
+    def cfg(self):
+        w = self.w
+        return P.make_config(w.num_heads, w.head_dim, w.group_size, w.rank_k, w.rank_v,
+                             w.page_size, w.rope_base, w.act_dtype, w.latent_dtype)
+
+    def oracle_latents(self, b: int):
+        """Float64 latents [G, T, r] as the decode step sees them (int4: dequantised)."""
+        w = self.w
+        if w.latent_dtype == "int4":
+            zk = O.dequantize_int4(self.zk[b].numpy(), self.zks[b].numpy(), w.act_dtype)
+            zv = O.dequantize_int4(self.zv[b].numpy(), self.zvs[b].numpy(), w.act_dtype)
+            return zk, zv
+        return self.zk[b].to(torch.float64).numpy(), self.zv[b].to(torch.float64).numpy()
+
+    def positions(self, b: int) -> np.ndarray:
+        return np.arange(self.seq_lens[b]) if self.pos[b] is None else self.pos[b].astype(np.int64)
+
+
+def make_decode_case(w: Workload, seq_lens, seed=None, explicit_positions=False, q_scale=1.0,
+                     extra_pages=3, q_pos=None) -> DecodeCase:
+    seed = w.seed if seed is None else seed
+    G, W, d_h = w.groups, w.width, w.head_dim
+    b = len(seq_lens)
+    Pz = w.page_size
+    max_pages = max(1, max((t + Pz - 1) // Pz for t in seq_lens))
+    total_pages = sum((t + Pz - 1) // Pz for t in seq_lens) + extra_pages
+    perm = page_permutation(seed, total_pages)
+    page_table = np.full((b, max_pages), -1, np.int32)
+    k = 0
+    for i, t in enumerate(seq_lens):
+        for p in range((t + Pz - 1) // Pz):
+            page_table[i, p] = perm[k]
+            k += 1
+    page_table[page_table < 0] = perm[-1]           # unused entries: a valid but unread page
+    q = normal_tensor(seed, "q", (b, w.num_heads, d_h), w.act_dtype, q_scale)
+    B_k = normal_tensor(seed, "B_k", (G, w.rank_k, W), w.act_dtype, 1 / math.sqrt(w.rank_k))
+    B_v = normal_tensor(seed, "B_v", (G, w.rank_v, W), w.act_dtype, 1 / math.sqrt(w.rank_v))
+    zk, zv, zks, zvs, pos = [], [], [], [], []
+    for i, t in enumerate(seq_lens):
+        if w.latent_dtype == "int4":
+            for side, r, out_c, out_s in (("zk", w.rank_k, zk, zks), ("zv", w.rank_v, zv, zvs)):
+                lat = normal(seed, side, (G, t, r), unit=(i,))
+                packed, sc = O.quantize_int4(lat)
+                out_c.append(torch.from_numpy(packed))
+                out_s.append(torch.from_numpy(sc))
+        else:
+            zk.append(normal_tensor(seed, "zk", (G, t, w.rank_k), w.latent_dtype, unit=(i,)))
+            zv.append(normal_tensor(seed, "zv", (G, t, w.rank_v), w.latent_dtype, unit=(i,)))
+        if explicit_positions:
+            rng = np.random.default_rng([seed, i, 77])
+            pos.append(np.sort(rng.choice(max(4 * t, 1), size=t, replace=False)).astype(np.int32)
+                       if t > 0 else np.zeros(0, np.int32))
+        else:
+            pos.append(None)
+    if q_pos is None:
+        q_pos = np.array([(int(pp[-1]) + 1 if pp is not None and len(pp) else max(t - 1, 0))
+                          for pp, t in zip(pos, seq_lens)], np.int32)
+    return DecodeCase(w, list(seq_lens), q, np.asarray(q_pos, np.int32), B_k, B_v, zk, zv,
+                      zks if w.latent_dtype == "int4" else None,
+                      zvs if w.latent_dtype == "int4" else None, pos, page_table, total_pages)
+
+
+def _as_bytes(t: torch.Tensor) -> np.ndarray:
+    return t.contiguous().view(torch.uint8).numpy() if t.dtype != torch.uint8 else t.numpy()
+
+
+def build_pools(case: DecodeCase, device="cuda"):
+    """Scatter each sequence's logical latents into the paged pools (host side), upload."""
+    w = case.w
+    cfg = case.cfg
+    kb, vb, ksb, vsb = P.palu_cache_strides(cfg)
+    G, Pz = w.groups, w.page_size
+    npg = case.num_pages
+    pools = {}
+    for name, lst, page_bytes in (("zk", case.zk, kb), ("zv", case.zv, vb),
+                                  ("zks", case.zks, ksb), ("zvs", case.zvs, vsb)):
+        if not page_bytes:
+            pools[name] = None
+            continue
+        row = page_bytes // (G * Pz)
+        host = np.zeros((npg, G, Pz, row), np.uint8)
+        for i, t in enumerate(case.seq_lens):
+            if t == 0:
+                continue
+            data = _as_bytes(lst[i]).reshape(G, t, -1)
+            for p in range((t + Pz - 1) // Pz):
+                t0, t1 = p * Pz, min(t, (p + 1) * Pz)
+                host[case.page_table[i, p], :, : t1 - t0, : data.shape[2]] = data[:, t0:t1]
+        pools[name] = torch.from_numpy(host.reshape(-1)).to(device)
+    pos_pool = None
+    if any(pp is not None for pp in case.pos):
+        host = np.zeros((npg, Pz), np.int32)
+        for i, t in enumerate(case.seq_lens):
+            for p in range((t + Pz - 1) // Pz):
+                t0, t1 = p * Pz, min(t, (p + 1) * Pz)
+                src = case.pos[i] if case.pos[i] is not None else np.arange(t, dtype=np.int32)
+                host[case.page_table[i, p], : t1 - t0] = src[t0:t1]
+        pos_pool = torch.from_numpy(host.reshape(-1)).to(device)
+    pools["pos"] = pos_pool
+    return pools
+
+
+def run_gpu_decode(case: DecodeCase, num_splits=0, device="cuda", pools=None, check_status=True):
+    cfg = case.cfg
+    if pools is None:
+        pools = build_pools(case, device)
+    b = len(case.seq_lens)
+    w = case.w
+    dev = lambda t: t.to(device)
+    ws_bytes = P.palu_decode_workspace_size(cfg, b, case.page_table.shape[1], num_splits)
+    ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=device)
+    out = torch.empty((b, w.num_heads, w.head_dim), dtype=TORCH_DTYPE[w.act_dtype], device=device)
+    lse = torch.empty((b, w.num_heads), dtype=torch.float32, device=device)
+    P.palu_decode_attn(cfg, dev(case.q), dev(torch.from_numpy(case.q_pos)), pools["zk"], pools["zv"],
+                       pools["zks"], pools["zvs"], pools["pos"],
+                       dev(torch.from_numpy(case.page_table)),
+                       dev(torch.tensor(case.seq_lens, dtype=torch.int32)), case.num_pages,
+                       dev(case.B_k), dev(case.B_v), out, lse, ws, num_splits)
+    torch.cuda.synchronize()
+    if check_status:
+        st, detail = P.palu_get_device_status(ws)
+        assert st == 0, f"device status {st} detail {detail}"
+    return out.to(torch.float64).cpu().numpy(), lse.to(torch.float64).cpu().numpy()
+
+
+def oracle_decode(case: DecodeCase, b: int, heads=None):
+    """Oracle out [len(heads), d_h], lse for sequence b."""
+    w = case.w
+    zk, zv = case.oracle_latents(b)
+    heads = range(w.num_heads) if heads is None else heads
+    q = case.q[b].to(torch.float64).numpy()
+    Bk = case.B_k.to(torch.float64).numpy()
+    Bv = case.B_v.to(torch.float64).numpy()
+    pos = case.positions(b)
+    outs, lses = [], []
+    for h in heads:
+        o, l = O.decode_attention_head(h, q, int(case.q_pos[b]), zk, zv, pos, Bk, Bv,
+                                       w.group_size, w.rope_base)
+        outs.append(o)
+        lses.append(l)
+    return np.array(outs), np.array(lses)

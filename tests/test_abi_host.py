@@ -1,0 +1,137 @@
+"""The C-ABI library loads, exports every symbol the header declares, and its
+host-side argument checks return the documented statuses.  CPU only: none of
+these calls reaches a kernel launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from rank_kv_cache_palu_b200 import api as P
+from rank_kv_cache_palu_b200._lib import LIB_PATH, SIGNATURES, PaluConfig, load
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "palu.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(palu_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(LIB_PATH)
+    names = declared_symbols()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in palu.h but not exported"
+        assert n in SIGNATURES, f"{n} has no binding signature"
+
+
+def cfg(**kw):
+    base = dict(num_heads=32, head_dim=128, group_size=4, rank_k=256, rank_v=128, page_size=128,
+                rope_base=10000.0, act_dtype="bf16", latent_dtype=None)
+    base.update(kw)
+    return P.make_config(**base)
+
+
+def status_of(fn, *args):
+    return int(fn(*args))
+
+
+def test_cache_strides():
+    assert P.palu_cache_strides(cfg()) == (8 * 128 * 512, 8 * 128 * 256, 0, 0)
+    k, v, ks, vs = P.palu_cache_strides(cfg(act_dtype="f16", latent_dtype="int4", rank_v=256))
+    assert (k, v) == (8 * 128 * 128, 8 * 128 * 128)
+    assert ks == vs == 8 * 128 * 16            # 8 fp16 scales per 256-entry row, 16-byte padded
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(num_heads=30), 1),                  # not a multiple of the group size
+    (dict(head_dim=0), 1),
+    (dict(head_dim=127), 1),                  # odd head_dim
+    (dict(rope_base=-1.0), 1),
+    (dict(act_dtype="f32", latent_dtype="bf16"), 2),
+    (dict(act_dtype="f32", latent_dtype="int4"), 2),
+    (dict(head_dim=256), 2),
+    (dict(rank_k=100), 3),                    # 16-byte rows need r % 8 == 0
+    (dict(act_dtype="f16", latent_dtype="int4", rank_k=48), 3),
+])
+def test_config_validation(bad, code):
+    lib = load()
+    k = ctypes.c_size_t()
+    c = cfg(**bad)
+    assert lib.palu_cache_strides(ctypes.byref(c), ctypes.byref(k), None, None, None) == code
+
+
+def test_workspace_size_and_splits():
+    c = cfg()
+    S = P.palu_decode_num_splits(c, 16, 128)
+    assert 1 <= S <= 128
+    ws = P.palu_decode_workspace_size(c, 16, 128, S)
+    assert ws >= 256 + 16 * 32 * S * (128 + 2) * 4
+    assert ws % 256 == 0
+    assert P.palu_decode_num_splits(c, 1, 1) == 1
+    assert P.palu_compress_workspace_size(c, 32, 4096) >= 256
+
+
+def test_decode_rejects_missing_workspace_before_launch():
+    lib = load()
+    c = cfg()
+    st = lib.palu_decode_attn(ctypes.byref(c), 1, None, None, None, None, None, None, None, None, 4,
+                              None, 8, None, None, None, None, None, 0, 0, None)
+    assert st == 4  # PALU_ERR_WORKSPACE
+
+
+def test_decode_rejects_too_many_splits():
+    lib = load()
+    c = cfg()
+    st = lib.palu_decode_attn(ctypes.byref(c), 1, None, None, None, None, None, None, None, None, 4,
+                              None, 8, None, None, None, None, None, 1 << 20, 5, None)
+    assert st == 1  # more splits than pages
+
+
+def test_decode_rejects_null_and_misaligned_pointers():
+    lib = load()
+    c = cfg()
+    ws = ctypes.create_string_buffer((1 << 20) + 512)
+    base = (ctypes.addressof(ws) + 255) // 256 * 256
+    st = lib.palu_decode_attn(ctypes.byref(c), 1, None, None, None, None, None, None, None, None, 4,
+                              None, 8, None, None, None, None, base, 1 << 20, 1, None)
+    assert st == 1  # NULL q etc.
+    p = base + 8   # not 16-byte aligned
+    st = lib.palu_decode_attn(ctypes.byref(c), 1, p, p, p, p, None, None, None, p, 4, p, 8, p, p,
+                              p, None, base, 1 << 20, 1, None)
+    assert st == 3  # PALU_ERR_ALIGNMENT
+
+
+def test_compress_rejects_bad_arguments():
+    lib = load()
+    c = cfg()
+    ws = ctypes.create_string_buffer(4096)
+    base = (ctypes.addressof(ws) + 255) // 256 * 256
+    assert lib.palu_compress_append(ctypes.byref(c), 4, 100, None, None, None, None, None, None, None,
+                                    None, None, None, 1, base, 1024, None) == 2   # d_model % 64
+    assert lib.palu_compress_append(ctypes.byref(c), 4, 128, None, None, None, None, None, None, None,
+                                    None, None, None, 1, None, 0, None) == 4      # no workspace
+    assert lib.palu_compress_append(ctypes.byref(c), 0, 128, None, None, None, None, None, None, None,
+                                    None, None, None, 1, base, 1024, None) == 0   # nothing to do
+    assert lib.palu_compress_append(ctypes.byref(c), 4, 128, None, None, None, None, None, None, None,
+                                    None, None, None, 1, base, 1024, None) == 1   # NULL inputs
+
+
+def test_status_strings():
+    lib = load()
+    for s in range(8):
+        assert lib.palu_status_string(s)
+    assert P.palu_kernel_launches() >= 0
+
+
+def test_product_path_does_not_import_oracle():
+    import rank_kv_cache_palu_b200
+    pkg = os.path.dirname(rank_kv_cache_palu_b200.__file__)
+    for root, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(root, f), encoding="utf-8").read()
+                assert "import oracle" not in text and "from oracle" not in text, f

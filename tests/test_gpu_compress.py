@@ -1,0 +1,156 @@
+"""GPU parity of palu_compress_append (z = x·A into the paged cache) against the oracle."""
+import dataclasses
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import palu_oracle as O
+from rank_kv_cache_palu_b200 import api as P
+from rank_kv_cache_palu_b200.synth import TORCH_DTYPE, WORKLOADS, normal_tensor
+
+pytestmark = pytest.mark.gpu
+
+SENTINEL = 0xAB
+
+
+def run_compress(w, x, A_k, A_v, slots, positions, num_pages):
+    cfg = P.make_config(w.num_heads, w.head_dim, w.group_size, w.rank_k, w.rank_v, w.page_size,
+                        w.rope_base, w.act_dtype, w.latent_dtype)
+    cache = P.LatentCache.allocate(cfg, num_pages, with_positions=True, fill=SENTINEL)
+    n, d_model = x.shape
+    ws = torch.zeros(P.palu_compress_workspace_size(cfg, n, d_model), dtype=torch.uint8, device="cuda")
+    P.palu_compress_append(cfg, x.cuda(), A_k.cuda(), A_v.cuda(), torch.from_numpy(slots).cuda(),
+                           None if positions is None else torch.from_numpy(positions).cuda(),
+                           cache.zk, cache.zv, cache.zks, cache.zvs, cache.pos, num_pages, ws)
+    torch.cuda.synchronize()
+    st, detail = P.palu_get_device_status(ws)
+    return cache, st, detail
+
+
+def gather_rows(pool: torch.Tensor, w, slots, r, row_bytes):
+    """Bytes of each token's row per group: [n, G, row_bytes] (slot < 0 rows are zero)."""
+    host = pool.cpu().numpy().reshape(-1, w.groups, w.page_size, row_bytes)
+    out = np.zeros((len(slots), w.groups, row_bytes), np.uint8)
+    for i, s in enumerate(slots):
+        if s >= 0:
+            out[i] = host[s // w.page_size, :, s % w.page_size]
+    return out
+
+
+def as_values(rows: np.ndarray, dtype: str) -> np.ndarray:
+    t = torch.from_numpy(rows.copy()).view(TORCH_DTYPE[dtype])
+    return t.to(torch.float64).numpy()
+
+
+def make_slots(n, num_pages, page_size, seed, holes=True):
+    rng = np.random.default_rng(seed)
+    slots = rng.choice(num_pages * page_size, size=n, replace=False).astype(np.int32)
+    if holes and n > 4:
+        slots[rng.choice(n, size=max(1, n // 16), replace=False)] = -1
+    return slots
+
+
+@pytest.mark.parametrize("dt", ["f32", "f16", "bf16"])
+@pytest.mark.parametrize("n", [1, 37, 200])
+def test_compress_small(dt, n):
+    w = dataclasses.replace(WORKLOADS["tiny_f32"], act_dtype=dt, latent_dtype=dt, rank_k=64,
+                            rank_v=32, d_model=192)
+    x = normal_tensor(7, "x", (n, w.d_model), dt)
+    A_k = normal_tensor(7, "A_k", (w.d_model, w.groups * w.rank_k), dt, 1 / math.sqrt(w.d_model))
+    A_v = normal_tensor(7, "A_v", (w.d_model, w.groups * w.rank_v), dt, 1 / math.sqrt(w.d_model))
+    num_pages = (n + w.page_size - 1) // w.page_size + 2
+    slots = make_slots(n, num_pages, w.page_size, seed=n)
+    positions = (np.arange(n) * 3 + 5).astype(np.int32)
+    cache, st, _ = run_compress(w, x, A_k, A_v, slots, positions, num_pages)
+    assert st == 0
+    esz = 4 if dt == "f32" else 2
+    tol = {"f32": 1e-5, "f16": 2 ** -10, "bf16": 2 ** -7}[dt]
+    for pool, A, r in ((cache.zk, A_k, w.rank_k), (cache.zv, A_v, w.rank_v)):
+        got = as_values(gather_rows(pool, w, slots, r, r * esz), dt)       # [n, G, r]
+        ref = O.compress(x.to(torch.float64).numpy(), A.to(torch.float64).numpy(), dt)
+        ref = ref.reshape(n, w.groups, r)
+        keep = slots >= 0
+        err = np.abs(got[keep] - ref[keep])
+        # within one rounding step of the dtype (float32 accumulation may cross a tie)
+        assert np.all(err <= tol * np.abs(ref[keep]) + 1e-6 * np.max(np.abs(ref))), float(err.max())
+    # skipped rows untouched, positions written
+    pos = cache.pos.cpu().numpy()
+    for i, s in enumerate(slots):
+        if s >= 0:
+            assert pos[s] == positions[i]
+
+
+def exact_inputs(w, n, seed):
+    """x on a dyadic grid and A a 0/1 column-selection matrix: x·A is exact in float32."""
+    rng = np.random.default_rng(seed)
+    x = (rng.integers(-24, 25, size=(n, w.d_model)) / 8.0).astype(np.float32)
+    def sel(ncol):
+        A = np.zeros((w.d_model, ncol), np.float32)
+        A[rng.integers(0, w.d_model, size=ncol), np.arange(ncol)] = 1.0
+        return A
+    t = TORCH_DTYPE[w.act_dtype]
+    return (torch.from_numpy(x).to(t), torch.from_numpy(sel(w.groups * w.rank_k)).to(t),
+            torch.from_numpy(sel(w.groups * w.rank_v)).to(t))
+
+
+@pytest.mark.parametrize("act", ["f16", "bf16"])
+def test_compress_int4_bit_exact(act):
+    # exactly representable latents: quantisation codes, bytes and scales match bit for bit
+    w = dataclasses.replace(WORKLOADS["tiny_f32"], act_dtype=act, latent_dtype="int4", rank_k=64,
+                            rank_v=96, d_model=256)
+    n = 150
+    x, A_k, A_v = exact_inputs(w, n, 3)
+    num_pages = 4
+    slots = make_slots(n, num_pages, w.page_size, seed=5)
+    cache, st, _ = run_compress(w, x, A_k, A_v, slots, None, num_pages)
+    assert st == 0
+    kb, vb, ksb, vsb = P.palu_cache_strides(P.make_config(
+        w.num_heads, w.head_dim, w.group_size, w.rank_k, w.rank_v, w.page_size, 10000.0, act, "int4"))
+    for pool, spool, A, r in ((cache.zk, cache.zks, A_k, w.rank_k), (cache.zv, cache.zvs, A_v, w.rank_v)):
+        z = O.compress(x.to(torch.float64).numpy(), A.to(torch.float64).numpy(), "f32")
+        packed, sc = O.quantize_int4(z.reshape(n, w.groups, r).astype(np.float32))
+        srow = (2 * (r // 32) + 15) // 16 * 16
+        got = gather_rows(pool, w, slots, r, r // 2)
+        got_s = gather_rows(spool, w, slots, r, srow)[..., : 2 * (r // 32)].copy().view(np.float16)
+        keep = slots >= 0
+        np.testing.assert_array_equal(got[keep], packed[keep])
+        np.testing.assert_array_equal(got_s[keep], sc[keep])
+
+
+def test_compress_int4_general():
+    # N(0,1) inputs: codes may differ from the oracle's only where float32
+    # accumulation order moves a value across a rounding boundary
+    w = dataclasses.replace(WORKLOADS["tiny_f32"], act_dtype="f16", latent_dtype="int4", rank_k=64,
+                            rank_v=64, d_model=256)
+    n = 100
+    x = normal_tensor(11, "x", (n, w.d_model), "f16")
+    A_k = normal_tensor(11, "A_k", (w.d_model, w.groups * w.rank_k), "f16", 1 / 16)
+    A_v = normal_tensor(11, "A_v", (w.d_model, w.groups * w.rank_v), "f16", 1 / 16)
+    slots = make_slots(n, 2, w.page_size, seed=9, holes=False)
+    cache, st, _ = run_compress(w, x, A_k, A_v, slots, None, 2)
+    assert st == 0
+    for pool, spool, A, r in ((cache.zk, cache.zks, A_k, w.rank_k), (cache.zv, cache.zvs, A_v, w.rank_v)):
+        z = O.compress(x.to(torch.float64).numpy(), A.to(torch.float64).numpy(), None).reshape(n, w.groups, r)
+        srow = 16
+        got = gather_rows(pool, w, slots, r, r // 2)
+        got_s = gather_rows(spool, w, slots, r, srow)[..., : 2 * (r // 32)].copy().view(np.float16)
+        deq = O.dequantize_int4(got, got_s, "f16")
+        s_full = np.repeat(got_s.astype(np.float64), 32, axis=-1)
+        assert np.all(np.abs(deq - z) <= 0.5 * s_full * 1.001 + 1e-3 * s_full + 1e-6)
+        _, sc_ref = O.quantize_int4(z.astype(np.float32))
+        assert np.all(np.abs(got_s.astype(np.float64) - sc_ref.astype(np.float64))
+                      <= 2 ** -10 * np.abs(sc_ref.astype(np.float64)) + 1e-7)
+
+
+def test_compress_bad_slot_reports_bounds():
+    w = dataclasses.replace(WORKLOADS["tiny_f32"], d_model=128)
+    n = 10
+    x = normal_tensor(1, "x", (n, w.d_model), "f32")
+    A_k = normal_tensor(1, "A_k", (w.d_model, w.groups * w.rank_k), "f32", 0.1)
+    A_v = normal_tensor(1, "A_v", (w.d_model, w.groups * w.rank_v), "f32", 0.1)
+    slots = np.arange(n, dtype=np.int32)
+    slots[3] = 10 ** 6
+    _, st, _ = run_compress(w, x, A_k, A_v, slots, None, 1)
+    assert st == 7

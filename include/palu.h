@@ -31,13 +31,21 @@
  *   - No exception, abort or trap crosses this ABI.
  *
  * Latent-cache layout (the "cache manager" side; paged by sequence):
- *   K pool  [num_pages][G][page_size][row_k]    row_k = rank_k elements of the
- *   V pool  [num_pages][G][page_size][row_v]    latent dtype (int4: rank/2 bytes)
+ *   K pool  [num_pages][G] blocks of page_size tokens × row_k bytes
+ *   V pool  [num_pages][G] blocks of page_size tokens × row_v bytes
+ *           row_k = rank_k elements of the latent dtype (int4: rank_k/2 bytes);
+ *           row_k and row_v must be multiples of 128 bytes.
+ *   Inside one (page, group) block the bytes are column-blocked and swizzled:
+ *   byte o of token t's latent row lives at
+ *       (o / 128)·(page_size·128) + t·128 + (((o % 128) / 16) XOR (t % 8))·16 + o % 16
+ *   i.e. 128-byte column blocks of all page_size tokens, the 16-byte units of
+ *   each token's 128 bytes permuted by t mod 8.  That is the 128-byte-swizzled
+ *   shared-memory image the tensor-core MMAs consume, so every 128-byte column
+ *   block of a page reaches shared memory as one contiguous bulk copy.
  *   int4 scale pools [num_pages][G][page_size][srow]   srow = 16-byte padded
- *           rank/32 fp16 scales (one per 32 consecutive latent entries)
+ *           rank/32 fp16 scales (one per 32 consecutive latent entries), token-major
  *   pos pool [num_pages][page_size] int32 (optional)
- *   A token lives at slot = page·page_size + offset.  Rows are token-major and
- *   16-byte aligned, so one page of one group is a 2-D tile a TMA box can move.
+ *   A token lives at slot = page·page_size + offset; page_size is a multiple of 8.
  */
 #ifndef PALU_H_
 #define PALU_H_
@@ -175,6 +183,22 @@ const char* palu_last_cuda_error(void);
 /* Which kernel family a decode call with this config would launch:
  * 0 = none (unsupported), 1 = CUDA-core kernels, 2 = tcgen05/TMA kernels. */
 int palu_decode_kernel_kind(const palu_config* cfg);
+
+/* Phase tracing of the tensor-core decode kernel, for performance analysis.
+ * After this call every palu_decode_attn launch of the tensor-core kernel
+ * records, per CTA and per tile (up to `tiles_per_cta`), the SM clock
+ * (clock64, relative to the CTA's start) at kPaluTraceEvents points:
+ *   0 MMA: slot free, key MMAs of the tile start   1 MMA: key MMAs issued
+ *   2 MMA: value MMAs of the previous tile issued  3 epilogue: tile keys ready
+ *   4 epilogue: scores done (both warpgroups)      5 epilogue: P written
+ *   6 z_k producer: first chunk of the tile issued 7 MMA: first chunk landed
+ * into `buffer` (device memory, int64 [cta][event][tile], CTA = linear block
+ * index); entries never reached stay as they were.  Pass NULL to stop.
+ * `bytes` must cover grid CTAs × 8 × tiles_per_cta × 8 bytes of the launches
+ * traced; launches whose grid does not fit are not traced.  Process-wide
+ * setting, not thread-safe with concurrent decode calls. */
+#define PALU_TRACE_EVENTS 8
+palu_status palu_debug_trace(void* buffer, size_t bytes, int tiles_per_cta);
 
 /* Number of CUDA kernels this library has launched in this process (all
  * entry points, all devices).  A monotone counter for instrumentation. */

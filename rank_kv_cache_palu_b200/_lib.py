@@ -51,6 +51,7 @@ SIGNATURES = {
     "palu_last_cuda_error": (ctypes.c_char_p, []),
     "palu_decode_kernel_kind": (c_int, [_CFG]),
     "palu_kernel_launches": (ctypes.c_uint64, []),
+    "palu_debug_trace": (c_int, [c_void_p, c_size_t, c_int]),
 }
 
 _lock = threading.Lock()

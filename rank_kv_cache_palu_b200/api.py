@@ -100,6 +100,15 @@ def palu_kernel_launches() -> int:
     return int(load().palu_kernel_launches())
 
 
+def palu_debug_trace(buffer, tiles_per_cta: int = 0) -> None:
+    """Record tensor-core decode phase timestamps into `buffer` (int64 CUDA tensor); None stops."""
+    if buffer is None:
+        _check(load().palu_debug_trace(None, 0, 0), "palu_debug_trace")
+    else:
+        _check(load().palu_debug_trace(_ptr(buffer), buffer.numel() * buffer.element_size(),
+                                       tiles_per_cta), "palu_debug_trace")
+
+
 def palu_compress_append(cfg: PaluConfig, x, A_k, A_v, slot_mapping, positions, zk_pool, zv_pool,
                          zk_scales, zv_scales, pos_pool, num_pages: int, workspace, stream=None):
     n, d_model = x.shape

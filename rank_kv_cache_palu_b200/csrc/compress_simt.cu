@@ -82,7 +82,9 @@ __global__ void __launch_bounds__(kThreads) compress_kernel(const CompressArgs a
             report(st, PALU_ERR_DEVICE_BOUNDS, 3000000 + gi);
           } else {
             const int g = gc / r, j0 = gc % r;
-            const long long prow = ((long long)(slot / a.P) * a.G + g) * a.P + slot % a.P;
+            const long long pgb = (long long)(slot / a.P) * a.G + g;   // (page, group) block
+            const int tok = slot % a.P;
+            const long long prow = pgb * a.P + tok;
             float amax = 0.f;
             for (int u = 0; u < 32; ++u) amax = fmaxf(amax, fabsf(ct[i][blk * 32 + u]));
             const __half s16 = __float2half_rn(__fdiv_rn(amax, 7.0f));
@@ -97,7 +99,8 @@ __global__ void __launch_bounds__(kThreads) compress_kernel(const CompressArgs a
               }
               words[u / 8] |= (uint32_t)(code & 0xF) << (4 * (u % 8));
             }
-            uint4* dst = reinterpret_cast<uint4*>(pool + prow * row_bytes + j0 / 2);
+            // 32 codes = one 16-byte unit of the swizzled page block
+            uint4* dst = reinterpret_cast<uint4*>(pool + pgb * a.P * row_bytes + swz_offset(tok, j0 / 2, a.P));
             *dst = make_uint4(words[0], words[1], words[2], words[3]);
             reinterpret_cast<__half*>(spool + prow * srow)[j0 / 32] = s16;
           }
@@ -121,8 +124,9 @@ __global__ void __launch_bounds__(kThreads) compress_kernel(const CompressArgs a
         const int gc = col0 + tx * 4 + v;
         if (gc >= N) continue;
         const int g = gc / r, j = gc % r;
-        const long long prow = ((long long)(slot / a.P) * a.G + g) * a.P + slot % a.P;
-        reinterpret_cast<TL*>(pool + prow * row_bytes)[j] = Dt<LAT>::from_f(ct[i][tx * 4 + v]);
+        const long long pgb = (long long)(slot / a.P) * a.G + g;   // (page, group) block
+        *reinterpret_cast<TL*>(pool + pgb * a.P * row_bytes + swz_offset(slot % a.P, (long long)j * sizeof(TL), a.P)) =
+            Dt<LAT>::from_f(ct[i][tx * 4 + v]);
       }
     }
   }

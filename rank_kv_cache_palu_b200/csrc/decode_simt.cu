@@ -111,8 +111,9 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const DecodeArgs a) {
         if (page < 0 || page >= a.num_pages) {
           report(st, PALU_ERR_DEVICE_BOUNDS, 2000000 + b);
         } else {
-          const size_t row = ((size_t)page * a.G + g) * a.P + t % a.P;
-          v = load_latent<LAT, ACT>(zk_base + row * a.k_row,
+          const size_t blk = (size_t)page * a.G + g;
+          const size_t row = blk * a.P + t % a.P;
+          v = load_latent<LAT, ACT>(zk_base + blk * a.P * a.k_row, t % a.P, a.P,
                                     LAT == PALU_INT4 ? zks_base + row * a.ks_row : nullptr, j);
         }
       }
@@ -125,8 +126,9 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const DecodeArgs a) {
         const int t = t0 + tt;
         const int page = ptab[t / a.P];
         if (page >= 0 && page < a.num_pages) {
-          const size_t row = ((size_t)page * a.G + g) * a.P + t % a.P;
-          v = load_latent<LAT, ACT>(zv_base + row * a.v_row,
+          const size_t blk = (size_t)page * a.G + g;
+          const size_t row = blk * a.P + t % a.P;
+          v = load_latent<LAT, ACT>(zv_base + blk * a.P * a.v_row, t % a.P, a.P,
                                     LAT == PALU_INT4 ? zvs_base + row * a.vs_row : nullptr, j);
         }
       }

@@ -11,11 +11,11 @@
 // pages, 128 tokens (one page) per tile:
 //   warp 0  TMA producer: B_k for the two heads once (MN-major, 128-byte
 //           swizzle, resident), then the z_k page in 64-wide K chunks.
-//   warp 6  TMA producer for z_v (its own ring, so neither stream waits on the other).
+//   warp 10 TMA producer for z_v (its own ring, so neither stream waits on the other).
 //   warp 1  MMA issuer: D[128 tok × 256] = z_k · B_k[:, 2 heads] into one of two
 //           TMEM slots (kind::f16, fp32 accumulate); then aᵀ[r_v × 16] =
 //           z_vᵀ · Pᵀ for the previous tile into the drained slot.
-//   warps 2-5 epilogue, one thread per token: tcgen05.ld the rebuilt keys,
+//   warps 2-9 epilogue, two warpgroups of one thread per token: tcgen05.ld the rebuilt keys,
 //           rotate them (RoPE at the token's position), score against the
 //           rotated query, online softmax (exp2), write P (bf16/fp16) for the
 //           value MMA, and fold each tile's aᵀ into running latent sums.
@@ -38,17 +38,20 @@ namespace {
 using namespace tc;
 
 constexpr int kTile = 128;         // tokens per tile = page size
-constexpr int kChunk = 64;         // K chunk of z_k (elements)
+constexpr int kChunk = 64;         // K chunk of z_k (elements) = one 128-byte column block of the page
 constexpr int kNKS = 3;            // z_k ring stages
+constexpr uint32_t kZkSwz = 2u;    // 128-byte swizzle
+constexpr uint32_t kZkSbo = 1024;  // bytes per 8-row swizzle atom
 constexpr int kNVS = 2;            // z_v ring stages
-constexpr int kThreads = 224;      // 7 warps
-constexpr int kZkBytes = kTile * kChunk * 2;   // 16 KB
+constexpr int kPrefetch = 3;       // pages pulled into L2 ahead of the TMA loads
+constexpr int kThreads = 384;      // 12 warps: producers + MMA (warps 0-3), two epilogue warpgroups
+constexpr int kZkBytes = kTile * kChunk * 2;   // bytes per z_k stage
 constexpr int kZvBytes = 64 * 128 * 2;         // 16 KB: 64 tokens × 128 latent entries
 constexpr int kPBytes = 16 * kTile * 2;        // 4 KB: 16 rows (heads, padded) × 128 tokens
 
 struct Smem {
   // offsets in bytes from a 1024-aligned base
-  uint32_t b, zk, zv, p, qr, omega, red, lred, bars, tmem_slot, abort, total;
+  uint32_t b, zk, zv, p, qr, psc, tb, omega, red, lred, bars, tmem_slot, abort, total;
 };
 
 __host__ __device__ inline Smem smem_layout(int r_k) {
@@ -58,7 +61,9 @@ __host__ __device__ inline Smem smem_layout(int r_k) {
   s.zk = o;     o += kNKS * kZkBytes;
   s.zv = o;     o += kNVS * kZvBytes;
   s.p = o;      o += 2 * kPBytes;
-  s.qr = o;     o += 2 * 128 * 4;
+  s.qr = o;     o += 3 * 128 * 4;                        // q'_i, q'_{i+64}, -q'_i per head pair row
+  s.psc = o;    o += 2 * 2 * 128 * 4;
+  s.tb = o;     o += 8 * 3 * 32 * 4;                     // per epilogue warp: cos, sin, -sin at t0
   s.omega = o;  o += 64 * 8;
   s.red = o;    o += 2 * 4 * 2 * 4;
   s.lred = o;   o += 4 * 2 * 4;
@@ -81,7 +86,9 @@ enum {
   BAR_P_FULL = BAR_D_EMPTY + 2,      // 2
   BAR_AT_FULL = BAR_P_FULL + 2,      // 1
   BAR_TEARDOWN = BAR_AT_FULL + 1,
-  BAR_EPI = BAR_TEARDOWN + 1,        // epilogue-wide sync (128 threads), bounded
+  BAR_EPI = BAR_TEARDOWN + 1,        // 2: per-warpgroup sync (4 warps), bounded
+  BAR_QR = BAR_EPI + 2,              // rotated query staged
+  BAR_XCH = BAR_QR + 1,              // 2: both warpgroups posted their cross-head partial scores
   BAR_COUNT
 };
 static_assert(BAR_COUNT <= 32, "barrier space");
@@ -144,10 +151,16 @@ __device__ __forceinline__ float from_bits(uint16_t u) {
   }
 }
 
+// Phase trace record (palu_debug_trace).
+__device__ __forceinline__ void trace_record(const DecodeArgs& a, int ev, int k, long long t_start) {
+  if (k >= a.trace_tiles) return;
+  const size_t cta = ((size_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
+  a.trace[(cta * 8 + ev) * a.trace_tiles + k] = clock64() - t_start;
+}
+
 template <int ACT, int NRV>
 __global__ void __launch_bounds__(kThreads, 1)
-    decode_tc_kernel(const __grid_constant__ CUtensorMap tm_zk, const __grid_constant__ CUtensorMap tm_zv,
-                     const __grid_constant__ CUtensorMap tm_bk, const DecodeArgs a) {
+    decode_tc_kernel(const __grid_constant__ CUtensorMap tm_bk, const DecodeArgs a) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -162,8 +175,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nhp = a.gs / 2;                         // head pairs per group
   const int g = blockIdx.y / nhp, hp = blockIdx.y % nhp;
   const int nkc = a.r_k / kChunk;
-  const int rows_total = a.num_pages * a.G * a.P;   // OOB row for bad pages => zero fill
   const TileRange tr = tile_range(a, b, st, threadIdx.x == 0);
+  const long long t_start = clock64();
+  auto trace = [&](int ev, int k) {
+    if (a.trace != nullptr) trace_record(a, ev, k, t_start);
+  };
 
   // ---------------------------------------------------------------- setup
   if (threadIdx.x == 0) {
@@ -179,19 +195,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(BAR_D_FULL + i), 1);
-      mbar_init(bar(BAR_D_EMPTY + i), 4);
-      mbar_init(bar(BAR_P_FULL + i), 4);
+      mbar_init(bar(BAR_D_EMPTY + i), 8);
+      mbar_init(bar(BAR_P_FULL + i), 8);
     }
     mbar_init(bar(BAR_AT_FULL), 1);
     mbar_init(bar(BAR_TEARDOWN), 1);
-    mbar_init(bar(BAR_EPI), 128);
+    mbar_init(bar(BAR_QR), 4);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(BAR_EPI + i), 4);
+      mbar_init(bar(BAR_XCH + i), 8);
+    }
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) {
-    prefetch_tmap(&tm_zk);
-    prefetch_tmap(&tm_zv);
-    prefetch_tmap(&tm_bk);
-  }
+  if (warp == 0 && lane == 0) prefetch_tmap(&tm_bk);
   if (warp == 1) {
     tmem_alloc(base + L.tmem_slot, 512);
     tmem_relinquish();
@@ -215,20 +231,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_2d(base + L.b + (uint32_t)nb * a.r_k * 128, &tm_bk, hp * 256 + nb * 64, g * a.r_k, bar(BAR_B));
       int stage = 0;
       uint32_t phase = 0;
+      // Pull the next pages of this split into L2 ahead of the TMA loads: the
+      // shared-memory ring is only a few chunks deep, so HBM latency is hidden
+      // in L2 instead.
+      auto prefetch_page = [&](int kk) {
+        if (kk >= tr.ntiles) return;
+        const int ppg = page_of(a, b, tr.t_begin / kTile + kk);
+        if (ppg < 0) return;
+        const size_t row = (size_t)(ppg * a.G + g) * a.P;
+        prefetch_l2(reinterpret_cast<const uint8_t*>(a.zk) + row * a.k_row, (uint32_t)(a.P * a.k_row));
+        if (!(tr.ragged_last && kk == tr.ntiles - 1))
+          prefetch_l2(reinterpret_cast<const uint8_t*>(a.zv) + row * a.v_row, (uint32_t)(a.P * a.v_row));
+      };
+      for (int kk = 0; kk < kPrefetch; ++kk) prefetch_page(kk);
       for (int k = 0; k < tr.ntiles && !*abort_flag; ++k) {
+        prefetch_page(k + kPrefetch);
         const int lp = tr.t_begin / kTile + k;
-        const int pg = page_of(a, b, lp);
-        if (pg < 0) report(st, PALU_ERR_DEVICE_BOUNDS, 2000000 + b);
-        const int row0 = pg < 0 ? rows_total : (pg * a.G + g) * a.P;
+        int pg = page_of(a, b, lp);
+        if (pg < 0) {
+          report(st, PALU_ERR_DEVICE_BOUNDS, 2000000 + b);
+          pg = 0;   // keep the pipeline fed from a valid page; the status says the result is void
+        }
+        // one (page, group) block is the shared-memory image of the tile: each
+        // 128-byte column block (64 latent entries of all 128 tokens) is one copy
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(a.zk) + (size_t)(pg * a.G + g) * a.P * a.k_row;
         for (int c = 0; c < nkc; ++c) {
           if (!mbar_wait(bar(BAR_ZK_EMPTY + stage), phase ^ 1, abort_flag, st, 10)) break;
           mbar_expect_tx(bar(BAR_ZK_FULL + stage), kZkBytes);
-          tma_load_2d(base + L.zk + stage * kZkBytes, &tm_zk, c * kChunk, row0, bar(BAR_ZK_FULL + stage));
+          bulk_load(base + L.zk + stage * kZkBytes, src + (size_t)c * kZkBytes, kZkBytes, bar(BAR_ZK_FULL + stage));
+          if (c == 0) trace(6, k);
           if (++stage == kNKS) { stage = 0; phase ^= 1; }
         }
       }
     }
-  } else if (warp == 6) {
+  } else if (warp == 2) {
     // ============================================================ z_v producer
     if (lane == 0) {
       int stage = 0;
@@ -236,15 +272,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int k = 0; k < tr.ntiles && !*abort_flag; ++k) {
         if (tr.ragged_last && k == tr.ntiles - 1) break;    // CUDA-core value sum for a partial page
         const int lp = tr.t_begin / kTile + k;
-        const int pg = page_of(a, b, lp);
-        const int row0 = pg < 0 ? rows_total : (pg * a.G + g) * a.P;
+        int pg = page_of(a, b, lp);
+        if (pg < 0) pg = 0;   // reported by the z_k producer
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(a.zv) + (size_t)(pg * a.G + g) * a.P * a.v_row;
         for (int mb = 0; mb < NRV; ++mb) {
           for (int th = 0; th < 2; ++th) {
             if (!mbar_wait(bar(BAR_ZV_EMPTY + stage), phase ^ 1, abort_flag, st, 11)) break;
             mbar_expect_tx(bar(BAR_ZV_FULL + stage), kZvBytes);
             const uint32_t dst = base + L.zv + stage * kZvBytes;
-            tma_load_2d(dst, &tm_zv, mb * 128, row0 + th * 64, bar(BAR_ZV_FULL + stage));
-            tma_load_2d(dst + 8192, &tm_zv, mb * 128 + 64, row0 + th * 64, bar(BAR_ZV_FULL + stage));
+            // 64 tokens of two 128-byte column blocks = the two MN-blocks of the value operand
+            const size_t off = (size_t)(2 * mb) * a.P * 128 + (size_t)th * 64 * 128;
+            bulk_load(dst, src + off, 8192, bar(BAR_ZV_FULL + stage));
+            bulk_load(dst + 8192, src + off + (size_t)a.P * 128, 8192, bar(BAR_ZV_FULL + stage));
             if (++stage == kNVS) { stage = 0; phase ^= 1; }
           }
         }
@@ -260,9 +299,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       int zs = 0, vs = 0;
       uint32_t zph = 0, vph = 0;
       bool ok = mbar_wait(bar(BAR_B), 0, abort_flag, st, 20);
+      int pv_pending = -1;   // tile whose value MMA waits for its P
 
+      // aᵀ[r_v × 16] = z_vᵀ · Pᵀ for tile j into its (drained) D slot
       auto issue_pv = [&](int j) -> bool {
-        if (!mbar_wait(bar(BAR_P_FULL + (j & 1)), (j >> 1) & 1, abort_flag, st, 21)) return false;
         tc_fence_after();
         const uint32_t a_tmem = tmem + (uint32_t)(j & 1) * 256;
         for (int mb = 0; mb < NRV; ++mb) {
@@ -273,8 +313,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t p_addr = base + L.p + (uint32_t)(j & 1) * kPBytes + th * 2048;
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t ad = sdesc_sw128(zv_addr + kk * 16 * 128, 8192, 1024);
-              const uint64_t bd = sdesc_sw128(p_addr + kk * 32, 16, 1024);
+              const uint64_t ad = sdesc(zv_addr + kk * 16 * 128, 8192, 1024, kSw128);
+              const uint64_t bd = sdesc(p_addr + kk * 32, 16, 1024, kSw128);
               umma_f16(a_tmem + mb * 16, ad, bd, idesc_pv, (th | kk) != 0);
             }
             umma_commit(bar(BAR_ZV_EMPTY + vs));
@@ -282,60 +322,94 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         umma_commit(bar(BAR_AT_FULL));
+        trace(2, j);
+        pv_pending = -1;
         return true;
+      };
+      // Wait for z_k data; meanwhile issue the pending value MMA as soon as its
+      // P is ready, so the epilogue gets its latent sums early.  Bounded.
+      auto wait_zk = [&]() -> bool {
+        const long long t0 = clock64();
+        while (true) {
+          if (mbar_test_wait(bar(BAR_ZK_FULL + zs), zph)) return true;
+          if (pv_pending >= 0 &&
+              mbar_test_wait(bar(BAR_P_FULL + (pv_pending & 1)), (pv_pending >> 1) & 1)) {
+            if (!issue_pv(pv_pending)) return false;
+          }
+          if (*abort_flag) return false;
+          __nanosleep(64);   // leave the issue slots of this SM partition to the epilogue warps
+          if (clock64() - t0 > kWaitCycles) {
+            report(st, PALU_ERR_DEVICE_TIMEOUT, 24);
+            *abort_flag = 1;
+            return false;
+          }
+        }
+      };
+      auto flush_pv = [&]() -> bool {
+        if (pv_pending < 0) return true;
+        if (!mbar_wait(bar(BAR_P_FULL + (pv_pending & 1)), (pv_pending >> 1) & 1, abort_flag, st, 21))
+          return false;
+        return issue_pv(pv_pending);
       };
 
       for (int k = 0; k < tr.ntiles && ok; ++k) {
         const int slot = k & 1;
         if (!mbar_wait(bar(BAR_D_EMPTY + slot), ((k >> 1) & 1) ^ 1, abort_flag, st, 23)) { ok = false; break; }
         tc_fence_after();
+        trace(0, k);
         const uint32_t d_tmem = tmem + (uint32_t)slot * 256;
-        const int pv_at = nkc >= 2 ? nkc - 2 : 0;
         for (int c = 0; c < nkc; ++c) {
-          if (!mbar_wait(bar(BAR_ZK_FULL + zs), zph, abort_flag, st, 24)) { ok = false; break; }
+          if (!wait_zk()) { ok = false; break; }
           tc_fence_after();
+          if (c == 0) trace(7, k);
           const uint32_t zk_addr = base + L.zk + zs * kZkBytes;
           const uint32_t b_addr = base + L.b + (uint32_t)c * kChunk * 128;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t ad = sdesc_sw128(zk_addr + kk * 32, 16, 1024);
-            const uint64_t bd = sdesc_sw128(b_addr + kk * 16 * 128, b_lbo, 1024);
+          for (int kk = 0; kk < kChunk / 16; ++kk) {
+            const uint64_t ad = sdesc(zk_addr + kk * 32, 16, kZkSbo, kZkSwz);
+            const uint64_t bd = sdesc(b_addr + kk * 16 * 128, b_lbo, 1024, kSw128);
             umma_f16(d_tmem, ad, bd, idesc_d, (c | kk) != 0);
           }
           umma_commit(bar(BAR_ZK_EMPTY + zs));
           if (++zs == kNKS) { zs = 0; zph ^= 1; }
-          if (c == pv_at && k >= 1 && !(tr.ragged_last && k - 1 == tr.ntiles - 1)) {
-            if (!issue_pv(k - 1)) { ok = false; break; }
-          }
         }
         if (!ok) break;
         umma_commit(bar(BAR_D_FULL + slot));
+        trace(1, k);
+        // the previous tile's value MMA must be out before this one queues
+        if (!flush_pv()) { ok = false; break; }
+        if (!(tr.ragged_last && k == tr.ntiles - 1)) pv_pending = k;
       }
-      if (ok && tr.ntiles > 0 && !tr.ragged_last) ok = issue_pv(tr.ntiles - 1);
+      if (ok) ok = flush_pv();
       // drain: every MMA issued above has completed before TMEM is released
       umma_commit(bar(BAR_TEARDOWN));
       mbar_wait(bar(BAR_TEARDOWN), 0, abort_flag, st, 25);
     }
-  } else {
-    // ============================================================ epilogue (warps 2-5)
+  } else if (warp >= 4) {
+    // ============================================================ epilogue (warps 4-11)
+    // Two warpgroups split the 64 RoPE frequency pairs of every key (wg 0:
+    // pairs [0, 32), wg 1: [32, 64)) for both heads, then each finishes one head.
+    const int wg = (warp - 4) >> 2;
     const int q4 = warp & 3;                 // TMEM lane quarter this warp may access
     const int row = q4 * 32 + lane;          // token row of the tile / latent row of aᵀ
     const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
     float* qr = reinterpret_cast<float*>(sbase + L.qr);
+    float* psc = reinterpret_cast<float*>(sbase + L.psc);   // [slot][head][128]
     const uint64_t* om = reinterpret_cast<const uint64_t*>(sbase + L.omega);
     const int head0 = g * a.gs + hp * 2;
     constexpr float kLog2e = 1.4426950408889634f;
-    // All 128 epilogue threads meet here; a bounded wait (unlike bar.sync), so a
-    // thread that gave up on a timed-out wait cannot strand the others.
+    // the 4 warps of one warpgroup meet here; a bounded wait (unlike bar.sync), so a thread that gave
+    // up on a timed-out wait cannot strand the others.
     uint32_t epi_phase = 0;
     auto ep_sync = [&](int where) -> bool {
-      mbar_arrive(bar(BAR_EPI));
-      const bool r = mbar_wait(bar(BAR_EPI), epi_phase, abort_flag, st, where);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(BAR_EPI + wg));
+      const bool r = mbar_wait(bar(BAR_EPI + wg), epi_phase, abort_flag, st, where);
       epi_phase ^= 1;
       return r;
     };
     // rotated query of both heads, scaled by log2(e)/sqrt(d_h) for exp2
-    {
+    if (wg == 0) {
       const int hh = row >> 6, i = row & 63;
       using TA = typename Dt<ACT>::T;
       const TA* qh = reinterpret_cast<const TA*>(a.q) + ((size_t)b * a.H + head0 + hh) * 128;
@@ -343,176 +417,240 @@ __global__ void __launch_bounds__(kThreads, 1)
       float c = 1.f, s = 0.f;
       if (a.rope) rope_cs_fast(a.q_pos[b], a.omega[i], c, s);
       const float sc = a.sm_scale * kLog2e;
-      qr[hh * 128 + i] = (x1 * c - x2 * s) * sc;
-      qr[hh * 128 + i + 64] = (x2 * c + x1 * s) * sc;
-    }
-    bool ok = ep_sync(32);
-
-    float m_run[2] = {-INFINITY, -INFINITY};
-    float l_part[2] = {0.f, 0.f};
-    float acc[2][NRV];
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-      for (int mb = 0; mb < NRV; ++mb) acc[hh][mb] = 0.f;
-    float prev_scale[2] = {0.f, 0.f};
-    float* red = reinterpret_cast<float*>(sbase + L.red);
-
-    auto fold_at = [&](int j, const float* scale) -> bool {
-      if (!mbar_wait(bar(BAR_AT_FULL), j & 1, abort_flag, st, 30)) return false;
-      tc_fence_after();
-#pragma unroll
-      for (int mb = 0; mb < NRV; ++mb) {
-        float v[2];
-        tmem_ld2(tmem + lane_addr + (uint32_t)(j & 1) * 256 + mb * 16, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) acc[hh][mb] = fmaf(acc[hh][mb], scale[hh], v[hh]);
-      }
-      tc_fence_before();
+      const float qa = (x1 * c - x2 * s) * sc, qb = (x2 * c + x1 * s) * sc;
+      qr[hh * 192 + i] = qa;
+      qr[hh * 192 + 64 + i] = qb;
+      qr[hh * 192 + 128 + i] = -qa;
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(BAR_D_EMPTY + (j & 1)));
-      return true;
-    };
+      if (lane == 0) mbar_arrive(bar(BAR_QR));
+    }
+    bool ok = mbar_wait(bar(BAR_QR), 0, abort_flag, st, 32);
 
-    for (int k = 0; k < tr.ntiles && ok; ++k) {
-      const int t0 = tr.t_begin + k * kTile;
-      const bool valid = t0 + row < tr.t_end;
-      int pos = t0 + row;
-      if (a.pos_pool != nullptr) {
-        const int pg = page_of(a, b, t0 / kTile);
-        pos = pg >= 0 ? a.pos_pool[(size_t)pg * a.P + row] : 0;
-      }
-      const int slot = k & 1;
-      if (!mbar_wait(bar(BAR_D_FULL + slot), (k >> 1) & 1, abort_flag, st, 31)) { ok = false; break; }
-      tc_fence_after();
-      float sacc[2] = {0.f, 0.f};
-#pragma unroll 1
-      for (int j = 0; j < 2; ++j) {
-        float cs[32], sn[32];
+    // Partial scores of both heads over this warpgroup's 32 frequency pairs i:
+    //   score += c_i (q'_i k_i + q'_{i+64} k_{i+64}) + s_i (q'_{i+64} k_i - q'_i k_{i+64})
+    // which is q'·k' with k' the key rotated by the token's angle (rotate-half).
+    // Contiguous positions (pos = t0 + row): (c, s) at t0 + row come from the
+    // tile base at t0 (one sincos per warp lane per tile) and this thread's
+    // fixed offset `row`, by angle addition; explicit positions take a sincos
+    // per token.  Math runs on packed fp32 pairs (two frequencies at a time).
+    const bool contig = a.pos_pool == nullptr;
+    float* tbw = reinterpret_cast<float*>(sbase + L.tb) + (warp - 4) * 96;   // [cos|sin|-sin][32]
+    f2 crow[16], srow[16];
+    if (contig) {
 #pragma unroll
-        for (int u = 0; u < 32; ++u) {
-          if (a.rope) {
-            rope_cs_fast(pos, om[j * 32 + u], cs[u], sn[u]);
-          } else {
-            cs[u] = 1.f;
-            sn[u] = 0.f;
+      for (int v = 0; v < 16; ++v) {
+        float c0, s0, c1, s1;
+        rope_cs_fast(row, om[wg * 32 + 2 * v], c0, s0);
+        rope_cs_fast(row, om[wg * 32 + 2 * v + 1], c1, s1);
+        crow[v] = f2_pack(c0, c1);
+        srow[v] = f2_pack(s0, s1);
+      }
+    }
+    auto half_scores = [&](int slot, int t0, int pos, float* part) {
+      if (contig) {
+        float c, sn;
+        rope_cs_fast(t0, om[wg * 32 + lane], c, sn);
+        __syncwarp();
+        tbw[lane] = c;
+        tbw[32 + lane] = sn;
+        tbw[64 + lane] = -sn;
+        __syncwarp();
+      }
+      f2 acc[2][2];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) acc[hh][0] = acc[hh][1] = 0ull;
+#pragma unroll
+      for (int jj = 0; jj < 2; ++jj) {
+        const int i0 = wg * 32 + jj * 16;
+        const uint32_t col = tmem + lane_addr + (uint32_t)slot * 256 + i0;
+        float lo[16], hi[16];
+        tmem_ld16(col, lo);
+        tmem_ld16(col + 64, hi);
+        f2 cs[8], sn[8];
+        if (contig) {
+          const float4* c4 = reinterpret_cast<const float4*>(tbw + jj * 16);
+          const float4* s4 = reinterpret_cast<const float4*>(tbw + 32 + jj * 16);
+          const float4* n4 = reinterpret_cast<const float4*>(tbw + 64 + jj * 16);
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4) {
+            const float4 cb = c4[v4], sb = s4[v4], nb = n4[v4];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int v = v4 * 2 + e;
+              const f2 c0 = e ? f2_pack(cb.z, cb.w) : f2_pack(cb.x, cb.y);
+              const f2 s0 = e ? f2_pack(sb.z, sb.w) : f2_pack(sb.x, sb.y);
+              const f2 n0 = e ? f2_pack(nb.z, nb.w) : f2_pack(nb.x, nb.y);
+              // cos(t0+row) = c0 cr - s0 sr ; sin(t0+row) = s0 cr + c0 sr
+              cs[v] = f2_fma(c0, crow[jj * 8 + v], f2_mul(n0, srow[jj * 8 + v]));
+              sn[v] = f2_fma(s0, crow[jj * 8 + v], f2_mul(c0, srow[jj * 8 + v]));
+            }
+          }
+        } else {
+          // explicit positions: a sincos per token
+#pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            float c0, s0, c1, s1;
+            rope_cs_fast(pos, om[i0 + 2 * v], c0, s0);
+            rope_cs_fast(pos, om[i0 + 2 * v + 1], c1, s1);
+            cs[v] = f2_pack(c0, c1);
+            sn[v] = f2_pack(s0, s1);
           }
         }
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
-          float lo[32], hi[32];
-          const uint32_t col = tmem + lane_addr + (uint32_t)slot * 256 + hh * 128 + j * 32;
-          tmem_ld32(col, lo);
-          tmem_ld32(col + 64, hi);
-          tmem_wait_ld();
-          const float* qa = qr + hh * 128 + j * 32;
-          float s = 0.f;
-#pragma unroll
-          for (int u = 0; u < 32; ++u) {
-            const float k1 = lo[u] * cs[u] - hi[u] * sn[u];
-            const float k2 = hi[u] * cs[u] + lo[u] * sn[u];
-            s = fmaf(qa[u], k1, s);
-            s = fmaf(qa[u + 64], k2, s);
+          if (hh == 1) {
+            tmem_ld16(col + 128, lo);
+            tmem_ld16(col + 192, hi);
           }
-          sacc[hh] += s;
-        }
-      }
-      tc_fence_before();
-      // tile max per head across the 128 tokens
-      float sc[2], mt[2];
+          tmem_wait_ld();
+          const float4* qa4 = reinterpret_cast<const float4*>(qr + hh * 192 + i0);
+          const float4* qb4 = reinterpret_cast<const float4*>(qr + hh * 192 + 64 + i0);
+          const float4* qn4 = reinterpret_cast<const float4*>(qr + hh * 192 + 128 + i0);
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        sc[hh] = valid ? sacc[hh] : -INFINITY;
-        float m = sc[hh];
+          for (int v4 = 0; v4 < 4; ++v4) {
+            const float4 qa = qa4[v4], qb = qb4[v4], qn = qn4[v4];
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-        if (lane == 0) red[(k & 1) * 8 + q4 * 2 + hh] = m;
-      }
-      if (!ep_sync(33)) { ok = false; break; }
-      float scale[2], p[2];
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const float* rr = red + (k & 1) * 8;
-        mt[hh] = fmaxf(fmaxf(rr[0 * 2 + hh], rr[1 * 2 + hh]), fmaxf(rr[2 * 2 + hh], rr[3 * 2 + hh]));
-        const float m_new = fmaxf(m_run[hh], mt[hh]);
-        scale[hh] = exp2f(m_run[hh] - m_new);                 // 0 on the first tile
-        const uint16_t pb = to_bits<ACT>(valid ? exp2f(sc[hh] - m_new) : 0.f);
-        p[hh] = from_bits<ACT>(pb);
-        *reinterpret_cast<uint16_t*>(sbase + L.p + slot * kPBytes + p_offset(hh, row)) = pb;
-        l_part[hh] = fmaf(l_part[hh], scale[hh], p[hh]);
-        m_run[hh] = m_new;
-      }
-      fence_proxy_async();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(BAR_P_FULL + slot));
-      if (k >= 1) {
-        if (!fold_at(k - 1, prev_scale)) { ok = false; break; }
-      }
-      prev_scale[0] = scale[0];
-      prev_scale[1] = scale[1];
-    }
-
-    if (ok && tr.ntiles > 0) {
-      const int kl = tr.ntiles - 1;
-      if (!tr.ragged_last) {
-        ok = fold_at(kl, prev_scale);
-      } else {
-        // partial last page: a += Σ_{valid tokens} p · z_v on CUDA cores,
-        // reading only the valid rows (the rest of the page is never touched)
-        ok = ep_sync(34);   // every P entry of this tile is written
-        const int t0 = tr.t_begin + kl * kTile;
-        const int nvalid = tr.t_end - t0;
-        const int pg = page_of(a, b, t0 / kTile);
-        using TL = typename Dt<ACT>::T;
-        float at[2][NRV];
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-          for (int mb = 0; mb < NRV; ++mb) at[hh][mb] = 0.f;
-        if (pg >= 0) {
-          const TL* zv = reinterpret_cast<const TL*>(
-              reinterpret_cast<const uint8_t*>(a.zv) + ((size_t)(pg * a.G + g) * a.P) * a.v_row);
-          const uint8_t* pb = sbase + L.p + (kl & 1) * kPBytes;
-          for (int t = 0; t < nvalid; ++t) {
-            const float p0 = from_bits<ACT>(*reinterpret_cast<const uint16_t*>(pb + p_offset(0, t)));
-            const float p1 = from_bits<ACT>(*reinterpret_cast<const uint16_t*>(pb + p_offset(1, t)));
-#pragma unroll
-            for (int mb = 0; mb < NRV; ++mb) {
-              const float z = Dt<ACT>::to_f(zv[(size_t)t * a.r_v + mb * 128 + row]);
-              at[0][mb] = fmaf(p0, z, at[0][mb]);
-              at[1][mb] = fmaf(p1, z, at[1][mb]);
+            for (int e = 0; e < 2; ++e) {
+              const int v = v4 * 2 + e;
+              const f2 a2 = e ? f2_pack(qa.z, qa.w) : f2_pack(qa.x, qa.y);
+              const f2 b2 = e ? f2_pack(qb.z, qb.w) : f2_pack(qb.x, qb.y);
+              const f2 n2 = e ? f2_pack(qn.z, qn.w) : f2_pack(qn.x, qn.y);
+              const f2 lo2 = f2_pack(lo[2 * v], lo[2 * v + 1]);
+              const f2 hi2 = f2_pack(hi[2 * v], hi[2 * v + 1]);
+              const f2 x = f2_fma(b2, hi2, f2_mul(a2, lo2));     // q'_i k_i + q'_{i+64} k_{i+64}
+              const f2 y = f2_fma(b2, lo2, f2_mul(n2, hi2));     // q'_{i+64} k_i - q'_i k_{i+64}
+              acc[hh][e] = f2_fma(cs[v], x, acc[hh][e]);
+              acc[hh][e] = f2_fma(sn[v], y, acc[hh][e]);
             }
           }
         }
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-          for (int mb = 0; mb < NRV; ++mb) acc[hh][mb] = fmaf(acc[hh][mb], prev_scale[hh], at[hh][mb]);
       }
-    }
-
-    // l: sum of the per-thread partials of each head
-    float* lred = reinterpret_cast<float*>(sbase + L.lred);
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      float v = l_part[hh];
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-      if (lane == 0) lred[q4 * 2 + hh] = v;
-    }
-    ok = ep_sync(35) && ok;
-    if (ok && !*abort_flag) {
-      constexpr float kLn2 = 0.6931471805599453f;
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
-        float* out = a.part + (((size_t)b * a.H + head0 + hh) * a.S + blockIdx.x) * (a.r_v + 2);
+        float a0, a1, a2, a3;
+        f2_unpack(acc[hh][0], a0, a1);
+        f2_unpack(acc[hh][1], a2, a3);
+        part[hh] = (a0 + a1) + (a2 + a3);
+      }
+    };
+
+    {
+      // Each warpgroup owns one head of the pair (hw = wg) for the softmax, P,
+      // the latent value sums and the output; the partial scores of the other
+      // head go across in shared memory.
+      const int hw = wg;
+      float m_run = -INFINITY, l_part = 0.f, prev_scale = 0.f;
+      float acc[NRV];
+#pragma unroll
+      for (int mb = 0; mb < NRV; ++mb) acc[mb] = 0.f;
+      float* red = reinterpret_cast<float*>(sbase + L.red);
+
+      auto fold_at = [&](int j, float scale) -> bool {
+        if (!mbar_wait(bar(BAR_AT_FULL), j & 1, abort_flag, st, 30)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int mb = 0; mb < NRV; ++mb) {
+          const float v = tmem_ld1(tmem + lane_addr + (uint32_t)(j & 1) * 256 + mb * 16 + hw);
+          tmem_wait_ld();
+          acc[mb] = fmaf(acc[mb], scale, v);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(BAR_D_EMPTY + (j & 1)));
+        return true;
+      };
+
+      for (int k = 0; k < tr.ntiles && ok; ++k) {
+        if (k >= 1 && !fold_at(k - 1, prev_scale)) { ok = false; break; }
+        const int t0 = tr.t_begin + k * kTile;
+        const bool valid = t0 + row < tr.t_end;
+        int pos = t0 + row;
+        if (a.pos_pool != nullptr) {
+          const int pg = page_of(a, b, t0 / kTile);
+          pos = pg >= 0 ? a.pos_pool[(size_t)pg * a.P + row] : 0;
+        }
+        const int slot = k & 1;
+        if (!mbar_wait(bar(BAR_D_FULL + slot), (k >> 1) & 1, abort_flag, st, 31)) { ok = false; break; }
+        tc_fence_after();
+        if (row == 0 && wg == 0) trace(3, k);
+        float part[2];
+        half_scores(slot, t0, pos, part);
+        tc_fence_before();
+        psc[(slot * 2 + (1 - hw)) * 128 + row] = part[1 - hw];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(BAR_XCH + slot));
+        if (!mbar_wait(bar(BAR_XCH + slot), (k >> 1) & 1, abort_flag, st, 36)) { ok = false; break; }
+        const float sfull = part[hw] + psc[(slot * 2 + hw) * 128 + row];
+        if (row == 0 && wg == 0) trace(4, k);
+        // tile max of this head across the 128 tokens
+        const float sc = valid ? sfull : -INFINITY;
+        float m = sc;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+        if (lane == 0) red[(k & 1) * 8 + wg * 4 + q4] = m;
+        if (!ep_sync(33)) { ok = false; break; }
+        const float* rr = red + (k & 1) * 8 + wg * 4;
+        const float mt = fmaxf(fmaxf(rr[0], rr[1]), fmaxf(rr[2], rr[3]));
+        const float m_new = fmaxf(m_run, mt);
+        const float scale = exp2f(m_run - m_new);                 // 0 on the first tile
+        const uint16_t pb = to_bits<ACT>(valid ? exp2f(sc - m_new) : 0.f);
+        *reinterpret_cast<uint16_t*>(sbase + L.p + slot * kPBytes + p_offset(hw, row)) = pb;
+        l_part = fmaf(l_part, scale, from_bits<ACT>(pb));
+        m_run = m_new;
+        fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(BAR_P_FULL + slot));
+        if (row == 0 && wg == 0) trace(5, k);
+        prev_scale = scale;
+      }
+
+      if (ok && tr.ntiles > 0) {
+        const int kl = tr.ntiles - 1;
+        if (!tr.ragged_last) {
+          ok = fold_at(kl, prev_scale);
+        } else {
+          // partial last page: a += Σ_{valid tokens} p · z_v on CUDA cores,
+          // reading only the valid rows (the rest of the page is never touched)
+          ok = ep_sync(34);   // every P entry of this head is written
+          const int t0 = tr.t_begin + kl * kTile;
+          const int nvalid = tr.t_end - t0;
+          const int pg = page_of(a, b, t0 / kTile);
+          using TL = typename Dt<ACT>::T;
+          float at[NRV];
+#pragma unroll
+          for (int mb = 0; mb < NRV; ++mb) at[mb] = 0.f;
+          if (pg >= 0) {
+            const uint8_t* zv = reinterpret_cast<const uint8_t*>(a.zv) + (size_t)(pg * a.G + g) * a.P * a.v_row;
+            const uint8_t* pbuf = sbase + L.p + (kl & 1) * kPBytes;
+            for (int t = 0; t < nvalid; ++t) {
+              const float pv = from_bits<ACT>(*reinterpret_cast<const uint16_t*>(pbuf + p_offset(hw, t)));
+#pragma unroll
+              for (int mb = 0; mb < NRV; ++mb)
+                at[mb] = fmaf(pv, Dt<ACT>::to_f(*reinterpret_cast<const TL*>(
+                                      zv + swz_offset(t, (long long)(mb * 128 + row) * 2, a.P))), at[mb]);
+            }
+          }
+#pragma unroll
+          for (int mb = 0; mb < NRV; ++mb) acc[mb] = fmaf(acc[mb], prev_scale, at[mb]);
+        }
+      }
+
+      // l: sum of the per-thread partials of this head
+      float* lred = reinterpret_cast<float*>(sbase + L.lred);
+      float v = l_part;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+      if (lane == 0) lred[wg * 4 + q4] = v;
+      ok = ep_sync(35) && ok;
+      if (ok && !*abort_flag) {
+        constexpr float kLn2 = 0.6931471805599453f;
+        float* out = a.part + (((size_t)b * a.H + head0 + hw) * a.S + blockIdx.x) * (a.r_v + 2);
         if (row == 0) {
-          out[0] = tr.ntiles > 0 ? m_run[hh] * kLn2 : -INFINITY;
-          out[1] = lred[0 * 2 + hh] + lred[1 * 2 + hh] + lred[2 * 2 + hh] + lred[3 * 2 + hh];
+          out[0] = tr.ntiles > 0 ? m_run * kLn2 : -INFINITY;
+          out[1] = (lred[wg * 4 + 0] + lred[wg * 4 + 1]) + (lred[wg * 4 + 2] + lred[wg * 4 + 3]);
         }
 #pragma unroll
-        for (int mb = 0; mb < NRV; ++mb) out[2 + mb * 128 + row] = acc[hh][mb];
+        for (int mb = 0; mb < NRV; ++mb) out[2 + mb * 128 + row] = acc[mb];
       }
     }
   }
@@ -542,7 +680,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 bool make_map_2d(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, int elt_bytes, uint64_t inner,
-                 uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+                 uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                 CUtensorMapSwizzle swz) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[2] = {inner, outer};
@@ -551,7 +690,7 @@ bool make_map_2d(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, int el
   cuuint32_t estr[2] = {1, 1};
   (void)elt_bytes;
   CUresult r = fn(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -559,19 +698,24 @@ bool make_map_2d(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, int el
 template <int ACT, int NRV>
 cudaError_t launch_t(const DecodeArgs& a, cudaStream_t st) {
   const CUtensorMapDataType dt = ACT == PALU_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-  const uint64_t rows = (uint64_t)a.num_pages * a.G * a.P;
-  CUtensorMap tm_zk, tm_zv, tm_bk;
-  if (!make_map_2d(&tm_zk, a.zk, dt, 2, a.r_k, rows, (uint64_t)a.r_k * 2, 64, 128) ||
-      !make_map_2d(&tm_zv, a.zv, dt, 2, a.r_v, rows, (uint64_t)a.r_v * 2, 64, 64) ||
-      !make_map_2d(&tm_bk, a.Bk, dt, 2, a.W, (uint64_t)a.G * a.r_k, (uint64_t)a.W * 2, 64, a.r_k))
+  CUtensorMap tm_bk;
+  if (!make_map_2d(&tm_bk, a.Bk, dt, 2, a.W, (uint64_t)a.G * a.r_k, (uint64_t)a.W * 2, 64, a.r_k,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   const Smem L = smem_layout(a.r_k);
   const size_t smem = L.total + 1024;
   auto kern = decode_tc_kernel<ACT, NRV>;
+  DecodeArgs args = a;
+  const TraceSetting ts = trace_setting();
+  const size_t ctas = (size_t)a.S * a.G * (a.gs / 2) * a.batch;
+  if (ts.buffer != nullptr && ctas * 8 * (size_t)ts.tiles * 8 <= ts.bytes) {
+    args.trace = static_cast<long long*>(ts.buffer);
+    args.trace_tiles = ts.tiles;
+  }
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(a.S, a.G * (a.gs / 2), a.batch);
-  kern<<<grid, kThreads, smem, st>>>(tm_zk, tm_zv, tm_bk, a);
+  kern<<<grid, kThreads, smem, st>>>(tm_bk, args);
   count_launch();
   return cudaGetLastError();
 }
@@ -583,7 +727,7 @@ bool tc_decode_supported(const palu_config* c) {
   if (c->group_size % 2 != 0) return false;
   if (c->act_dtype != PALU_F16 && c->act_dtype != PALU_BF16) return false;
   if (c->latent_dtype != c->act_dtype) return false;
-  if (c->rank_k % kChunk != 0 || c->rank_k > 256) return false;
+  if (c->rank_k % 64 != 0 || c->rank_k > 256) return false;
   if (c->rank_v != 128 && c->rank_v != 256) return false;
   const Smem L = smem_layout(c->rank_k);
   return L.total + 1024 <= 227 * 1024;

@@ -13,6 +13,8 @@
 
 namespace palu {
 static std::atomic<unsigned long long> g_launches{0};
+static TraceSetting g_trace{nullptr, 0, 0};
+TraceSetting trace_setting() { return g_trace; }
 void count_launch(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
 }  // namespace palu
 
@@ -44,9 +46,11 @@ palu_status check_config(const palu_config* c) {
   if (!pair_ok) return PALU_ERR_UNSUPPORTED;
   if (c->head_dim > 2 * palu::kMaxHalfDim) return PALU_ERR_UNSUPPORTED;
   if (c->rank_k > 512 || c->rank_v > 512) return PALU_ERR_UNSUPPORTED;
-  // 16-byte latent rows (TMA rows, vector stores); int4 needs whole 32-entry blocks
-  const int mult = c->latent_dtype == PALU_INT4 ? 32 : (c->latent_dtype == PALU_F32 ? 4 : 8);
-  if (c->rank_k % mult != 0 || c->rank_v % mult != 0) return PALU_ERR_ALIGNMENT;
+  // latent rows are whole 128-byte column blocks (the swizzled page layout)
+  if (palu::latent_row_bytes(c->latent_dtype, c->rank_k) % 128 != 0 ||
+      palu::latent_row_bytes(c->latent_dtype, c->rank_v) % 128 != 0)
+    return PALU_ERR_ALIGNMENT;
+  if (c->page_size % 8 != 0) return PALU_ERR_ALIGNMENT;
   return PALU_OK;
 }
 
@@ -112,6 +116,12 @@ const char* palu_status_string(palu_status s) {
 const char* palu_last_cuda_error(void) { return g_cuda_err; }
 
 int palu_decode_kernel_kind(const palu_config* cfg) { return kernel_kind(cfg); }
+
+palu_status palu_debug_trace(void* buffer, size_t bytes, int tiles_per_cta) {
+  if (buffer != nullptr && (tiles_per_cta <= 0 || bytes == 0)) return PALU_ERR_INVALID_ARG;
+  palu::g_trace = palu::TraceSetting{buffer, buffer ? bytes : 0, buffer ? tiles_per_cta : 0};
+  return PALU_OK;
+}
 
 uint64_t palu_kernel_launches(void) { return palu::g_launches.load(std::memory_order_relaxed); }
 

@@ -7,7 +7,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/palu.h"
+#include "palu.h"
 
 namespace palu {
 
@@ -46,18 +46,27 @@ template <> struct Dt<PALU_BF16> {
   __device__ __forceinline__ static T from_f(float v) { return __float2bfloat16_rn(v); }
 };
 
-// Decode one latent entry j of a row (int4: code × fp16 scale, rounded to the
-// compute dtype ACT exactly as the dequantised value the MMA path feeds).
+// Decode latent entry j of token t from its (page, group) block `blk` of P
+// tokens (swizzled layout; int4: code × fp16 scale from the token-major scale
+// row `srow`, rounded to the compute dtype ACT exactly as the dequantised value
+// the MMA path feeds).
+__host__ __device__ inline long long swz_offset(int t, long long o, int P) {
+  const long long b = o >> 7;
+  const int unit = (int)((o >> 4) & 7) ^ (t & 7);
+  return b * (long long)P * 128 + (long long)t * 128 + unit * 16 + (o & 15);
+}
+
 template <int LAT, int ACT>
-__device__ __forceinline__ float load_latent(const uint8_t* row, const uint8_t* srow, int j) {
+__device__ __forceinline__ float load_latent(const uint8_t* blk, int t, int P, const uint8_t* srow, int j) {
   if constexpr (LAT == PALU_INT4) {
-    uint8_t byte = row[j >> 1];
+    const uint8_t byte = blk[swz_offset(t, j >> 1, P)];
     int code = (j & 1) ? (byte >> 4) : (byte & 0xF);
     code = (code ^ 8) - 8;  // sign-extend the 4-bit two's complement
-    float s = __half2float(reinterpret_cast<const __half*>(srow)[j >> 5]);
+    const float s = __half2float(reinterpret_cast<const __half*>(srow)[j >> 5]);
     return Dt<ACT>::to_f(Dt<ACT>::from_f(float(code) * s));
   } else {
-    return Dt<LAT>::to_f(reinterpret_cast<const typename Dt<LAT>::T*>(row)[j]);
+    using T = typename Dt<LAT>::T;
+    return Dt<LAT>::to_f(*reinterpret_cast<const T*>(blk + swz_offset(t, (long long)j * sizeof(T), P)));
   }
 }
 

@@ -6,7 +6,7 @@
 #include <stddef.h>
 #include <stdint.h>
 
-#include "../../include/palu.h"
+#include "palu.h"
 
 namespace palu {
 
@@ -36,7 +36,17 @@ struct DecodeArgs {
   void* status;        // DevStatus*
   long long k_row, v_row, ks_row, vs_row;  // bytes per latent / scale row
   uint64_t omega[kMaxHalfDim];             // RoPE frequencies as 64-bit fixed-point turns
+  long long* trace;                        // phase trace (palu_debug_trace) or NULL
+  int trace_tiles;
 };
+
+// Phase-trace buffer set by palu_debug_trace (NULL: off).
+struct TraceSetting {
+  void* buffer;
+  size_t bytes;
+  int tiles;
+};
+TraceSetting trace_setting();
 
 struct CompressArgs {
   int n, d_model, G, r_k, r_v, P, num_pages;

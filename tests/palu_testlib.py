@@ -104,6 +104,32 @@ def make_decode_case(w: Workload, seq_lens, seed=None, explicit_positions=False,
                       zvs if w.latent_dtype == "int4" else None, pos, page_table, total_pages)
 
 
+# ------------------------------------------------------------------ cache page layout
+# One (page, group) block holds P tokens x R bytes (R a multiple of 128) as
+# 128-byte column blocks of all P tokens, the 16-byte units of token t's 128
+# bytes permuted by XOR (t mod 8) -- the layout include/palu.h documents.
+def _unit_perm(P: int) -> np.ndarray:
+    return np.arange(8)[None, :] ^ (np.arange(P)[:, None] & 7)          # [P, 8]
+
+
+def swizzle_block(rows: np.ndarray) -> np.ndarray:
+    """[P, R] token-major bytes -> the swizzled block image (flat uint8, P*R)."""
+    P, R = rows.shape
+    assert R % 128 == 0
+    src = rows.reshape(P, R // 128, 8, 16).transpose(1, 0, 2, 3)       # [nb, P, unit, 16]
+    out = np.empty_like(src)
+    out[:, np.arange(P)[:, None], _unit_perm(P), :] = src
+    return out.reshape(-1)
+
+
+def unswizzle_block(img: np.ndarray, P: int) -> np.ndarray:
+    """Inverse of swizzle_block: flat block image -> [P, R] token-major bytes."""
+    R = img.size // P
+    blk = img.reshape(R // 128, P, 8, 16)
+    src = blk[:, np.arange(P)[:, None], _unit_perm(P), :]               # [nb, P, unit, 16]
+    return src.transpose(1, 0, 2, 3).reshape(P, R)
+
+
 def _as_bytes(t: torch.Tensor) -> np.ndarray:
     return t.contiguous().view(torch.uint8).numpy() if t.dtype != torch.uint8 else t.numpy()
 
@@ -122,14 +148,18 @@ def build_pools(case: DecodeCase, device="cuda"):
             pools[name] = None
             continue
         row = page_bytes // (G * Pz)
-        host = np.zeros((npg, G, Pz, row), np.uint8)
+        swz = name in ("zk", "zv")            # latent pools are swizzled; scale pools are token-major
+        host = np.zeros((npg, G, Pz * row), np.uint8)
         for i, t in enumerate(case.seq_lens):
             if t == 0:
                 continue
             data = _as_bytes(lst[i]).reshape(G, t, -1)
             for p in range((t + Pz - 1) // Pz):
                 t0, t1 = p * Pz, min(t, (p + 1) * Pz)
-                host[case.page_table[i, p], :, : t1 - t0, : data.shape[2]] = data[:, t0:t1]
+                for g in range(G):
+                    blk = np.zeros((Pz, row), np.uint8)
+                    blk[: t1 - t0, : data.shape[2]] = data[g, t0:t1]
+                    host[case.page_table[i, p], g] = swizzle_block(blk) if swz else blk.reshape(-1)
         pools[name] = torch.from_numpy(host.reshape(-1)).to(device)
     pos_pool = None
     if any(pp is not None for pp in case.pos):

@@ -7,6 +7,7 @@ import pytest
 import torch
 
 from oracle import palu_oracle as O
+from palu_testlib import unswizzle_block
 from rank_kv_cache_palu_b200 import api as P
 from rank_kv_cache_palu_b200.synth import TORCH_DTYPE, WORKLOADS, normal_tensor
 
@@ -29,13 +30,20 @@ def run_compress(w, x, A_k, A_v, slots, positions, num_pages):
     return cache, st, detail
 
 
-def gather_rows(pool: torch.Tensor, w, slots, r, row_bytes):
+def gather_rows(pool: torch.Tensor, w, slots, r, row_bytes, swizzled=True):
     """Bytes of each token's row per group: [n, G, row_bytes] (slot < 0 rows are zero)."""
-    host = pool.cpu().numpy().reshape(-1, w.groups, w.page_size, row_bytes)
+    host = pool.cpu().numpy().reshape(-1, w.groups, w.page_size * row_bytes)
     out = np.zeros((len(slots), w.groups, row_bytes), np.uint8)
+    cache = {}
     for i, s in enumerate(slots):
         if s >= 0:
-            out[i] = host[s // w.page_size, :, s % w.page_size]
+            for g in range(w.groups):
+                key = (s // w.page_size, g)
+                if key not in cache:
+                    img = host[key[0], g]
+                    cache[key] = unswizzle_block(img, w.page_size) if swizzled else \
+                        img.reshape(w.page_size, row_bytes)
+                out[i, g] = cache[key][s % w.page_size]
     return out
 
 
@@ -56,7 +64,7 @@ def make_slots(n, num_pages, page_size, seed, holes=True):
 @pytest.mark.parametrize("n", [1, 37, 200])
 def test_compress_small(dt, n):
     w = dataclasses.replace(WORKLOADS["tiny_f32"], act_dtype=dt, latent_dtype=dt, rank_k=64,
-                            rank_v=32, d_model=192)
+                            rank_v=128, d_model=192)
     x = normal_tensor(7, "x", (n, w.d_model), dt)
     A_k = normal_tensor(7, "A_k", (w.d_model, w.groups * w.rank_k), dt, 1 / math.sqrt(w.d_model))
     A_v = normal_tensor(7, "A_v", (w.d_model, w.groups * w.rank_v), dt, 1 / math.sqrt(w.d_model))
@@ -98,8 +106,8 @@ def exact_inputs(w, n, seed):
 @pytest.mark.parametrize("act", ["f16", "bf16"])
 def test_compress_int4_bit_exact(act):
     # exactly representable latents: quantisation codes, bytes and scales match bit for bit
-    w = dataclasses.replace(WORKLOADS["tiny_f32"], act_dtype=act, latent_dtype="int4", rank_k=64,
-                            rank_v=96, d_model=256)
+    w = dataclasses.replace(WORKLOADS["tiny_f32"], act_dtype=act, latent_dtype="int4", rank_k=256,
+                            rank_v=512, d_model=256)
     n = 150
     x, A_k, A_v = exact_inputs(w, n, 3)
     num_pages = 4
@@ -113,7 +121,7 @@ def test_compress_int4_bit_exact(act):
         packed, sc = O.quantize_int4(z.reshape(n, w.groups, r).astype(np.float32))
         srow = (2 * (r // 32) + 15) // 16 * 16
         got = gather_rows(pool, w, slots, r, r // 2)
-        got_s = gather_rows(spool, w, slots, r, srow)[..., : 2 * (r // 32)].copy().view(np.float16)
+        got_s = gather_rows(spool, w, slots, r, srow, swizzled=False)[..., : 2 * (r // 32)].copy().view(np.float16)
         keep = slots >= 0
         np.testing.assert_array_equal(got[keep], packed[keep])
         np.testing.assert_array_equal(got_s[keep], sc[keep])
@@ -122,8 +130,8 @@ def test_compress_int4_bit_exact(act):
 def test_compress_int4_general():
     # N(0,1) inputs: codes may differ from the oracle's only where float32
     # accumulation order moves a value across a rounding boundary
-    w = dataclasses.replace(WORKLOADS["tiny_f32"], act_dtype="f16", latent_dtype="int4", rank_k=64,
-                            rank_v=64, d_model=256)
+    w = dataclasses.replace(WORKLOADS["tiny_f32"], act_dtype="f16", latent_dtype="int4", rank_k=256,
+                            rank_v=256, d_model=256)
     n = 100
     x = normal_tensor(11, "x", (n, w.d_model), "f16")
     A_k = normal_tensor(11, "A_k", (w.d_model, w.groups * w.rank_k), "f16", 1 / 16)
@@ -133,12 +141,16 @@ def test_compress_int4_general():
     assert st == 0
     for pool, spool, A, r in ((cache.zk, cache.zks, A_k, w.rank_k), (cache.zv, cache.zvs, A_v, w.rank_v)):
         z = O.compress(x.to(torch.float64).numpy(), A.to(torch.float64).numpy(), None).reshape(n, w.groups, r)
-        srow = 16
+        srow = (2 * (r // 32) + 15) // 16 * 16
         got = gather_rows(pool, w, slots, r, r // 2)
-        got_s = gather_rows(spool, w, slots, r, srow)[..., : 2 * (r // 32)].copy().view(np.float16)
+        got_s = gather_rows(spool, w, slots, r, srow, swizzled=False)[..., : 2 * (r // 32)].copy().view(np.float16)
         deq = O.dequantize_int4(got, got_s, "f16")
         s_full = np.repeat(got_s.astype(np.float64), 32, axis=-1)
-        assert np.all(np.abs(deq - z) <= 0.5 * s_full * 1.001 + 1e-3 * s_full + 1e-6)
+        # quantisation step (s/2, s itself rounded to fp16), plus the fp16 rounding of
+        # the dequantised product code*s (half an ulp at |code*s| <= 7s), plus the
+        # float32 accumulation of x.A
+        bound = 0.5 * s_full * (1 + 2 ** -10) + 7 * s_full * 2 ** -11 + 1e-5 * (np.abs(z) + 1)
+        assert np.all(np.abs(deq - z) <= bound), float(np.max(np.abs(deq - z) / s_full))
         _, sc_ref = O.quantize_int4(z.astype(np.float32))
         assert np.all(np.abs(got_s.astype(np.float64) - sc_ref.astype(np.float64))
                       <= 2 ** -10 * np.abs(sc_ref.astype(np.float64)) + 1e-7)

@@ -41,7 +41,7 @@ def test_tiny_f32_config():
 
 @pytest.mark.parametrize("dt", ["f32", "f16", "bf16"])
 def test_ragged_batch_shuffled_pages(dt):
-    w = dataclasses.replace(WORKLOADS["tiny_f32"], act_dtype=dt, latent_dtype=dt, rank_k=64, rank_v=32)
+    w = dataclasses.replace(WORKLOADS["tiny_f32"], act_dtype=dt, latent_dtype=dt, rank_k=64, rank_v=64)
     case = make_decode_case(w, [1, 127, 128, 129, 300, 0, 1000])
     for s in (1, 3, 0):
         check_case(case, num_splits=s)

@@ -8,7 +8,8 @@ import pytest
 import torch
 
 from oracle import palu_oracle as O
-from palu_testlib import TOL, build_pools, make_decode_case, oracle_decode, rel_err, run_gpu_decode
+from palu_testlib import (TOL, build_pools, make_decode_case, oracle_decode, rel_err, run_gpu_decode,
+                          swizzle_block, unswizzle_block)
 from rank_kv_cache_palu_b200 import api as P
 from rank_kv_cache_palu_b200.synth import TORCH_DTYPE, WORKLOADS, normal, normal_tensor, page_permutation
 
@@ -99,9 +100,15 @@ def test_tc_nan_in_unused_page_rows_is_ignored():
     pools = build_pools(case)
     G, Pz = w.groups, w.page_size
     last_page = int(case.page_table[0, 1])
+    nan = np.frombuffer(np.array([np.nan], np.float32).astype(np.float32).tobytes()[2:], np.uint8)  # bf16 NaN
     for name, r in (("zk", w.rank_k), ("zv", w.rank_v)):
-        v = pools[name].view(torch.bfloat16).view(case.num_pages, G, Pz, r)
-        v[last_page, :, 200 - Pz:, :] = float("nan")
+        blocks = pools[name].view(case.num_pages, G, Pz * r * 2)
+        for g in range(G):
+            img = blocks[last_page, g].cpu().numpy()
+            rows = unswizzle_block(img, Pz).copy()
+            rows[200 - Pz:, 0::2] = nan[0]
+            rows[200 - Pz:, 1::2] = nan[1]
+            blocks[last_page, g] = torch.from_numpy(swizzle_block(rows)).cuda()
     out, _ = run_gpu_decode(case, 1, pools=pools)
     ref, _ = oracle_decode(case, 0)
     assert np.all(np.isfinite(out))
@@ -154,10 +161,13 @@ def sampled_full_size(w, context, units, seed=123, num_splits=0):
         for name, r, pool in (("zk", w.rank_k, cache.zk), ("zv", w.rank_v, cache.zv)):
             z = torch.from_numpy(normal(seed, name, (context, r), unit=(bi, g))).to(lat)
             host[(name, bi, g)] = z
-            view = pool.view(lat).view(num_pages, G, Pz, r)
+            blocks = pool.view(num_pages, G, Pz * r * 2)
+            zb = z.view(torch.uint8).numpy()
             for p in range(max_pages):
                 t0, t1 = p * Pz, min(context, (p + 1) * Pz)
-                view[pt[bi, p], g, : t1 - t0].copy_(z[t0:t1].to(dev))
+                rows = np.zeros((Pz, r * 2), np.uint8)
+                rows[: t1 - t0] = zb[t0:t1]
+                blocks[pt[bi, p], g].copy_(torch.from_numpy(swizzle_block(rows)).to(dev))
     q = normal_tensor(seed, "q", (b, w.num_heads, w.head_dim), w.act_dtype)
     B_k = normal_tensor(seed, "B_k", (G, w.rank_k, W), w.act_dtype, 1 / math.sqrt(w.rank_k))
     B_v = normal_tensor(seed, "B_v", (G, w.rank_v, W), w.act_dtype, 1 / math.sqrt(w.rank_v))

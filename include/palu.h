@@ -169,6 +169,41 @@ palu_status palu_decode_attn(const palu_config* cfg, int batch, const void* q, c
                              void* workspace, size_t workspace_bytes, int num_splits,
                              palu_stream_t stream);
 
+/* Allocation-free decode step (the paper has no counterpart: this is a
+ * deployment convenience of this library).
+ * Some callers cannot call cudaMalloc at all: plug-ins whose host framework
+ * owns all device memory and forbids further allocations, processes held to a
+ * fixed device-memory budget, or latency-critical paths that must not pay for
+ * an allocation (cudaMalloc can synchronise the device).  This entry point runs
+ * exactly palu_decode_attn, but keeps the workspace in a fixed array of device
+ * memory owned by the library: PALU_NOALLOC_SCRATCH_BYTES on every GPU that
+ * loads the library, held until the process exits.  The caller still passes
+ * every input and output.
+ *   - Calls whose workspace (palu_decode_workspace_size) exceeds the array
+ *     return PALU_ERR_WORKSPACE before launching anything.
+ *   - The first call on a device looks up the array's device address for that
+ *     device (cudaGetSymbolAddress, with that device current); make that first
+ *     call before any stream capture.
+ *   - Every call on a device shares the one array and leaves its contents
+ *     behind; each call clears the status word (an asynchronous memset on
+ *     `stream`) and rewrites all partials.  Calls that overlap on the GPU (on
+ *     different streams, or from different threads) race on the array: the
+ *     caller must order them.
+ *   - Nothing is allocated: no cudaMalloc, cudaFree or allocating library call.
+ *   - status_out NULL: asynchronous like palu_decode_attn; faults the kernels
+ *     detect are still skipped, but not reported.  status_out non-NULL: the
+ *     call waits for `stream`, returns the device status (PALU_OK,
+ *     PALU_ERR_DEVICE_TIMEOUT or PALU_ERR_DEVICE_BOUNDS) and stores the
+ *     kernel's detail code in *status_out (host memory). */
+#define PALU_NOALLOC_SCRATCH_BYTES (8u << 20)
+palu_status palu_decode_attn_noalloc(const palu_config* cfg, int batch, const void* q,
+                                     const int32_t* q_pos, const void* zk_pool, const void* zv_pool,
+                                     const void* zk_scales, const void* zv_scales,
+                                     const int32_t* pos_pool, const int32_t* page_table, int max_pages,
+                                     const int32_t* seq_lens, int num_pages, const void* B_k,
+                                     const void* B_v, void* out, float* lse, int num_splits,
+                                     palu_stream_t stream, int32_t* status_out);
+
 /* Synchronises `stream`, then reads and clears the device status word at the
  * start of `workspace`.  Returns PALU_OK, PALU_ERR_DEVICE_TIMEOUT or
  * PALU_ERR_DEVICE_BOUNDS; *detail (optional) receives the kernel's detail code. */

@@ -46,6 +46,10 @@ SIGNATURES = {
     "palu_decode_attn": (c_int, [_CFG, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                  c_void_p, c_void_p, c_void_p, c_int, c_void_p, c_int, c_void_p,
                                  c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_int, c_void_p]),
+    "palu_decode_attn_noalloc": (c_int, [_CFG, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                         c_void_p, c_void_p, c_void_p, c_int, c_void_p, c_int,
+                                         c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_void_p,
+                                         _P(c_int32)]),
     "palu_get_device_status": (c_int, [c_void_p, c_void_p, _P(c_int32)]),
     "palu_status_string": (ctypes.c_char_p, [c_int]),
     "palu_last_cuda_error": (ctypes.c_char_p, []),

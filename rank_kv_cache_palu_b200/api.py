@@ -133,6 +133,27 @@ def palu_decode_attn(cfg: PaluConfig, q, q_pos, zk_pool, zv_pool, zk_scales, zv_
     _check(st, "palu_decode_attn")
 
 
+NOALLOC_SCRATCH_BYTES = 8 << 20
+
+
+def palu_decode_attn_noalloc(cfg: PaluConfig, q, q_pos, zk_pool, zv_pool, zk_scales, zv_scales,
+                             pos_pool, page_table, seq_lens, num_pages: int, B_k, B_v, out, lse,
+                             num_splits: int = 0, stream=None, report_status: bool = False):
+    """palu_decode_attn without a caller workspace (the library's fixed device array).
+
+    report_status=True waits for the stream and raises on a device-detected fault.
+    """
+    batch = q.shape[0]
+    max_pages = page_table.shape[1]
+    detail = ctypes.c_int32()
+    st = load().palu_decode_attn_noalloc(
+        ctypes.byref(cfg), batch, _ptr(q), _ptr(q_pos), _ptr(zk_pool), _ptr(zv_pool),
+        _ptr(zk_scales), _ptr(zv_scales), _ptr(pos_pool), _ptr(page_table), max_pages,
+        _ptr(seq_lens), num_pages, _ptr(B_k), _ptr(B_v), _ptr(out), _ptr(lse), num_splits,
+        _stream(stream), ctypes.byref(detail) if report_status else None)
+    _check(st, "palu_decode_attn_noalloc")
+
+
 def palu_get_device_status(workspace, stream=None) -> tuple[int, int]:
     """(status, detail) of the device status word; clears it."""
     detail = ctypes.c_int32()

@@ -95,7 +95,9 @@ palu_status palu_cache_strides(const palu_config* cfg, size_t* k_page_bytes, siz
                                size_t* k_scale_page_bytes, size_t* v_scale_page_bytes);
 
 /* Workspace bytes palu_compress_append needs for n_tokens rows (status word +
- * any partial sums).  Always >= 256. */
+ * per-split partial sums and counters when the K range is split across CTAs).
+ * Always >= 256.  Zero-fill a workspace once before its first use; every call
+ * leaves its counters back at zero. */
 palu_status palu_compress_workspace_size(const palu_config* cfg, int n_tokens, int d_model,
                                          size_t* bytes);
 

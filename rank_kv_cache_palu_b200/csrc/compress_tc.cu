@@ -1,0 +1,386 @@
+// Tensor-core compress / append (sm_100a): z = x · A into the paged latent cache.
+//
+// Method: "PALU 论文低秩投影分解" §低秩投影分解 (z_k = x A_k, z_v = x A_v) and
+// §把它放进一次真实推理流程里看, Prefill 阶段 (compute the latents and cache them).
+//
+// The GEMM runs transposed: D[128 latent columns × NT tokens] = Aᵀ · xᵀ, so the
+// TMEM lane of an epilogue thread is one latent column and its TMEM columns are
+// tokens.  A thread then writes its column of every token straight into the
+// paged, swizzled cache, and for int4 the 32 lanes of a warp are exactly one
+// 32-entry quantisation block (max by warp shuffle).
+//
+// Prefill (many tokens): one CTA per (column tile, 256-token tile), full K.
+// Append (a few tokens per decode step): the whole step is one token tile and
+// the K range is split across CTAs so the weight matrix streams from every SM;
+// each split writes its fp32 partial to the workspace and the last split of a
+// column tile (atomic counter) sums them and runs the epilogue.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "palu_common.cuh"
+#include "palu_internal.h"
+#include "palu_tc.h"
+#include "tc_ptx.cuh"
+
+namespace palu {
+namespace {
+
+using namespace tc;
+
+constexpr int kThreads = 192;           // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+constexpr int kM = 128;                 // latent columns per tile
+constexpr int kKStage = 64;             // K rows per stage
+constexpr int kABytes = kM * kKStage * 2;  // 16 KB: two 64-column MN-major boxes
+
+struct Plan {
+  int NT;       // tokens per tile (multiple of 16, <= 256)
+  int ntt;      // token tiles
+  int tk, tv;   // column tiles of A_k and A_v
+  int KS;       // K splits
+  int stages;
+  size_t counter_bytes, partial_bytes;
+};
+
+Plan make_plan(int n, int d_model, int G, int r_k, int r_v) {
+  Plan p{};
+  p.NT = n <= 256 ? ((n + 15) / 16) * 16 : 256;
+  p.ntt = (n + p.NT - 1) / p.NT;
+  p.tk = (G * r_k + kM - 1) / kM;
+  p.tv = (G * r_v + kM - 1) / kM;
+  const int tiles = (p.tk + p.tv) * p.ntt;
+  const int kst = d_model / kKStage;
+  int ks = 1;
+  if (p.ntt == 1) {
+    ks = (2 * 148 + tiles - 1) / tiles;
+    if (ks > kst / 2) ks = kst / 2;   // at least two stages per split
+    if (ks > 16) ks = 16;
+    if (ks < 1) ks = 1;
+  }
+  p.KS = ks;
+  const int stage_bytes = kABytes + p.NT * 128;
+  p.stages = (200 * 1024) / stage_bytes;
+  if (p.stages > 8) p.stages = 8;
+  if (p.stages < 2) p.stages = 2;
+  p.counter_bytes = p.KS > 1 ? ((size_t)tiles * sizeof(int) + 255) / 256 * 256 : 0;
+  p.partial_bytes = p.KS > 1 ? (size_t)p.KS * tiles * kM * p.NT * sizeof(float) : 0;
+  return p;
+}
+
+struct TcArgs {
+  CompressArgs a;
+  Plan p;
+  int* counters;
+  float* partials;
+};
+
+// Write one latent column `j` (of group g) for token row i of the tile.
+template <int LAT>
+__device__ __forceinline__ void store_latent(const CompressArgs& a, uint8_t* pool, long long row_bytes, int g,
+                                             int j, int slot, float v) {
+  using TL = typename Dt<LAT>::T;
+  const long long pgb = (long long)(slot / a.P) * a.G + g;
+  *reinterpret_cast<TL*>(pool + pgb * a.P * row_bytes + swz_offset(slot % a.P, (long long)j * sizeof(TL), a.P)) =
+      Dt<LAT>::from_f(v);
+}
+
+template <int ACT, int LAT>
+__global__ void __launch_bounds__(kThreads, 1)
+    compress_tc_kernel(const __grid_constant__ CUtensorMap tm_ak, const __grid_constant__ CUtensorMap tm_av,
+                       const __grid_constant__ CUtensorMap tm_x, const TcArgs t) {
+  extern __shared__ uint8_t smem_raw[];
+  const CompressArgs& a = t.a;
+  const Plan& p = t.p;
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* sbase = smem_raw + (base - raw);
+  const int stage_bytes = kABytes + p.NT * 128;
+  const uint32_t bars = base + (uint32_t)p.stages * stage_bytes;      // 2·stages + 2 barriers
+  uint8_t* misc = sbase + (uint32_t)p.stages * stage_bytes + 256;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 16);
+  int* last_flag = reinterpret_cast<int*>(misc + 32);
+  auto full = [&](int s) { return bars + 8u * s; };
+  auto empty = [&](int s) { return bars + 8u * (p.stages + s); };
+  const uint32_t d_full = bars + 8u * (2 * p.stages);
+  const uint32_t epi_bar = d_full + 8;
+  DevStatus* st = reinterpret_cast<DevStatus*>(a.status);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // tile coordinates
+  const bool is_v = blockIdx.x >= p.tk;
+  const int ctile = is_v ? blockIdx.x - p.tk : blockIdx.x;
+  const int c0 = ctile * kM;
+  const int r = is_v ? a.r_v : a.r_k;
+  const int ncols = a.G * r;
+  const int t0 = blockIdx.y * p.NT;
+  const int kst = a.d_model / kKStage;
+  const int split = blockIdx.z;
+  const int ks0 = (int)((long long)kst * split / p.KS), ks1 = (int)((long long)kst * (split + 1) / p.KS);
+  const CUtensorMap* tm_a = is_v ? &tm_av : &tm_ak;
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    for (int s = 0; s < p.stages; ++s) {
+      mbar_init(full(s), 1);
+      mbar_init(empty(s), 1);
+    }
+    mbar_init(d_full, 1);
+    mbar_init(epi_bar, 4);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tmap(tm_a);
+      prefetch_tmap(&tm_x);
+      int s = 0;
+      uint32_t ph = 0;
+      for (int kb = ks0; kb < ks1 && !*abort_flag; ++kb) {
+        if (!mbar_wait(empty(s), ph ^ 1, abort_flag, st, 50)) break;
+        mbar_expect_tx(full(s), (uint32_t)stage_bytes);
+        const uint32_t dst = base + (uint32_t)s * stage_bytes;
+        tma_load_2d(dst, tm_a, c0, kb * kKStage, full(s));
+        tma_load_2d(dst + kABytes / 2, tm_a, c0 + 64, kb * kKStage, full(s));
+        tma_load_2d(dst + kABytes, &tm_x, kb * kKStage, t0, full(s));
+        if (++s == p.stages) { s = 0; ph ^= 1; }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr int kBf = ACT == PALU_BF16 ? 1 : 0;
+      const uint32_t idesc = idesc_f16(kBf, 1, 0, p.NT, kM);    // Aᵀ MN-major, xᵀ K-major
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int kb = ks0; kb < ks1; ++kb) {
+        if (!mbar_wait(full(s), ph, abort_flag, st, 51)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t sa = base + (uint32_t)s * stage_bytes;
+        const uint32_t sx = sa + kABytes;
+#pragma unroll
+        for (int kk = 0; kk < kKStage / 16; ++kk) {
+          const uint64_t ad = sdesc(sa + kk * 16 * 128, kABytes / 2, 1024, kSw128);
+          const uint64_t bd = sdesc(sx + kk * 32, 16, 1024, kSw128);
+          umma_f16(tmem, ad, bd, idesc, (kb > ks0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(empty(s));
+        if (++s == p.stages) { s = 0; ph ^= 1; }
+      }
+      (void)ok;
+      umma_commit(d_full);   // also drains: fires once every MMA above has completed
+    }
+  } else {
+    // ============================================================ epilogue (warps 2-5)
+    const int q4 = warp & 3;
+    const int c = q4 * 32 + lane;            // latent column of this thread within the tile
+    const int gc = c0 + c;
+    const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
+    uint32_t epi_phase = 0;
+    auto ep_sync = [&](int where) -> bool {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(epi_bar);
+      const bool rr = mbar_wait(epi_bar, epi_phase, abort_flag, st, where);
+      epi_phase ^= 1;
+      return rr;
+    };
+    bool ok = mbar_wait(d_full, 0, abort_flag, st, 52);
+    tc_fence_after();
+    const int tile_id = blockIdx.x * p.ntt + blockIdx.y;
+    const int tiles = (p.tk + p.tv) * p.ntt;
+    bool finalize = true;
+    float* my_part = nullptr;
+    if (p.KS > 1) {
+      // publish this split's partial, then find out whether this CTA closes the tile
+      my_part = t.partials + ((size_t)split * tiles + tile_id) * kM * p.NT + (size_t)c * p.NT;
+      for (int j0 = 0; ok && j0 < p.NT; j0 += 16) {
+        float v[16];
+        tmem_ld16(tmem + lane_addr + j0, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int u = 0; u < 16; u += 4)
+          *reinterpret_cast<float4*>(my_part + j0 + u) = make_float4(v[u], v[u + 1], v[u + 2], v[u + 3]);
+      }
+      __threadfence();
+      ok = ep_sync(53) && ok;
+      if (threadIdx.x == 64) {
+        const int prev = atomicAdd(t.counters + tile_id, 1);
+        *last_flag = (prev == p.KS - 1);
+      }
+      ok = ep_sync(54) && ok;
+      finalize = *last_flag != 0;
+      if (finalize) __threadfence();
+    }
+    if (ok && finalize) {
+      uint8_t* pool = reinterpret_cast<uint8_t*>(is_v ? a.zv : a.zk);
+      const long long row_bytes = is_v ? a.v_row : a.k_row;
+      const long long cap = (long long)a.num_pages * a.P;
+      const int g = gc / r, j = gc % r;
+      const bool col_ok = gc < ncols;
+      const int ntok = min(p.NT, a.n - t0);
+      for (int j0 = 0; j0 < ntok; j0 += 16) {
+        float v[16];
+        if (p.KS == 1) {
+          tmem_ld16(tmem + lane_addr + j0, v);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int u = 0; u < 16; ++u) v[u] = 0.f;
+          for (int sp = 0; sp < p.KS; ++sp) {
+            const float* src = t.partials + ((size_t)sp * tiles + tile_id) * kM * p.NT + (size_t)c * p.NT + j0;
+#pragma unroll
+            for (int u = 0; u < 16; u += 4) {
+              const float4 f = __ldcg(reinterpret_cast<const float4*>(src + u));
+              v[u] += f.x;
+              v[u + 1] += f.y;
+              v[u + 2] += f.z;
+              v[u + 3] += f.w;
+            }
+          }
+        }
+#pragma unroll 1
+        for (int u = 0; u < 16; ++u) {
+          const int ti = t0 + j0 + u;
+          if (j0 + u >= ntok) break;
+          const int slot = a.slots[ti];
+          if (slot < 0) continue;
+          if (slot >= cap) {
+            if (col_ok && c == 0) report(st, PALU_ERR_DEVICE_BOUNDS, 3000000 + ti);
+            continue;
+          }
+          if constexpr (LAT == PALU_INT4) {
+            // the warp's 32 columns are one quantisation block of this token
+            float amax = col_ok ? fabsf(v[u]) : 0.f;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+            const __half s16 = __float2half_rn(__fdiv_rn(amax, 7.0f));
+            const float s = __half2float(s16);
+            int code = 0;
+            if (s != 0.f) code = (int)fminf(fmaxf(rintf(__fdiv_rn(v[u], s)), -7.f), 7.f);
+            const int hi = __shfl_down_sync(0xffffffffu, code, 1);
+            if (col_ok && (lane & 1) == 0) {
+              const long long pgb = (long long)(slot / a.P) * a.G + g;
+              pool[pgb * a.P * row_bytes + swz_offset(slot % a.P, j >> 1, a.P)] =
+                  (uint8_t)((code & 0xF) | ((hi & 0xF) << 4));
+            }
+            if (col_ok && lane == 0) {
+              uint8_t* spool = reinterpret_cast<uint8_t*>(is_v ? a.zvs : a.zks);
+              const long long srow = is_v ? a.vs_row : a.ks_row;
+              const long long prow = ((long long)(slot / a.P) * a.G + g) * a.P + slot % a.P;
+              reinterpret_cast<__half*>(spool + prow * srow)[j >> 5] = s16;
+            }
+          } else {
+            if (col_ok) store_latent<LAT>(a, pool, row_bytes, g, j, slot, v[u]);
+          }
+        }
+      }
+      // positions, once per token
+      if (!is_v && ctile == 0 && a.positions != nullptr && a.pos_pool != nullptr) {
+        for (int i = c; i < ntok; i += kM) {
+          const int slot = a.slots[t0 + i];
+          if (slot >= 0 && slot < cap) a.pos_pool[slot] = a.positions[t0 + i];
+        }
+      }
+      if (p.KS > 1 && threadIdx.x == 64) t.counters[tile_id] = 0;   // reusable for the next call
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* ptr = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+bool map2d(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, uint64_t inner, uint64_t outer,
+           uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int ACT, int LAT>
+cudaError_t launch_t(const CompressArgs& a, cudaStream_t st) {
+  const Plan p = make_plan(a.n, a.d_model, a.G, a.r_k, a.r_v);
+  const CUtensorMapDataType dt = ACT == PALU_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  CUtensorMap tm_ak, tm_av, tm_x;
+  if (!map2d(&tm_ak, a.Ak, dt, (uint64_t)a.G * a.r_k, a.d_model, (uint64_t)a.G * a.r_k * 2, 64, kKStage) ||
+      !map2d(&tm_av, a.Av, dt, (uint64_t)a.G * a.r_v, a.d_model, (uint64_t)a.G * a.r_v * 2, 64, kKStage) ||
+      !map2d(&tm_x, a.x, dt, a.d_model, a.n, (uint64_t)a.d_model * 2, 64, p.NT))
+    return cudaErrorInvalidValue;
+  TcArgs t{};
+  t.a = a;
+  t.p = p;
+  uint8_t* scratch = reinterpret_cast<uint8_t*>(a.scratch);
+  t.counters = reinterpret_cast<int*>(scratch);
+  t.partials = reinterpret_cast<float*>(scratch + p.counter_bytes);
+  const size_t smem = (size_t)p.stages * (kABytes + p.NT * 128) + 256 + 64 + 1024;
+  auto kern = compress_tc_kernel<ACT, LAT>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(p.tk + p.tv, p.ntt, p.KS);
+  kern<<<grid, kThreads, smem, st>>>(tm_ak, tm_av, tm_x, t);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool tc_compress_supported(const palu_config* c, int n_tokens, int d_model) {
+  if (c->act_dtype != PALU_F16 && c->act_dtype != PALU_BF16) return false;
+  if (c->latent_dtype != c->act_dtype && c->latent_dtype != PALU_INT4) return false;
+  if (d_model % kKStage != 0 || d_model < 2 * kKStage) return false;
+  if (n_tokens <= 0) return false;
+  const int G = c->num_heads / c->group_size;
+  if ((G * c->rank_k) % 8 != 0 || (G * c->rank_v) % 8 != 0) return false;
+  if (c->latent_dtype == PALU_INT4 && (c->rank_k % 32 != 0 || c->rank_v % 32 != 0)) return false;
+  return true;
+}
+
+size_t tc_compress_scratch_bytes(const palu_config* c, int n_tokens, int d_model) {
+  if (!tc_compress_supported(c, n_tokens, d_model)) return 0;
+  const int G = c->num_heads / c->group_size;
+  const Plan p = make_plan(n_tokens, d_model, G, c->rank_k, c->rank_v);
+  return p.counter_bytes + p.partial_bytes;
+}
+
+cudaError_t launch_compress_tc(const CompressArgs& a, cudaStream_t st) {
+  if (a.act == PALU_BF16) {
+    if (a.lat == PALU_INT4) return launch_t<PALU_BF16, PALU_INT4>(a, st);
+    return launch_t<PALU_BF16, PALU_BF16>(a, st);
+  }
+  if (a.lat == PALU_INT4) return launch_t<PALU_F16, PALU_INT4>(a, st);
+  return launch_t<PALU_F16, PALU_F16>(a, st);
+}
+
+}  // namespace palu

@@ -166,3 +166,67 @@ def test_compress_bad_slot_reports_bounds():
     slots[3] = 10 ** 6
     _, st, _ = run_compress(w, x, A_k, A_v, slots, None, 1)
     assert st == 7
+
+
+def _check_rows(w, x, A, pool, slots, rows, r, dt):
+    """Oracle z for the sampled token rows vs the cache contents of those tokens."""
+    esz = 2
+    got = as_values(gather_rows(pool, w, slots[rows], r, r * esz), dt)
+    ref = O.compress(x[rows].to(torch.float64).numpy(), A.to(torch.float64).numpy(), dt)
+    ref = ref.reshape(len(rows), w.groups, r)
+    tol = {"f16": 2 ** -10, "bf16": 2 ** -7}[dt]
+    err = np.abs(got - ref)
+    assert np.all(err <= tol * np.abs(ref) + 1e-6 * np.max(np.abs(ref))), float(err.max())
+
+
+@pytest.mark.parametrize("dt", ["bf16", "f16"])
+def test_compress_prefill_multi_tile(dt):
+    # several 256-token tiles and a ragged last one (no K split)
+    w = dataclasses.replace(WORKLOADS["7b_bf16_r256v128_b1_t4k"], act_dtype=dt, latent_dtype=dt,
+                            num_heads=8, d_model=512)
+    n = 600
+    x = normal_tensor(21, "x", (n, w.d_model), dt)
+    A_k = normal_tensor(21, "A_k", (w.d_model, w.groups * w.rank_k), dt, 1 / math.sqrt(w.d_model))
+    A_v = normal_tensor(21, "A_v", (w.d_model, w.groups * w.rank_v), dt, 1 / math.sqrt(w.d_model))
+    num_pages = 8
+    slots = make_slots(n, num_pages, w.page_size, seed=21)
+    cache, st, _ = run_compress(w, x, A_k, A_v, slots, None, num_pages)
+    assert st == 0
+    rows = np.flatnonzero(slots >= 0)
+    _check_rows(w, x, A_k, cache.zk, slots, rows, w.rank_k, dt)
+    _check_rows(w, x, A_v, cache.zv, slots, rows, w.rank_v, dt)
+
+
+@pytest.mark.slow
+def test_compress_prefill_full_size_sampled():
+    # 8192 tokens of a 7B layer, x [8192 x 4096] bf16 into rank 256/256 latents; sampled tokens
+    w = WORKLOADS["7b_bf16_r256_b32_t16k"]
+    n = 8192
+    x = normal_tensor(5, "x", (n, w.d_model), "bf16")
+    A_k = normal_tensor(5, "A_k", (w.d_model, w.groups * w.rank_k), "bf16", 1 / math.sqrt(w.d_model))
+    A_v = normal_tensor(5, "A_v", (w.d_model, w.groups * w.rank_v), "bf16", 1 / math.sqrt(w.d_model))
+    num_pages = n // w.page_size + 1
+    slots = np.random.default_rng(5).permutation(num_pages * w.page_size)[:n].astype(np.int32)
+    cache, st, _ = run_compress(w, x, A_k, A_v, slots, None, num_pages)
+    assert st == 0
+    rows = np.random.default_rng(6).choice(n, size=48, replace=False)
+    rows = np.concatenate([rows, [0, 255, 256, n - 1]])
+    _check_rows(w, x, A_k, cache.zk, slots, rows, w.rank_k, "bf16")
+    _check_rows(w, x, A_v, cache.zv, slots, rows, w.rank_v, "bf16")
+
+
+def test_compress_append_step_full_size():
+    # the per-step append of a decode batch: 32 tokens of a 7B layer (K split across CTAs)
+    w = WORKLOADS["7b_bf16_r256v128_b16_t16k"]
+    n = 32
+    x = normal_tensor(9, "x", (n, w.d_model), "bf16")
+    A_k = normal_tensor(9, "A_k", (w.d_model, w.groups * w.rank_k), "bf16", 1 / math.sqrt(w.d_model))
+    A_v = normal_tensor(9, "A_v", (w.d_model, w.groups * w.rank_v), "bf16", 1 / math.sqrt(w.d_model))
+    num_pages = 40
+    slots = make_slots(n, num_pages, w.page_size, seed=9)
+    for _ in range(2):                       # twice: the split counters must come back to zero
+        cache, st, _ = run_compress(w, x, A_k, A_v, slots, None, num_pages)
+        assert st == 0
+    rows = np.flatnonzero(slots >= 0)
+    _check_rows(w, x, A_k, cache.zk, slots, rows, w.rank_k, "bf16")
+    _check_rows(w, x, A_v, cache.zv, slots, rows, w.rank_v, "bf16")

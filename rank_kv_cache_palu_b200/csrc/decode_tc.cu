@@ -11,7 +11,10 @@
 // pages, 128 tokens (one page) per tile:
 //   warp 0  TMA producer: B_k for the two heads once (MN-major, 128-byte
 //           swizzle, resident), then the z_k page in 64-wide K chunks.
-//   warp 10 TMA producer for z_v (its own ring, so neither stream waits on the other).
+//   warp 2  bulk-copy producer for z_v (its own ring, so neither stream waits on the other).
+//   int4 latents: warps 0 and 3 dequantise z_k and warp 2 z_v into the same
+//           rings instead (code × fp16 scale, rounded to the compute dtype),
+//           so the MMAs below are the same for every latent dtype.
 //   warp 1  MMA issuer: D[128 tok × 256] = z_k · B_k[:, 2 heads] into one of two
 //           TMEM slots (kind::f16, fp32 accumulate); then aᵀ[r_v × 16] =
 //           z_vᵀ · Pᵀ for the previous tile into the drained slot.
@@ -151,6 +154,56 @@ __device__ __forceinline__ float from_bits(uint16_t u) {
   }
 }
 
+// ---------------------------------------------------------------- int4 latents
+// Sixteen bytes of a latent row = the 32 codes of one scale block.  Word m
+// holds entries 8m..8m+7, entry e in bits 4e..4e+3 (two's complement; the even
+// entry of each byte in its low nibble).  dequant8 turns one word into the 8
+// values code × s rounded to the compute dtype, as one 16-byte unit of the
+// shared-memory operand.
+__device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+__device__ __forceinline__ __half2 bits_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
+
+template <int ACT>
+__device__ __forceinline__ uint4 dequant8(uint32_t x, uint16_t sbits) {
+  uint4 o;
+  if constexpr (ACT == PALU_F16) {
+    // (code + 8) | 0x6400 is the half 1024 + code + 8: subtracting 1032 gives
+    // the code exactly, and one half multiply rounds code × s once.
+    const uint32_t r0 = (x & 0x000F000Fu) ^ 0x64086408u;           // entries 0, 4
+    const uint32_t r1 = ((x >> 4) & 0x000F000Fu) ^ 0x64086408u;    // 1, 5
+    const uint32_t r2 = ((x >> 8) & 0x000F000Fu) ^ 0x64086408u;    // 2, 6
+    const uint32_t r3 = ((x >> 12) & 0x000F000Fu) ^ 0x64086408u;   // 3, 7
+    const __half2 bias = bits_h2(0x64086408u);
+    const __half sh = __ushort_as_half(sbits);
+    const __half2 s2 = __halves2half2(sh, sh);
+    o.x = h2_bits(__hmul2(__hsub2(bits_h2(__byte_perm(r0, r1, 0x5410)), bias), s2));
+    o.y = h2_bits(__hmul2(__hsub2(bits_h2(__byte_perm(r2, r3, 0x5410)), bias), s2));
+    o.z = h2_bits(__hmul2(__hsub2(bits_h2(__byte_perm(r0, r1, 0x7632)), bias), s2));
+    o.w = h2_bits(__hmul2(__hsub2(bits_h2(__byte_perm(r2, r3, 0x7632)), bias), s2));
+  } else {
+    // (code + 8) | 0x4B000000 is the float 2^23 + code + 8; code × s is exact
+    // in fp32 and the pack rounds it to bf16 once.
+    const float s = __half2float(__ushort_as_half(sbits));
+    float v[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      v[e] = (__int_as_float(((x >> (4 * e)) & 0xFu) ^ 0x4B000008u) - 8388616.0f) * s;
+    uint32_t w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+      w[e] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    o = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  return o;
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
 // Phase trace record (palu_debug_trace).
 __device__ __forceinline__ void trace_record(const DecodeArgs& a, int ev, int k, long long t_start) {
   if (k >= a.trace_tiles) return;
@@ -158,7 +211,7 @@ __device__ __forceinline__ void trace_record(const DecodeArgs& a, int ev, int k,
   a.trace[(cta * 8 + ev) * a.trace_tiles + k] = clock64() - t_start;
 }
 
-template <int ACT, int NRV>
+template <int ACT, int NRV, int LAT>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tm_bk, const DecodeArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -167,6 +220,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sbase = smem_raw + (base - raw);
   const Smem L = smem_layout(a.r_k);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr bool kInt4 = LAT == PALU_INT4;
+  static_assert(!kInt4 || NRV == 2, "int4 latents: r_v = 256");
   DevStatus* st = reinterpret_cast<DevStatus*>(a.status);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sbase + L.abort);
   auto bar = [&](int i) { return base + L.bars + 8u * i; };
@@ -186,7 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     mbar_init(bar(BAR_B), 1);
     for (int i = 0; i < kNKS; ++i) {
-      mbar_init(bar(BAR_ZK_FULL + i), 1);
+      mbar_init(bar(BAR_ZK_FULL + i), kInt4 ? 2 : 1);   // int4: one arrival per dequantising warp
       mbar_init(bar(BAR_ZK_EMPTY + i), 1);
     }
     for (int i = 0; i < kNVS; ++i) {
@@ -223,12 +278,121 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sbase + L.tmem_slot);
 
-  if (warp == 0) {
-    // ============================================================ z_k producer
+  if (warp == 0 && lane == 0) {
+    mbar_expect_tx(bar(BAR_B), (uint32_t)a.r_k * 256 * 2);
+    for (int nb = 0; nb < 4; ++nb)
+      tma_load_2d(base + L.b + (uint32_t)nb * a.r_k * 128, &tm_bk, hp * 256 + nb * 64, g * a.r_k, bar(BAR_B));
+  }
+  if (kInt4 && (warp == 0 || warp == 2 || warp == 3)) {
+    {
+      // ============================================================ int4 dequantising producers
+      // z_k (warps 0, 3): chunk c of a tile = entries [64c, 64c + 64) of all 128
+      // tokens, i.e. scale blocks 2c and 2c+1.  Thread zt takes block 2c + (zt & 1)
+      // of tokens zt/2 + 32i.  z_v (warp 2): ring stage (mb, th) = entries
+      // [128mb, 128mb + 128) of tokens [64th, 64th + 64), in two steps of 32
+      // tokens; lane takes block 4mb + lane/8 of tokens 64th + lane%8 + 8i.
+      // Loads run two steps ahead of the conversion (three register slots).
+      const bool is_k = warp != 2;
+      const int zt = (warp == 3 ? 32 : 0) + lane;
+      const int nv_tiles = tr.ntiles - (tr.ragged_last ? 1 : 0);
+      const int N = is_k ? tr.ntiles * 4 : nv_tiles * 8;
+      const uint8_t* pool = reinterpret_cast<const uint8_t*>(is_k ? a.zk : a.zv);
+      const uint8_t* spool = reinterpret_cast<const uint8_t*>(is_k ? a.zks : a.zvs);
+      const long long srow_bytes = is_k ? a.ks_row : a.vs_row;
+      struct Slot {
+        uint4 raw[4];
+        uint16_t sc[4];
+      };
+      auto issue = [&](int n, Slot& sl) {
+        if (n >= N) return;
+        const int k = is_k ? (n >> 2) : (n >> 3);
+        int pg = page_of(a, b, tr.t_begin / kTile + k);
+        if (pg < 0) {
+          if (is_k && (n & 3) == 0 && zt == 0) report(st, PALU_ERR_DEVICE_BOUNDS, 2000000 + b);
+          pg = 0;   // keep the pipeline fed from a valid page; the status says the result is void
+        }
+        if (is_k && (n & 3) == 0 && zt == 0 && k + kPrefetch < tr.ntiles) {
+          // pull a later page of this split into L2 while this one converts
+          const int ppg = page_of(a, b, tr.t_begin / kTile + k + kPrefetch);
+          if (ppg >= 0) {
+            const size_t prow = (size_t)(ppg * a.G + g) * a.P;
+            prefetch_l2(reinterpret_cast<const uint8_t*>(a.zk) + prow * a.k_row, (uint32_t)(a.P * a.k_row));
+            prefetch_l2(reinterpret_cast<const uint8_t*>(a.zks) + prow * a.ks_row, (uint32_t)(a.P * a.ks_row));
+            prefetch_l2(reinterpret_cast<const uint8_t*>(a.zv) + prow * a.v_row, (uint32_t)(a.P * a.v_row));
+            prefetch_l2(reinterpret_cast<const uint8_t*>(a.zvs) + prow * a.vs_row, (uint32_t)(a.P * a.vs_row));
+          }
+        }
+        const size_t row0 = (size_t)(pg * a.G + g) * a.P;
+        const uint8_t* blk = pool + row0 * 128;
+        const uint8_t* sblk = spool + row0 * srow_bytes;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          int t, u;
+          if (is_k) {
+            t = (zt >> 1) + 32 * i;
+            u = 2 * (n & 3) + (zt & 1);
+          } else {
+            const int sidx = n & 7;   // (mb, th, half) of this tile
+            t = 64 * ((sidx >> 1) & 1) + (lane & 7) + 8 * (4 * (sidx & 1) + i);
+            u = 4 * (sidx >> 2) + (lane >> 3);
+          }
+          sl.raw[i] = __ldg(reinterpret_cast<const uint4*>(blk + t * 128 + ((u ^ (t & 7)) << 4)));
+          sl.sc[i] = __ldg(reinterpret_cast<const unsigned short*>(sblk + t * srow_bytes + 2 * u));
+        }
+      };
+      int stage = 0;
+      uint32_t phase = 0;
+      auto consume = [&](int n, const Slot& sl) -> bool {
+        if (n >= N) return true;
+        const int nst = is_k ? kNKS : kNVS;
+        const int first = is_k || (n & 1) == 0;
+        const int last = is_k || (n & 1) == 1;
+        const int ebar = is_k ? BAR_ZK_EMPTY : BAR_ZV_EMPTY;
+        const int fbar = is_k ? BAR_ZK_FULL : BAR_ZV_FULL;
+        if (first && !mbar_wait(bar(ebar + stage), phase ^ 1, abort_flag, st, is_k ? 12 : 13)) return false;
+        const uint32_t dst = base + (is_k ? L.zk + stage * kZkBytes : L.zv + stage * kZvBytes);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t w[4] = {sl.raw[i].x, sl.raw[i].y, sl.raw[i].z, sl.raw[i].w};
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            const uint4 o = dequant8<ACT>(w[m], sl.sc[i]);
+            uint32_t off;
+            if (is_k) {
+              const int t = (zt >> 1) + 32 * i;
+              off = t * 128 + (((4 * (zt & 1) + m) ^ (t & 7)) << 4);
+            } else {
+              const int tl = (lane & 7) + 8 * (4 * (n & 1) + i);   // token within the 64 of the stage
+              const int ul = lane >> 3;
+              off = (ul >> 1) * 8192 + tl * 128 + (((4 * (ul & 1) + m) ^ (lane & 7)) << 4);
+            }
+            st_shared_v4(dst + off, o);
+          }
+        }
+        if (last) {
+          fence_proxy_async();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(fbar + stage));
+          if (is_k && zt == 0 && (n & 3) == 0) trace(6, n >> 2);
+          if (++stage == nst) { stage = 0; phase ^= 1; }
+        }
+        return true;
+      };
+      Slot s0, s1, s2;
+      issue(0, s0);
+      issue(1, s1);
+      for (int n = 0; n < N && !*abort_flag; n += 3) {
+        issue(n + 2, s2);
+        if (!consume(n, s0)) break;
+        issue(n + 3, s0);
+        if (!consume(n + 1, s1)) break;
+        issue(n + 4, s1);
+        if (!consume(n + 2, s2)) break;
+      }
+    }
+  } else if (warp == 0) {
+    // ============================================================ z_k producer (bulk copies)
     if (lane == 0) {
-      mbar_expect_tx(bar(BAR_B), (uint32_t)a.r_k * 256 * 2);
-      for (int nb = 0; nb < 4; ++nb)
-        tma_load_2d(base + L.b + (uint32_t)nb * a.r_k * 128, &tm_bk, hp * 256 + nb * 64, g * a.r_k, bar(BAR_B));
       int stage = 0;
       uint32_t phase = 0;
       // Pull the next pages of this split into L2 ahead of the TMA loads: the
@@ -265,7 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == 2) {
-    // ============================================================ z_v producer
+    // ============================================================ z_v producer (bulk copies)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
@@ -615,19 +779,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int t0 = tr.t_begin + kl * kTile;
           const int nvalid = tr.t_end - t0;
           const int pg = page_of(a, b, t0 / kTile);
-          using TL = typename Dt<ACT>::T;
           float at[NRV];
 #pragma unroll
           for (int mb = 0; mb < NRV; ++mb) at[mb] = 0.f;
           if (pg >= 0) {
-            const uint8_t* zv = reinterpret_cast<const uint8_t*>(a.zv) + (size_t)(pg * a.G + g) * a.P * a.v_row;
+            const size_t row0 = (size_t)(pg * a.G + g) * a.P;
+            const uint8_t* zv = reinterpret_cast<const uint8_t*>(a.zv) + row0 * a.v_row;
+            const uint8_t* zvs = kInt4 ? reinterpret_cast<const uint8_t*>(a.zvs) + row0 * a.vs_row : nullptr;
             const uint8_t* pbuf = sbase + L.p + (kl & 1) * kPBytes;
             for (int t = 0; t < nvalid; ++t) {
               const float pv = from_bits<ACT>(*reinterpret_cast<const uint16_t*>(pbuf + p_offset(hw, t)));
+              const uint8_t* srow = kInt4 ? zvs + (size_t)t * a.vs_row : nullptr;
 #pragma unroll
               for (int mb = 0; mb < NRV; ++mb)
-                at[mb] = fmaf(pv, Dt<ACT>::to_f(*reinterpret_cast<const TL*>(
-                                      zv + swz_offset(t, (long long)(mb * 128 + row) * 2, a.P))), at[mb]);
+                at[mb] = fmaf(pv, load_latent<LAT, ACT>(zv, t, a.P, srow, mb * 128 + row), at[mb]);
             }
           }
 #pragma unroll
@@ -695,7 +860,7 @@ bool make_map_2d(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, int el
   return r == CUDA_SUCCESS;
 }
 
-template <int ACT, int NRV>
+template <int ACT, int NRV, int LAT>
 cudaError_t launch_t(const DecodeArgs& a, cudaStream_t st) {
   const CUtensorMapDataType dt = ACT == PALU_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   CUtensorMap tm_bk;
@@ -704,7 +869,7 @@ cudaError_t launch_t(const DecodeArgs& a, cudaStream_t st) {
     return cudaErrorInvalidValue;
   const Smem L = smem_layout(a.r_k);
   const size_t smem = L.total + 1024;
-  auto kern = decode_tc_kernel<ACT, NRV>;
+  auto kern = decode_tc_kernel<ACT, NRV, LAT>;
   DecodeArgs args = a;
   const TraceSetting ts = trace_setting();
   const size_t ctas = (size_t)a.S * a.G * (a.gs / 2) * a.batch;
@@ -726,9 +891,14 @@ bool tc_decode_supported(const palu_config* c) {
   if (c->head_dim != 128 || c->page_size != kTile) return false;
   if (c->group_size % 2 != 0) return false;
   if (c->act_dtype != PALU_F16 && c->act_dtype != PALU_BF16) return false;
-  if (c->latent_dtype != c->act_dtype) return false;
-  if (c->rank_k % 64 != 0 || c->rank_k > 256) return false;
-  if (c->rank_v != 128 && c->rank_v != 256) return false;
+  if (c->latent_dtype == PALU_INT4) {
+    // one 128-byte row of codes per token and side: rank 256 for keys and values
+    if (c->rank_k != 256 || c->rank_v != 256) return false;
+  } else {
+    if (c->latent_dtype != c->act_dtype) return false;
+    if (c->rank_k % 64 != 0 || c->rank_k > 256) return false;
+    if (c->rank_v != 128 && c->rank_v != 256) return false;
+  }
   const Smem L = smem_layout(c->rank_k);
   return L.total + 1024 <= 227 * 1024;
 }
@@ -737,8 +907,13 @@ int tc_head_blocks(const palu_config* c) { return c->group_size / 2; }
 
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st) {
   if (a.gs % 2 != 0) return cudaErrorInvalidValue;
-  if (a.act == PALU_BF16) return a.r_v == 256 ? launch_t<PALU_BF16, 2>(a, st) : launch_t<PALU_BF16, 1>(a, st);
-  return a.r_v == 256 ? launch_t<PALU_F16, 2>(a, st) : launch_t<PALU_F16, 1>(a, st);
+  if (a.lat == PALU_INT4) {
+    if (a.r_k != 256 || a.r_v != 256) return cudaErrorInvalidValue;
+    return a.act == PALU_BF16 ? launch_t<PALU_BF16, 2, PALU_INT4>(a, st) : launch_t<PALU_F16, 2, PALU_INT4>(a, st);
+  }
+  if (a.act == PALU_BF16)
+    return a.r_v == 256 ? launch_t<PALU_BF16, 2, PALU_BF16>(a, st) : launch_t<PALU_BF16, 1, PALU_BF16>(a, st);
+  return a.r_v == 256 ? launch_t<PALU_F16, 2, PALU_F16>(a, st) : launch_t<PALU_F16, 1, PALU_F16>(a, st);
 }
 
 }  // namespace palu

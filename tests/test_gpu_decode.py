@@ -105,3 +105,20 @@ def test_bad_page_index_reports_bounds():
     assert st == 7                                      # PALU_ERR_DEVICE_BOUNDS
     st2, _ = P.palu_get_device_status(ws)               # reading cleared it
     assert st2 == 0
+
+
+@pytest.mark.parametrize("act", ["f16", "bf16"])
+def test_int4_cuda_core_path(act):
+    # head_dim 64 is not a tensor-core shape: int4 latents through the CUDA-core split kernel
+    w = dataclasses.replace(WORKLOADS["tiny_f32"], act_dtype=act, latent_dtype="int4", rank_k=256,
+                            rank_v=256)
+    case = make_decode_case(w, [256, 77, 300, 0])
+    assert P.palu_decode_kernel_kind(case.cfg) == 1
+    out, lse = run_gpu_decode(case)
+    for b, T in enumerate(case.seq_lens):
+        if T == 0:
+            assert np.all(out[b] == 0) and np.all(np.isneginf(lse[b]))
+            continue
+        ref, ref_lse = oracle_decode(case, b)
+        assert rel_err(out[b], ref) <= TOL[act]
+        np.testing.assert_allclose(lse[b], ref_lse, rtol=0, atol=2e-2)

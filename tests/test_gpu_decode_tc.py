@@ -132,6 +132,30 @@ def test_tc_bad_page_reports_bounds():
     assert st == 7
 
 
+# ------------------------------------------------------------ int4 latents on the tensor cores
+def int4_7b(act="f16", H=8):
+    return dataclasses.replace(WORKLOADS["7b_int4_r256_b8_t32k"], act_dtype=act, num_heads=H)
+
+
+def test_tc_int4_path_is_selected():
+    for act in ("f16", "bf16"):
+        case = make_decode_case(int4_7b(act), [10])
+        assert P.palu_decode_kernel_kind(case.cfg) == 2
+
+
+@pytest.mark.parametrize("act", ["f16", "bf16"])
+def test_tc_int4_ragged_batch_and_splits(act):
+    # full pages, a ragged last page, single tokens, an empty sequence; two split counts
+    case = make_decode_case(int4_7b(act), [300, 1, 1000, 129, 0, 128, 640])
+    check(case)
+    check(case, num_splits=3)
+
+
+def test_tc_int4_explicit_positions_and_peaky_query():
+    case = make_decode_case(int4_7b("f16"), [700, 257], explicit_positions=True, q_scale=4.0)
+    check(case)
+
+
 # ------------------------------------------------------------ full-size, sampled units
 def sampled_full_size(w, context, units, seed=123, num_splits=0):
     """Run the full workload on the GPU; check the sampled (sequence, group) units.
@@ -147,27 +171,46 @@ def sampled_full_size(w, context, units, seed=123, num_splits=0):
     num_pages = b * max_pages
     pt = page_permutation(seed, num_pages).reshape(b, max_pages)
     dev = torch.device("cuda")
-    lat = TORCH_DTYPE[w.latent_dtype]
+    int4 = w.latent_dtype == "int4"
     cache = P.LatentCache.allocate(cfg, num_pages, device=dev)
     gen = torch.Generator(device=dev)
     gen.manual_seed(seed)
     for pool in (cache.zk, cache.zv):
-        view = pool.view(lat)
+        if int4:                                   # random codes, every nibble value included
+            pool.copy_(torch.randint(0, 256, pool.shape, dtype=torch.uint8, device=dev, generator=gen))
+            continue
+        view = pool.view(TORCH_DTYPE[w.latent_dtype])
         for i in range(0, view.numel(), 1 << 28):
             seg = view[i:i + (1 << 28)]
             seg.copy_(torch.randn(seg.shape, device=dev, generator=gen))
+    for sp in (cache.zks, cache.zvs):
+        if sp is not None:
+            sp.view(torch.float16).copy_(torch.rand(sp.numel() // 2, device=dev, generator=gen) * 0.5)
     host = {}
     for (bi, g) in units:
-        for name, r, pool in (("zk", w.rank_k, cache.zk), ("zv", w.rank_v, cache.zv)):
-            z = torch.from_numpy(normal(seed, name, (context, r), unit=(bi, g))).to(lat)
-            host[(name, bi, g)] = z
-            blocks = pool.view(num_pages, G, Pz * r * 2)
-            zb = z.view(torch.uint8).numpy()
+        for name, r, pool, spool in (("zk", w.rank_k, cache.zk, cache.zks), ("zv", w.rank_v, cache.zv, cache.zvs)):
+            z32 = normal(seed, name, (context, r), unit=(bi, g))
+            if int4:
+                packed, sc = O.quantize_int4(z32)
+                host[(name, bi, g)] = torch.from_numpy(O.dequantize_int4(packed, sc, w.act_dtype))
+                zb, row_bytes = packed, r // 2
+                srows = spool.view(num_pages, G, Pz, -1)
+                sb = np.zeros((context, srows.shape[3]), np.uint8)
+                sb[:, : sc.shape[1] * 2] = sc.view(np.uint8)
+            else:
+                z = torch.from_numpy(z32).to(TORCH_DTYPE[w.latent_dtype])
+                host[(name, bi, g)] = z
+                zb, row_bytes = z.view(torch.uint8).numpy(), r * 2
+            blocks = pool.view(num_pages, G, Pz * row_bytes)
             for p in range(max_pages):
                 t0, t1 = p * Pz, min(context, (p + 1) * Pz)
-                rows = np.zeros((Pz, r * 2), np.uint8)
+                rows = np.zeros((Pz, row_bytes), np.uint8)
                 rows[: t1 - t0] = zb[t0:t1]
                 blocks[pt[bi, p], g].copy_(torch.from_numpy(swizzle_block(rows)).to(dev))
+                if int4:
+                    srow = np.zeros((Pz, srows.shape[3]), np.uint8)
+                    srow[: t1 - t0] = sb[t0:t1]
+                    srows[pt[bi, p], g].copy_(torch.from_numpy(srow).to(dev))
     q = normal_tensor(seed, "q", (b, w.num_heads, w.head_dim), w.act_dtype)
     B_k = normal_tensor(seed, "B_k", (G, w.rank_k, W), w.act_dtype, 1 / math.sqrt(w.rank_k))
     B_v = normal_tensor(seed, "B_v", (G, w.rank_v, W), w.act_dtype, 1 / math.sqrt(w.rank_v))
@@ -177,7 +220,7 @@ def sampled_full_size(w, context, units, seed=123, num_splits=0):
     lse = torch.empty((b, w.num_heads), dtype=torch.float32, device=dev)
     q_pos = torch.full((b,), context - 1, dtype=torch.int32, device=dev)
     lens = torch.full((b,), context, dtype=torch.int32, device=dev)
-    P.palu_decode_attn(cfg, q.to(dev), q_pos, cache.zk, cache.zv, None, None, None,
+    P.palu_decode_attn(cfg, q.to(dev), q_pos, cache.zk, cache.zv, cache.zks, cache.zvs, None,
                        torch.from_numpy(pt).to(dev), lens, num_pages, B_k.to(dev), B_v.to(dev), out, lse,
                        ws, S)
     torch.cuda.synchronize()
@@ -221,3 +264,11 @@ def test_full_size_7b_bf16_r256_b32_t16k_sampled():
     w = WORKLOADS["7b_bf16_r256_b32_t16k"]
     worst, S = sampled_full_size(w, w.context + 31, [(0, 2), (31, 6)])
     print(f"r256/256 16k x 32 (S={S}): worst rel err {worst:.2e}")
+
+
+@pytest.mark.slow
+def test_full_size_7b_int4_b8_t32k_sampled():
+    # int4 latents (rank 256/256, fp16 compute), batch 8, context 32k (+77, a ragged page)
+    w = WORKLOADS["7b_int4_r256_b8_t32k"]
+    worst, S = sampled_full_size(w, w.context + 77, [(0, 1), (5, 6)])
+    print(f"int4 32k x 8 (S={S}): worst rel err {worst:.2e}")

@@ -42,27 +42,31 @@ using namespace tc;
 
 constexpr int kTile = 128;         // tokens per tile = page size
 constexpr int kChunk = 64;         // K chunk of z_k (elements) = one 128-byte column block of the page
-constexpr int kNKS = 3;            // z_k ring stages
+constexpr int kNKS = 3;            // z_k ring stages (barrier slots)
+__host__ __device__ constexpr int zk_stages(bool int4) { return int4 ? 2 : kNKS; }  // int4: room for the value-code buffer
 constexpr uint32_t kZkSwz = 2u;    // 128-byte swizzle
 constexpr uint32_t kZkSbo = 1024;  // bytes per 8-row swizzle atom
 constexpr int kNVS = 2;            // z_v ring stages
 constexpr int kPrefetch = 3;       // pages pulled into L2 ahead of the TMA loads
 constexpr int kThreads = 384;      // 12 warps: producers + MMA (warps 0-3), two epilogue warpgroups
 constexpr int kZkBytes = kTile * kChunk * 2;   // bytes per z_k stage
-constexpr int kZvBytes = 64 * 128 * 2;         // 16 KB: 64 tokens × 128 latent entries
+constexpr int kZvBytes = 128 * 64 * 2;         // 16 KB: one 64-entry column block of a page (128 tokens)
 constexpr int kPBytes = 16 * kTile * 2;        // 4 KB: 16 rows (heads, padded) × 128 tokens
 
 struct Smem {
   // offsets in bytes from a 1024-aligned base
-  uint32_t b, zk, zv, p, qr, psc, tb, omega, red, lred, bars, tmem_slot, abort, total;
+  uint32_t b, zk, zv, vraw, p, qr, psc, tb, omega, red, lred, bars, tmem_slot, abort, total;
 };
 
-__host__ __device__ inline Smem smem_layout(int r_k) {
+constexpr int kVRawBytes = 128 * 128 + 128 * 16;   // int4: one page of value codes + its scale rows
+
+__host__ __device__ inline Smem smem_layout(int r_k, bool int4) {
   Smem s{};
   uint32_t o = 0;
   s.b = o;      o += (uint32_t)r_k * 256 * 2;          // B_k for 2 heads
-  s.zk = o;     o += kNKS * kZkBytes;
+  s.zk = o;     o += zk_stages(int4) * kZkBytes;
   s.zv = o;     o += kNVS * kZvBytes;
+  s.vraw = o;   o += int4 ? kVRawBytes : 0;
   s.p = o;      o += 2 * kPBytes;
   s.qr = o;     o += 3 * 128 * 4;                        // q'_i, q'_{i+64}, -q'_i per head pair row
   s.psc = o;    o += 2 * 2 * 128 * 4;
@@ -92,6 +96,7 @@ enum {
   BAR_EPI = BAR_TEARDOWN + 1,        // 2: per-warpgroup sync (4 warps), bounded
   BAR_QR = BAR_EPI + 2,              // rotated query staged
   BAR_XCH = BAR_QR + 1,              // 2: both warpgroups posted their cross-head partial scores
+  BAR_VRAW = BAR_XCH + 2,            // int4: a page of value codes landed in the staging buffer
   BAR_COUNT
 };
 static_assert(BAR_COUNT <= 32, "barrier space");
@@ -163,7 +168,10 @@ __device__ __forceinline__ float from_bits(uint16_t u) {
 __device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 __device__ __forceinline__ __half2 bits_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
 
-template <int ACT>
+// PAIRED = false: the unit holds entries 0..7 in order.  PAIRED = true: the unit
+// holds entries (0, 4, 1, 5, 2, 6, 3, 7), which saves the byte permutes where
+// the consumer tracks the order (a row permutation of the value operand).
+template <int ACT, bool PAIRED>
 __device__ __forceinline__ uint4 dequant8(uint32_t x, uint16_t sbits) {
   uint4 o;
   if constexpr (ACT == PALU_F16) {
@@ -176,10 +184,13 @@ __device__ __forceinline__ uint4 dequant8(uint32_t x, uint16_t sbits) {
     const __half2 bias = bits_h2(0x64086408u);
     const __half sh = __ushort_as_half(sbits);
     const __half2 s2 = __halves2half2(sh, sh);
-    o.x = h2_bits(__hmul2(__hsub2(bits_h2(__byte_perm(r0, r1, 0x5410)), bias), s2));
-    o.y = h2_bits(__hmul2(__hsub2(bits_h2(__byte_perm(r2, r3, 0x5410)), bias), s2));
-    o.z = h2_bits(__hmul2(__hsub2(bits_h2(__byte_perm(r0, r1, 0x7632)), bias), s2));
-    o.w = h2_bits(__hmul2(__hsub2(bits_h2(__byte_perm(r2, r3, 0x7632)), bias), s2));
+    auto cv = [&](uint32_t r) { return h2_bits(__hmul2(__hsub2(bits_h2(r), bias), s2)); };
+    if constexpr (PAIRED) {
+      o = make_uint4(cv(r0), cv(r1), cv(r2), cv(r3));
+    } else {
+      o = make_uint4(cv(__byte_perm(r0, r1, 0x5410)), cv(__byte_perm(r2, r3, 0x5410)),
+                     cv(__byte_perm(r0, r1, 0x7632)), cv(__byte_perm(r2, r3, 0x7632)));
+    }
   } else {
     // (code + 8) | 0x4B000000 is the float 2^23 + code + 8; code × s is exact
     // in fp32 and the pack rounds it to bf16 once.
@@ -191,12 +202,26 @@ __device__ __forceinline__ uint4 dequant8(uint32_t x, uint16_t sbits) {
     uint32_t w[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+      __nv_bfloat162 h = PAIRED ? __floats2bfloat162_rn(v[e], v[e + 4]) : __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
       w[e] = *reinterpret_cast<uint32_t*>(&h);
     }
     o = make_uint4(w[0], w[1], w[2], w[3]);
   }
   return o;
+}
+
+// Latent entry held by row r of the value operand when its units are PAIRED.
+__device__ __forceinline__ int paired_row(int r) { return (r & ~7) | ((r & 7) >> 1) | ((r & 1) << 2); }
+
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ uint16_t ld_shared_u16(uint32_t addr) {
+  uint16_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+  return v;
 }
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
@@ -218,9 +243,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* sbase = smem_raw + (base - raw);
-  const Smem L = smem_layout(a.r_k);
+  const Smem L = smem_layout(a.r_k, LAT == PALU_INT4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr bool kInt4 = LAT == PALU_INT4;
+  constexpr int kNZK = zk_stages(kInt4);
   static_assert(!kInt4 || NRV == 2, "int4 latents: r_v = 256");
   DevStatus* st = reinterpret_cast<DevStatus*>(a.status);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sbase + L.abort);
@@ -240,7 +266,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     *abort_flag = 0;
     mbar_init(bar(BAR_B), 1);
-    for (int i = 0; i < kNKS; ++i) {
+    for (int i = 0; i < kNZK; ++i) {
       mbar_init(bar(BAR_ZK_FULL + i), kInt4 ? 2 : 1);   // int4: one arrival per dequantising warp
       mbar_init(bar(BAR_ZK_EMPTY + i), 1);
     }
@@ -256,6 +282,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(BAR_AT_FULL), 1);
     mbar_init(bar(BAR_TEARDOWN), 1);
     mbar_init(bar(BAR_QR), 4);
+    mbar_init(bar(BAR_VRAW), 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(BAR_EPI + i), 4);
       mbar_init(bar(BAR_XCH + i), 8);
@@ -283,112 +310,132 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int nb = 0; nb < 4; ++nb)
       tma_load_2d(base + L.b + (uint32_t)nb * a.r_k * 128, &tm_bk, hp * 256 + nb * 64, g * a.r_k, bar(BAR_B));
   }
-  if (kInt4 && (warp == 0 || warp == 2 || warp == 3)) {
-    {
-      // ============================================================ int4 dequantising producers
-      // z_k (warps 0, 3): chunk c of a tile = entries [64c, 64c + 64) of all 128
-      // tokens, i.e. scale blocks 2c and 2c+1.  Thread zt takes block 2c + (zt & 1)
-      // of tokens zt/2 + 32i.  z_v (warp 2): ring stage (mb, th) = entries
-      // [128mb, 128mb + 128) of tokens [64th, 64th + 64), in two steps of 32
-      // tokens; lane takes block 4mb + lane/8 of tokens 64th + lane%8 + 8i.
-      // Loads run two steps ahead of the conversion (three register slots).
-      const bool is_k = warp != 2;
-      const int zt = (warp == 3 ? 32 : 0) + lane;
-      const int nv_tiles = tr.ntiles - (tr.ragged_last ? 1 : 0);
-      const int N = is_k ? tr.ntiles * 4 : nv_tiles * 8;
-      const uint8_t* pool = reinterpret_cast<const uint8_t*>(is_k ? a.zk : a.zv);
-      const uint8_t* spool = reinterpret_cast<const uint8_t*>(is_k ? a.zks : a.zvs);
-      const long long srow_bytes = is_k ? a.ks_row : a.vs_row;
-      struct Slot {
-        uint4 raw[4];
-        uint16_t sc[4];
-      };
-      auto issue = [&](int n, Slot& sl) {
-        if (n >= N) return;
-        const int k = is_k ? (n >> 2) : (n >> 3);
-        int pg = page_of(a, b, tr.t_begin / kTile + k);
-        if (pg < 0) {
-          if (is_k && (n & 3) == 0 && zt == 0) report(st, PALU_ERR_DEVICE_BOUNDS, 2000000 + b);
-          pg = 0;   // keep the pipeline fed from a valid page; the status says the result is void
-        }
-        if (is_k && (n & 3) == 0 && zt == 0 && k + kPrefetch < tr.ntiles) {
-          // pull a later page of this split into L2 while this one converts
-          const int ppg = page_of(a, b, tr.t_begin / kTile + k + kPrefetch);
-          if (ppg >= 0) {
-            const size_t prow = (size_t)(ppg * a.G + g) * a.P;
-            prefetch_l2(reinterpret_cast<const uint8_t*>(a.zk) + prow * a.k_row, (uint32_t)(a.P * a.k_row));
-            prefetch_l2(reinterpret_cast<const uint8_t*>(a.zks) + prow * a.ks_row, (uint32_t)(a.P * a.ks_row));
-            prefetch_l2(reinterpret_cast<const uint8_t*>(a.zv) + prow * a.v_row, (uint32_t)(a.P * a.v_row));
-            prefetch_l2(reinterpret_cast<const uint8_t*>(a.zvs) + prow * a.vs_row, (uint32_t)(a.P * a.vs_row));
-          }
-        }
-        const size_t row0 = (size_t)(pg * a.G + g) * a.P;
-        const uint8_t* blk = pool + row0 * 128;
-        const uint8_t* sblk = spool + row0 * srow_bytes;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          int t, u;
-          if (is_k) {
-            t = (zt >> 1) + 32 * i;
-            u = 2 * (n & 3) + (zt & 1);
-          } else {
-            const int sidx = n & 7;   // (mb, th, half) of this tile
-            t = 64 * ((sidx >> 1) & 1) + (lane & 7) + 8 * (4 * (sidx & 1) + i);
-            u = 4 * (sidx >> 2) + (lane >> 3);
-          }
-          sl.raw[i] = __ldg(reinterpret_cast<const uint4*>(blk + t * 128 + ((u ^ (t & 7)) << 4)));
-          sl.sc[i] = __ldg(reinterpret_cast<const unsigned short*>(sblk + t * srow_bytes + 2 * u));
-        }
-      };
-      int stage = 0;
-      uint32_t phase = 0;
-      auto consume = [&](int n, const Slot& sl) -> bool {
-        if (n >= N) return true;
-        const int nst = is_k ? kNKS : kNVS;
-        const int first = is_k || (n & 1) == 0;
-        const int last = is_k || (n & 1) == 1;
-        const int ebar = is_k ? BAR_ZK_EMPTY : BAR_ZV_EMPTY;
-        const int fbar = is_k ? BAR_ZK_FULL : BAR_ZV_FULL;
-        if (first && !mbar_wait(bar(ebar + stage), phase ^ 1, abort_flag, st, is_k ? 12 : 13)) return false;
-        const uint32_t dst = base + (is_k ? L.zk + stage * kZkBytes : L.zv + stage * kZvBytes);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint32_t w[4] = {sl.raw[i].x, sl.raw[i].y, sl.raw[i].z, sl.raw[i].w};
-#pragma unroll
-          for (int m = 0; m < 4; ++m) {
-            const uint4 o = dequant8<ACT>(w[m], sl.sc[i]);
-            uint32_t off;
-            if (is_k) {
-              const int t = (zt >> 1) + 32 * i;
-              off = t * 128 + (((4 * (zt & 1) + m) ^ (t & 7)) << 4);
-            } else {
-              const int tl = (lane & 7) + 8 * (4 * (n & 1) + i);   // token within the 64 of the stage
-              const int ul = lane >> 3;
-              off = (ul >> 1) * 8192 + tl * 128 + (((4 * (ul & 1) + m) ^ (lane & 7)) << 4);
-            }
-            st_shared_v4(dst + off, o);
-          }
-        }
-        if (last) {
-          fence_proxy_async();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(fbar + stage));
-          if (is_k && zt == 0 && (n & 3) == 0) trace(6, n >> 2);
-          if (++stage == nst) { stage = 0; phase ^= 1; }
-        }
-        return true;
-      };
-      Slot s0, s1, s2;
-      issue(0, s0);
-      issue(1, s1);
-      for (int n = 0; n < N && !*abort_flag; n += 3) {
-        issue(n + 2, s2);
-        if (!consume(n, s0)) break;
-        issue(n + 3, s0);
-        if (!consume(n + 1, s1)) break;
-        issue(n + 4, s1);
-        if (!consume(n + 2, s2)) break;
+  if (kInt4 && (warp == 0 || warp == 3)) {
+    // ============================================================ int4 key codes (warps 0, 3)
+    // Chunk c of a tile = entries [64c, 64c + 64) of all 128 tokens, i.e. scale
+    // blocks 2c and 2c+1.  Thread zt takes block 2c + (zt & 1) of tokens
+    // zt/2 + 32i, loaded straight into registers three chunks ahead of the
+    // conversion (four register slots), while later pages are pulled into L2.
+    const int zt = (warp == 3 ? 32 : 0) + lane;
+    const int N = tr.ntiles * 4;
+    struct Slot {
+      uint4 raw[4];
+      uint16_t sc[4];
+    };
+    auto issue = [&](int n, Slot& sl) {
+      if (n >= N) return;
+      const int k = n >> 2;
+      int pg = page_of(a, b, tr.t_begin / kTile + k);
+      if (pg < 0) {
+        if ((n & 3) == 0 && zt == 0) report(st, PALU_ERR_DEVICE_BOUNDS, 2000000 + b);
+        pg = 0;   // keep the pipeline fed from a valid page; the status says the result is void
       }
+      if ((n & 3) == 0 && zt == 0) {
+        for (int kk = (k == 0 ? 1 : k + kPrefetch); kk <= k + kPrefetch && kk < tr.ntiles; ++kk) {
+          const int ppg = page_of(a, b, tr.t_begin / kTile + kk);
+          if (ppg < 0) continue;
+          const size_t prow = (size_t)(ppg * a.G + g) * a.P;
+          prefetch_l2(reinterpret_cast<const uint8_t*>(a.zk) + prow * a.k_row, (uint32_t)(a.P * a.k_row));
+          prefetch_l2(reinterpret_cast<const uint8_t*>(a.zks) + prow * a.ks_row, (uint32_t)(a.P * a.ks_row));
+          prefetch_l2(reinterpret_cast<const uint8_t*>(a.zv) + prow * a.v_row, (uint32_t)(a.P * a.v_row));
+          prefetch_l2(reinterpret_cast<const uint8_t*>(a.zvs) + prow * a.vs_row, (uint32_t)(a.P * a.vs_row));
+        }
+      }
+      const size_t row0 = (size_t)(pg * a.G + g) * a.P;
+      const uint8_t* blk = reinterpret_cast<const uint8_t*>(a.zk) + row0 * 128;
+      const uint8_t* sblk = reinterpret_cast<const uint8_t*>(a.zks) + row0 * a.ks_row;
+      const int u = 2 * (n & 3) + (zt & 1);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int t = (zt >> 1) + 32 * i;
+        sl.raw[i] = __ldg(reinterpret_cast<const uint4*>(blk + t * 128 + ((u ^ (t & 7)) << 4)));
+        sl.sc[i] = __ldg(reinterpret_cast<const unsigned short*>(sblk + t * a.ks_row + 2 * u));
+      }
+    };
+    int stage = 0;
+    uint32_t phase = 0;
+    auto consume = [&](int n, const Slot& sl) -> bool {
+      if (n >= N) return true;
+      if (!mbar_wait(bar(BAR_ZK_EMPTY + stage), phase ^ 1, abort_flag, st, 12)) return false;
+      const uint32_t dst = base + L.zk + stage * kZkBytes;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int t = (zt >> 1) + 32 * i;
+        const uint32_t w[4] = {sl.raw[i].x, sl.raw[i].y, sl.raw[i].z, sl.raw[i].w};
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+          st_shared_v4(dst + t * 128 + (((4 * (zt & 1) + m) ^ (t & 7)) << 4), dequant8<ACT, false>(w[m], sl.sc[i]));
+      }
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(BAR_ZK_FULL + stage));
+      if (zt == 0 && (n & 3) == 0) trace(6, n >> 2);
+      if (++stage == kNZK) { stage = 0; phase ^= 1; }
+      return true;
+    };
+    Slot s0, s1, s2, s3;
+    issue(0, s0);
+    issue(1, s1);
+    issue(2, s2);
+    for (int n = 0; n < N && !*abort_flag; n += 4) {
+      issue(n + 3, s3);
+      if (!consume(n, s0)) break;
+      issue(n + 4, s0);
+      if (!consume(n + 1, s1)) break;
+      issue(n + 5, s1);
+      if (!consume(n + 2, s2)) break;
+      issue(n + 6, s2);
+      if (!consume(n + 3, s3)) break;
+    }
+  } else if (kInt4 && warp == 2) {
+    // ============================================================ int4 value codes (warp 2)
+    // One page of codes and its scale rows per tile, staged in shared memory by
+    // a bulk copy; ring stage (mb, cb) = the 64 entries [128mb + 64cb, +64) of
+    // all 128 tokens, i.e. scale blocks 4mb + 2cb and 4mb + 2cb + 1.  Lane takes
+    // block 4mb + 2cb + (lane/8 & 1) of tokens lane%8 + 8(2i + lane/16).  Units
+    // are written PAIRED: row r of the value operand holds entry paired_row(r).
+    const int nv_tiles = tr.ntiles - (tr.ragged_last ? 1 : 0);
+    const uint32_t vraw = base + L.vraw;
+    auto load_raw = [&](int k) {
+      int pg = page_of(a, b, tr.t_begin / kTile + k);
+      if (pg < 0) pg = 0;   // reported by the key producer
+      const size_t row0 = (size_t)(pg * a.G + g) * a.P;
+      mbar_expect_tx(bar(BAR_VRAW), kVRawBytes);
+      bulk_load(vraw, reinterpret_cast<const uint8_t*>(a.zv) + row0 * 128, 128 * 128, bar(BAR_VRAW));
+      bulk_load(vraw + 128 * 128, reinterpret_cast<const uint8_t*>(a.zvs) + row0 * a.vs_row, 128 * 16,
+                bar(BAR_VRAW));
+    };
+    if (lane == 0 && nv_tiles > 0) load_raw(0);
+    int stage = 0;
+    uint32_t phase = 0;
+    const int x = lane & 7, ub = (lane >> 3) & 1, tg = lane >> 4;
+    for (int k = 0; k < nv_tiles && !*abort_flag; ++k) {
+      if (!mbar_wait(bar(BAR_VRAW), k & 1, abort_flag, st, 14)) break;
+      bool ok = true;
+      for (int sidx = 0; sidx < 2 * NRV; ++sidx) {   // column block 2mb + cb of the page
+        if (!mbar_wait(bar(BAR_ZV_EMPTY + stage), phase ^ 1, abort_flag, st, 13)) { ok = false; break; }
+        const uint32_t dst = base + L.zv + stage * kZvBytes;
+        const int u = 2 * sidx + ub;
+#pragma unroll 4
+        for (int i = 0; i < 8; ++i) {
+          const int t = x + 8 * (2 * i + tg);
+          const uint4 raw = ld_shared_v4(vraw + t * 128 + ((u ^ x) << 4));
+          const uint16_t sc = ld_shared_u16(vraw + 128 * 128 + t * 16 + 2 * u);
+          const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+          for (int m = 0; m < 4; ++m)
+            st_shared_v4(dst + t * 128 + (((4 * ub + m) ^ x) << 4), dequant8<ACT, true>(w[m], sc));
+        }
+        fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(BAR_ZV_FULL + stage));
+        if (++stage == kNVS) { stage = 0; phase ^= 1; }
+      }
+      if (!ok) break;
+      // every lane has read this page's codes: refill the buffer with the next page
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0 && k + 1 < nv_tiles) load_raw(k + 1);
     }
   } else if (warp == 0) {
     // ============================================================ z_k producer (bulk copies)
@@ -424,7 +471,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_expect_tx(bar(BAR_ZK_FULL + stage), kZkBytes);
           bulk_load(base + L.zk + stage * kZkBytes, src + (size_t)c * kZkBytes, kZkBytes, bar(BAR_ZK_FULL + stage));
           if (c == 0) trace(6, k);
-          if (++stage == kNKS) { stage = 0; phase ^= 1; }
+          if (++stage == kNZK) { stage = 0; phase ^= 1; }
         }
       }
     }
@@ -439,17 +486,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         int pg = page_of(a, b, lp);
         if (pg < 0) pg = 0;   // reported by the z_k producer
         const uint8_t* src = reinterpret_cast<const uint8_t*>(a.zv) + (size_t)(pg * a.G + g) * a.P * a.v_row;
-        for (int mb = 0; mb < NRV; ++mb) {
-          for (int th = 0; th < 2; ++th) {
-            if (!mbar_wait(bar(BAR_ZV_EMPTY + stage), phase ^ 1, abort_flag, st, 11)) break;
-            mbar_expect_tx(bar(BAR_ZV_FULL + stage), kZvBytes);
-            const uint32_t dst = base + L.zv + stage * kZvBytes;
-            // 64 tokens of two 128-byte column blocks = the two MN-blocks of the value operand
-            const size_t off = (size_t)(2 * mb) * a.P * 128 + (size_t)th * 64 * 128;
-            bulk_load(dst, src + off, 8192, bar(BAR_ZV_FULL + stage));
-            bulk_load(dst + 8192, src + off + (size_t)a.P * 128, 8192, bar(BAR_ZV_FULL + stage));
-            if (++stage == kNVS) { stage = 0; phase ^= 1; }
-          }
+        // one copy per 128-byte column block of the page (64 latent entries of
+        // all 128 tokens); two consecutive blocks are the two MN-blocks of one
+        // value-MMA operand
+        for (int cb = 0; cb < 2 * NRV; ++cb) {
+          if (!mbar_wait(bar(BAR_ZV_EMPTY + stage), phase ^ 1, abort_flag, st, 11)) break;
+          mbar_expect_tx(bar(BAR_ZV_FULL + stage), kZvBytes);
+          bulk_load(base + L.zv + stage * kZvBytes, src + (size_t)cb * a.P * 128, kZvBytes,
+                    bar(BAR_ZV_FULL + stage));
+          if (++stage == kNVS) { stage = 0; phase ^= 1; }
         }
       }
     }
@@ -460,7 +505,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc_d = idesc_f16(kBf, 0, 1, 256, 128);    // z_k K-major, B_k MN-major
       const uint32_t idesc_pv = idesc_f16(kBf, 1, 0, 16, 128);    // z_vᵀ MN-major, Pᵀ K-major
       const uint32_t b_lbo = (uint32_t)a.r_k * 128;                // bytes between 64-column blocks of B
-      int zs = 0, vs = 0;
+      int zs = 0;
       uint32_t zph = 0, vph = 0;
       bool ok = mbar_wait(bar(BAR_B), 0, abort_flag, st, 20);
       int pv_pending = -1;   // tile whose value MMA waits for its P
@@ -469,21 +514,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto issue_pv = [&](int j) -> bool {
         tc_fence_after();
         const uint32_t a_tmem = tmem + (uint32_t)(j & 1) * 256;
+        const uint32_t p_base = base + L.p + (uint32_t)(j & 1) * kPBytes;
+        static_assert(kNVS == 2, "one value MMA operand = the two ring stages");
         for (int mb = 0; mb < NRV; ++mb) {
-          for (int th = 0; th < 2; ++th) {
-            if (!mbar_wait(bar(BAR_ZV_FULL + vs), vph, abort_flag, st, 22)) return false;
-            tc_fence_after();
-            const uint32_t zv_addr = base + L.zv + vs * kZvBytes;
-            const uint32_t p_addr = base + L.p + (uint32_t)(j & 1) * kPBytes + th * 2048;
+          for (int cb = 0; cb < 2; ++cb)
+            if (!mbar_wait(bar(BAR_ZV_FULL + cb), vph, abort_flag, st, 22)) return false;
+          tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t ad = sdesc(zv_addr + kk * 16 * 128, 8192, 1024, kSw128);
-              const uint64_t bd = sdesc(p_addr + kk * 32, 16, 1024, kSw128);
-              umma_f16(a_tmem + mb * 16, ad, bd, idesc_pv, (th | kk) != 0);
-            }
-            umma_commit(bar(BAR_ZV_EMPTY + vs));
-            if (++vs == kNVS) { vs = 0; vph ^= 1; }
+          for (int kk = 0; kk < kTile / 16; ++kk) {
+            // rows = latent entries (two 64-entry blocks, one per stage), K = tokens
+            const uint64_t ad = sdesc(base + L.zv + kk * 16 * 128, kZvBytes, 1024, kSw128);
+            const uint64_t bd = sdesc(p_base + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024, kSw128);
+            umma_f16(a_tmem + mb * 16, ad, bd, idesc_pv, kk != 0);
           }
+          umma_commit(bar(BAR_ZV_EMPTY + 0));
+          umma_commit(bar(BAR_ZV_EMPTY + 1));
+          vph ^= 1;
         }
         umma_commit(bar(BAR_AT_FULL));
         trace(2, j);
@@ -535,7 +581,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma_f16(d_tmem, ad, bd, idesc_d, (c | kk) != 0);
           }
           umma_commit(bar(BAR_ZK_EMPTY + zs));
-          if (++zs == kNKS) { zs = 0; zph ^= 1; }
+          if (++zs == kNZK) { zs = 0; zph ^= 1; }
         }
         if (!ok) break;
         umma_commit(bar(BAR_D_FULL + slot));
@@ -610,7 +656,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         srow[v] = f2_pack(s0, s1);
       }
     }
-    auto half_scores = [&](int slot, int t0, int pos, float* part) {
+    auto half_scores = [&](int slot, int t0, int pos, float* part, auto&& mid) {
       if (contig) {
         float c, sn;
         rope_cs_fast(t0, om[wg * 32 + lane], c, sn);
@@ -625,6 +671,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int hh = 0; hh < 2; ++hh) acc[hh][0] = acc[hh][1] = 0ull;
 #pragma unroll
       for (int jj = 0; jj < 2; ++jj) {
+        if (jj == 1) mid();
         const int i0 = wg * 32 + jj * 16;
         const uint32_t col = tmem + lane_addr + (uint32_t)slot * 256 + i0;
         float lo[16], hi[16];
@@ -703,6 +750,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the latent value sums and the output; the partial scores of the other
       // head go across in shared memory.
       const int hw = wg;
+      // latent entry of TMEM lane `row` of aᵀ (int4: the value operand's units are PAIRED)
+      const int vrow = kInt4 ? paired_row(row) : row;
       float m_run = -INFINITY, l_part = 0.f, prev_scale = 0.f;
       float acc[NRV];
 #pragma unroll
@@ -725,7 +774,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
 
       for (int k = 0; k < tr.ntiles && ok; ++k) {
-        if (k >= 1 && !fold_at(k - 1, prev_scale)) { ok = false; break; }
         const int t0 = tr.t_begin + k * kTile;
         const bool valid = t0 + row < tr.t_end;
         int pos = t0 + row;
@@ -738,7 +786,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         if (row == 0 && wg == 0) trace(3, k);
         float part[2];
-        half_scores(slot, t0, pos, part);
+        // The previous tile's latent sums are folded halfway through this tile's
+        // scores: its value MMA has had that long to finish, and its TMEM slot
+        // (where the next key MMA goes) is released early enough for that MMA
+        // to finish before the next tile's scores start.
+        bool folded = true;
+        half_scores(slot, t0, pos, part, [&] {
+          if (k >= 1) folded = fold_at(k - 1, prev_scale);
+        });
+        if (!folded) { ok = false; break; }
         tc_fence_before();
         psc[(slot * 2 + (1 - hw)) * 128 + row] = part[1 - hw];
         __syncwarp();
@@ -792,7 +848,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const uint8_t* srow = kInt4 ? zvs + (size_t)t * a.vs_row : nullptr;
 #pragma unroll
               for (int mb = 0; mb < NRV; ++mb)
-                at[mb] = fmaf(pv, load_latent<LAT, ACT>(zv, t, a.P, srow, mb * 128 + row), at[mb]);
+                at[mb] = fmaf(pv, load_latent<LAT, ACT>(zv, t, a.P, srow, mb * 128 + vrow), at[mb]);
             }
           }
 #pragma unroll
@@ -815,7 +871,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           out[1] = (lred[wg * 4 + 0] + lred[wg * 4 + 1]) + (lred[wg * 4 + 2] + lred[wg * 4 + 3]);
         }
 #pragma unroll
-        for (int mb = 0; mb < NRV; ++mb) out[2 + mb * 128 + row] = acc[mb];
+        for (int mb = 0; mb < NRV; ++mb) out[2 + mb * 128 + vrow] = acc[mb];
       }
     }
   }
@@ -867,7 +923,7 @@ cudaError_t launch_t(const DecodeArgs& a, cudaStream_t st) {
   if (!make_map_2d(&tm_bk, a.Bk, dt, 2, a.W, (uint64_t)a.G * a.r_k, (uint64_t)a.W * 2, 64, a.r_k,
                    CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  const Smem L = smem_layout(a.r_k);
+  const Smem L = smem_layout(a.r_k, LAT == PALU_INT4);
   const size_t smem = L.total + 1024;
   auto kern = decode_tc_kernel<ACT, NRV, LAT>;
   DecodeArgs args = a;
@@ -899,7 +955,7 @@ bool tc_decode_supported(const palu_config* c) {
     if (c->rank_k % 64 != 0 || c->rank_k > 256) return false;
     if (c->rank_v != 128 && c->rank_v != 256) return false;
   }
-  const Smem L = smem_layout(c->rank_k);
+  const Smem L = smem_layout(c->rank_k, c->latent_dtype == PALU_INT4);
   return L.total + 1024 <= 227 * 1024;
 }
 

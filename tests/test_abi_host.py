@@ -135,3 +135,15 @@ def test_product_path_does_not_import_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 text = open(os.path.join(root, f), encoding="utf-8").read()
                 assert "import oracle" not in text and "from oracle" not in text, f
+
+
+def test_tensor_core_kernel_fits_every_7b_workload():
+    # host-side check (no GPU): the tensor-core split kernel's shared-memory
+    # layout fits for every 7B-shaped workload, int4 latents included
+    from rank_kv_cache_palu_b200.synth import WORKLOADS
+    for w in WORKLOADS.values():
+        if w.head_dim != 128:
+            continue
+        c = P.make_config(w.num_heads, w.head_dim, w.group_size, w.rank_k, w.rank_v, w.page_size,
+                          w.rope_base, w.act_dtype, w.latent_dtype)
+        assert P.palu_decode_kernel_kind(c) == 2, w.name

@@ -674,64 +674,52 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (jj == 1) mid();
         const int i0 = wg * 32 + jj * 16;
         const uint32_t col = tmem + lane_addr + (uint32_t)slot * 256 + i0;
-        float lo[16], hi[16];
-        tmem_ld16(col, lo);
-        tmem_ld16(col + 64, hi);
-        f2 cs[8], sn[8];
-        if (contig) {
-          const float4* c4 = reinterpret_cast<const float4*>(tbw + jj * 16);
-          const float4* s4 = reinterpret_cast<const float4*>(tbw + 32 + jj * 16);
-          const float4* n4 = reinterpret_cast<const float4*>(tbw + 64 + jj * 16);
+        // both heads' keys of these 16 frequency pairs in one TMEM round trip
+        float lo[2][16], hi[2][16];
+        tmem_ld16(col, lo[0]);
+        tmem_ld16(col + 64, hi[0]);
+        tmem_ld16(col + 128, lo[1]);
+        tmem_ld16(col + 192, hi[1]);
+        tmem_wait_ld();
 #pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4) {
-            const float4 cb = c4[v4], sb = s4[v4], nb = n4[v4];
+        for (int v4 = 0; v4 < 4; ++v4) {
+          float4 cb4 = make_float4(0.f, 0.f, 0.f, 0.f), sb4 = cb4, nb4 = cb4;
+          if (contig) {
+            cb4 = reinterpret_cast<const float4*>(tbw + jj * 16)[v4];
+            sb4 = reinterpret_cast<const float4*>(tbw + 32 + jj * 16)[v4];
+            nb4 = reinterpret_cast<const float4*>(tbw + 64 + jj * 16)[v4];
+          }
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int v = v4 * 2 + e;
-              const f2 c0 = e ? f2_pack(cb.z, cb.w) : f2_pack(cb.x, cb.y);
-              const f2 s0 = e ? f2_pack(sb.z, sb.w) : f2_pack(sb.x, sb.y);
-              const f2 n0 = e ? f2_pack(nb.z, nb.w) : f2_pack(nb.x, nb.y);
+          for (int e = 0; e < 2; ++e) {
+            const int v = v4 * 2 + e;
+            f2 cs, sn;
+            if (contig) {
+              const f2 c0 = e ? f2_pack(cb4.z, cb4.w) : f2_pack(cb4.x, cb4.y);
+              const f2 s0 = e ? f2_pack(sb4.z, sb4.w) : f2_pack(sb4.x, sb4.y);
+              const f2 n0 = e ? f2_pack(nb4.z, nb4.w) : f2_pack(nb4.x, nb4.y);
               // cos(t0+row) = c0 cr - s0 sr ; sin(t0+row) = s0 cr + c0 sr
-              cs[v] = f2_fma(c0, crow[jj * 8 + v], f2_mul(n0, srow[jj * 8 + v]));
-              sn[v] = f2_fma(s0, crow[jj * 8 + v], f2_mul(c0, srow[jj * 8 + v]));
+              cs = f2_fma(c0, crow[jj * 8 + v], f2_mul(n0, srow[jj * 8 + v]));
+              sn = f2_fma(s0, crow[jj * 8 + v], f2_mul(c0, srow[jj * 8 + v]));
+            } else {
+              // explicit positions: a sincos per token
+              float c0, s0, c1, s1;
+              rope_cs_fast(pos, om[i0 + 2 * v], c0, s0);
+              rope_cs_fast(pos, om[i0 + 2 * v + 1], c1, s1);
+              cs = f2_pack(c0, c1);
+              sn = f2_pack(s0, s1);
             }
-          }
-        } else {
-          // explicit positions: a sincos per token
 #pragma unroll
-          for (int v = 0; v < 8; ++v) {
-            float c0, s0, c1, s1;
-            rope_cs_fast(pos, om[i0 + 2 * v], c0, s0);
-            rope_cs_fast(pos, om[i0 + 2 * v + 1], c1, s1);
-            cs[v] = f2_pack(c0, c1);
-            sn[v] = f2_pack(s0, s1);
-          }
-        }
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          if (hh == 1) {
-            tmem_ld16(col + 128, lo);
-            tmem_ld16(col + 192, hi);
-          }
-          tmem_wait_ld();
-          const float4* qa4 = reinterpret_cast<const float4*>(qr + hh * 192 + i0);
-          const float4* qb4 = reinterpret_cast<const float4*>(qr + hh * 192 + 64 + i0);
-          const float4* qn4 = reinterpret_cast<const float4*>(qr + hh * 192 + 128 + i0);
-#pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4) {
-            const float4 qa = qa4[v4], qb = qb4[v4], qn = qn4[v4];
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int v = v4 * 2 + e;
-              const f2 a2 = e ? f2_pack(qa.z, qa.w) : f2_pack(qa.x, qa.y);
-              const f2 b2 = e ? f2_pack(qb.z, qb.w) : f2_pack(qb.x, qb.y);
-              const f2 n2 = e ? f2_pack(qn.z, qn.w) : f2_pack(qn.x, qn.y);
-              const f2 lo2 = f2_pack(lo[2 * v], lo[2 * v + 1]);
-              const f2 hi2 = f2_pack(hi[2 * v], hi[2 * v + 1]);
+            for (int hh = 0; hh < 2; ++hh) {
+              const float* qh = qr + hh * 192 + i0 + 4 * v4 + 2 * e;
+              const f2 a2 = *reinterpret_cast<const f2*>(qh);
+              const f2 b2 = *reinterpret_cast<const f2*>(qh + 64);
+              const f2 n2 = *reinterpret_cast<const f2*>(qh + 128);
+              const f2 lo2 = f2_pack(lo[hh][2 * v], lo[hh][2 * v + 1]);
+              const f2 hi2 = f2_pack(hi[hh][2 * v], hi[hh][2 * v + 1]);
               const f2 x = f2_fma(b2, hi2, f2_mul(a2, lo2));     // q'_i k_i + q'_{i+64} k_{i+64}
               const f2 y = f2_fma(b2, lo2, f2_mul(n2, hi2));     // q'_{i+64} k_i - q'_i k_{i+64}
-              acc[hh][e] = f2_fma(cs[v], x, acc[hh][e]);
-              acc[hh][e] = f2_fma(sn[v], y, acc[hh][e]);
+              acc[hh][e] = f2_fma(cs, x, acc[hh][e]);
+              acc[hh][e] = f2_fma(sn, y, acc[hh][e]);
             }
           }
         }

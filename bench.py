@@ -171,8 +171,13 @@ def step_work(w, seq_lens):
     tok = sum(seq_lens)
     bytes_ = tok * G * row + G * (w.rank_k + w.rank_v) * W * elt \
         + len(seq_lens) * w.num_heads * w.head_dim * elt * 2
-    flops = tok * G * (2 * w.rank_k * W + 2 * gs * w.rank_v) \
-        + len(seq_lens) * w.num_heads * 2 * w.rank_v * w.head_dim
+    if w.rope_base == 0:
+        # fused path: scores in latent space (q̃ = B_k q per head, r_k long)
+        flops = tok * G * (2 * gs * w.rank_k + 2 * gs * w.rank_v) \
+            + len(seq_lens) * w.num_heads * 2 * (w.rank_k + w.rank_v) * w.head_dim
+    else:
+        flops = tok * G * (2 * w.rank_k * W + 2 * gs * w.rank_v) \
+            + len(seq_lens) * w.num_heads * 2 * w.rank_v * w.head_dim
     return bytes_, flops
 
 
@@ -425,7 +430,8 @@ def run_ours(args):
     roof["tensor_achieved_tflops"] = tfs
     roof["algorithmic_bytes_per_launch"] = dbytes
     roof["algorithmic_flops_per_launch"] = dflops
-    roof["kernel"] = "palu_decode_attn (split + combine), kernel kind %d" % kind
+    roof["kernel"] = "palu_decode_attn (%s), kernel kind %d" % (
+        "fold-query + fused split + combine" if kind == 3 else "split + combine", kind)
     roof["avg_launch_ms"] = dec_avg_s * 1e3
 
     line = {

@@ -1,0 +1,526 @@
+// Fused decode for attention without rotary embedding (sm_100a: tcgen05 + TMEM).
+//
+// Method: "PALU 论文低秩投影分解" §低秩投影分解 (the latent is either restored
+// to full K/V or fused with the operators that follow) and §把它放进一次真实推理
+// 流程里看, Decode 阶段 (attention fused with the up-projection, so full K/V are
+// never materialised); the v1 abstract of "Palu: Compressing KV-Cache with
+// Low-Rank Projection" names matrix fusion.  Without RoPE the key up-projection
+// folds into the query:
+//   s_{t,h} = q_h · (B_k,hᵀ z_k,t) = (B_k,h q_h) · z_k,t,   B_k,h = B_k[g][:, cols_h],
+// so scores come straight from the cached latents and no key is rebuilt; the
+// values stay in latent space as on the RoPE path (a = Σ p z_v, then a·B_v in
+// the combine).  With RoPE the rotation sits between B_k and q and the fold is
+// not available, which is why the main kernel rebuilds keys.
+//
+// fold_query_kernel: q̃_h = B_k,h q_h · log2(e)/√d_h for the g heads of a group,
+//   stored as the sum of two 16-bit numbers (hi + lo) so the tensor cores see
+//   q̃ to ~16 significant bits.
+// decode_fused_kernel: one CTA per (sequence, group, split), 128 tokens (a page)
+//   per tile:
+//   warp 0  bulk copies of the z_k and z_v pages through two rings (q̃ is
+//           staged into shared memory by all threads at the start);
+//   warp 1  MMAs: D[128 tok × 16] = z_k · [q̃_hi ; q̃_lo]ᵀ (scores of the g
+//           heads twice, hi and lo parts) and aᵀ[r_v × 16] = z_vᵀ · Pᵀ;
+//   warps 2-5  one thread per token / latent row: scores, online softmax of the
+//           g heads, P (bf16/fp16), and the fold of aᵀ into running sums.
+// Output: per (b, head, split) the partial (m, l, a[r_v]) the combine merges.
+#include <cuda.h>
+#include <math.h>
+
+#include "palu_common.cuh"
+#include "palu_internal.h"
+#include "palu_tc.h"
+#include "tc_ptx.cuh"
+
+namespace palu {
+namespace {
+
+using namespace tc;
+
+constexpr int kTile = 128;          // tokens per tile = page size
+constexpr int kChunk = 64;          // K chunk (latent entries) = one 128-byte column block
+constexpr int kThreads = 192;       // producer, MMA, four epilogue warps
+constexpr int kMaxG = 4;            // heads per group the fused kernel takes
+constexpr int kNZK = 6;             // z_k ring stages
+constexpr int kNZV = 4;             // z_v ring stages (pairs of column blocks)
+constexpr int kStageBytes = kTile * kChunk * 2;   // 16 KB: one column block of a page
+constexpr int kPBytes = 16 * kTile * 2;           // P tile: 16 rows (heads, padded) × 128 tokens
+constexpr int kPrefetch = 4;        // pages pulled into L2 ahead of the copies
+constexpr int kTmemCols = 128;      // D: 2 × 16 columns; aᵀ: 2 × 32 columns
+
+struct Smem {
+  uint32_t qt, zk, zv, p, red, lred, bars, tmem_slot, abort, total;
+};
+
+__host__ __device__ inline Smem smem_layout(int r_k) {
+  Smem s{};
+  uint32_t o = 0;
+  s.qt = o;   o += (uint32_t)(r_k / kChunk) * 16 * 128;   // [K chunk][16 rows][128 B], 128-byte swizzle
+  s.zk = o;   o += kNZK * kStageBytes;
+  s.zv = o;   o += kNZV * kStageBytes;
+  s.p = o;    o += 2 * kPBytes;
+  s.red = o;  o += 2 * 4 * kMaxG * 4;                    // [tile parity][warp][head] maxima
+  s.lred = o; o += 4 * kMaxG * 4;                        // [warp][head] softmax denominators
+  s.bars = o; o += 32 * 8;
+  s.tmem_slot = o; o += 16;
+  s.abort = o;     o += 16;
+  s.total = o;
+  return s;
+}
+
+enum {
+  BAR_ZK_FULL = 0,
+  BAR_ZK_EMPTY = BAR_ZK_FULL + kNZK,
+  BAR_ZV_FULL = BAR_ZK_EMPTY + kNZK,
+  BAR_ZV_EMPTY = BAR_ZV_FULL + kNZV,
+  BAR_D_FULL = BAR_ZV_EMPTY + kNZV,    // 2
+  BAR_D_EMPTY = BAR_D_FULL + 2,        // 2
+  BAR_P_FULL = BAR_D_EMPTY + 2,        // 2
+  BAR_AT_FULL = BAR_P_FULL + 2,        // 2
+  BAR_AT_EMPTY = BAR_AT_FULL + 2,      // 2
+  BAR_EPI = BAR_AT_EMPTY + 2,          // epilogue warps meet (bounded)
+  BAR_TEARDOWN = BAR_EPI + 1,
+  BAR_COUNT
+};
+static_assert(BAR_COUNT <= 32, "barrier space");
+
+__device__ __forceinline__ int page_of(const DecodeArgs& a, int b, int lp) {
+  const int pg = a.page_table[(size_t)b * a.max_pages + lp];
+  return (pg < 0 || pg >= a.num_pages) ? -1 : pg;
+}
+
+// P tile, K-major with the 128-byte swizzle: row n (head), token k; tokens
+// 0-63 and 64-127 sit in two 2 KB atoms of 16 rows.
+__device__ __forceinline__ uint32_t p_offset(int n, int k) {
+  const int region = k >> 6, kin = k & 63;
+  return (uint32_t)(region * 2048 + n * 128 + (((kin >> 3) ^ (n & 7)) << 4) + (kin & 7) * 2);
+}
+
+template <int ACT>
+__device__ __forceinline__ uint16_t to_bits(float v) {
+  const auto h = Dt<ACT>::from_f(v);
+  return *reinterpret_cast<const uint16_t*>(&h);
+}
+template <int ACT>
+__device__ __forceinline__ float from_bits(uint16_t u) {
+  return Dt<ACT>::to_f(*reinterpret_cast<const typename Dt<ACT>::T*>(&u));
+}
+
+// q̃ = B_k,h q_h (scaled) for the heads of one group, as hi + lo 16-bit rows:
+// out[b][g][h] = hi, out[b][g][4 + h] = lo (h < gs; other rows zero), each r_k
+// long.  One thread per latent entry j; the B_k row j of the group serves all
+// its heads.
+template <int ACT>
+__global__ void __launch_bounds__(256) fold_query_kernel(const DecodeArgs a, void* qt) {
+  using TA = typename Dt<ACT>::T;
+  __shared__ float qs[kMaxG * 128];
+  const int g = blockIdx.x, b = blockIdx.y;
+  const int gs = a.gs, d_h = a.d_h;
+  for (int i = threadIdx.x; i < gs * d_h; i += blockDim.x)
+    qs[i] = Dt<ACT>::to_f(reinterpret_cast<const TA*>(a.q)[((size_t)b * a.H + g * gs) * d_h + i]);
+  __syncthreads();
+  constexpr float kLog2e = 1.4426950408889634f;
+  const float sc = a.sm_scale * kLog2e;
+  TA* out = reinterpret_cast<TA*>(qt) + ((size_t)b * a.G + g) * 2 * kMaxG * a.r_k;
+  for (int j = threadIdx.x; j < a.r_k; j += blockDim.x) {
+    const TA* brow = reinterpret_cast<const TA*>(a.Bk) + ((size_t)g * a.r_k + j) * a.W;
+    for (int h = 0; h < kMaxG; ++h) {
+      float acc = 0.f;
+      if (h < gs)
+        for (int d = 0; d < d_h; ++d) acc = fmaf(Dt<ACT>::to_f(brow[h * d_h + d]), qs[h * d_h + d], acc);
+      acc *= sc;
+      const TA hi = Dt<ACT>::from_f(acc);
+      const TA lo = Dt<ACT>::from_f(acc - Dt<ACT>::to_f(hi));
+      out[(size_t)h * a.r_k + j] = hi;
+      out[(size_t)(kMaxG + h) * a.r_k + j] = lo;
+    }
+  }
+}
+
+template <int ACT, int NRV>
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_fused_kernel(const DecodeArgs a, const void* qt) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* sbase = smem_raw + (base - raw);
+  const Smem L = smem_layout(a.r_k);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  DevStatus* st = reinterpret_cast<DevStatus*>(a.status);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sbase + L.abort);
+  auto bar = [&](int i) { return base + L.bars + 8u * i; };
+
+  const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int gs = a.gs;
+  const int nkc = a.r_k / kChunk;
+  int T = a.seq_lens[b];
+  const int cap = a.max_pages * a.P;
+  if (T < 0 || T > cap) {
+    if (threadIdx.x == 0) report(st, PALU_ERR_DEVICE_BOUNDS, 1000000 + b);
+    T = T < 0 ? 0 : cap;
+  }
+  const int npg = (T + kTile - 1) / kTile;
+  const int pps = (npg + a.S - 1) / a.S;
+  const int pg0 = s * pps;
+  const int pg1 = min(npg, pg0 + pps);
+  const int ntiles = max(0, pg1 - pg0);
+  const int t_end = min(T, pg1 * kTile);
+  const bool ragged_last = ntiles > 0 && t_end - (pg0 + ntiles - 1) * kTile < kTile;
+  const int nvt = ntiles - (ragged_last ? 1 : 0);   // tiles whose value sum runs on the tensor cores
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    for (int i = 0; i < kNZK; ++i) {
+      mbar_init(bar(BAR_ZK_FULL + i), 1);
+      mbar_init(bar(BAR_ZK_EMPTY + i), 1);
+    }
+    for (int i = 0; i < kNZV; ++i) {
+      mbar_init(bar(BAR_ZV_FULL + i), 1);
+      mbar_init(bar(BAR_ZV_EMPTY + i), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(BAR_D_FULL + i), 1);
+      mbar_init(bar(BAR_D_EMPTY + i), 4);
+      mbar_init(bar(BAR_P_FULL + i), 4);
+      mbar_init(bar(BAR_AT_FULL + i), 1);
+      mbar_init(bar(BAR_AT_EMPTY + i), 4);
+    }
+    mbar_init(bar(BAR_EPI), 4);
+    mbar_init(bar(BAR_TEARDOWN), 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(base + L.tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  // P padding rows stay zero; q̃ rows 2·gs..15 stay zero
+  for (int i = threadIdx.x; i < 2 * kPBytes / 4; i += kThreads) reinterpret_cast<uint32_t*>(sbase + L.p)[i] = 0u;
+  for (int i = threadIdx.x; i < nkc * 16 * 32; i += kThreads) reinterpret_cast<uint32_t*>(sbase + L.qt)[i] = 0u;   // rows 8-15
+  __syncthreads();
+  // q̃ into the K-major swizzled B operand: row n (hi/lo head), entry j
+  {
+    const uint16_t* src = reinterpret_cast<const uint16_t*>(qt) + ((size_t)b * a.G + g) * 2 * kMaxG * a.r_k;
+    for (int i = threadIdx.x; i < 2 * kMaxG * a.r_k; i += kThreads) {
+      const int n = i / a.r_k, j = i % a.r_k;
+      const int c = j / kChunk, kin = j % kChunk;
+      *reinterpret_cast<uint16_t*>(sbase + L.qt + c * 2048 + n * 128 + ((((kin >> 3) ^ (n & 7))) << 4) + (kin & 7) * 2) =
+          src[i];
+    }
+  }
+  fence_proxy_async();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sbase + L.tmem_slot);
+
+  if (warp == 0) {
+    // ============================================================ producer (bulk copies)
+    if (lane == 0) {
+      auto prefetch_page = [&](int k) {
+        if (k >= ntiles) return;
+        const int pg = page_of(a, b, pg0 + k);
+        if (pg < 0) return;
+        const size_t row = (size_t)(pg * a.G + g) * a.P;
+        prefetch_l2(reinterpret_cast<const uint8_t*>(a.zk) + row * a.k_row, (uint32_t)(a.P * a.k_row));
+        prefetch_l2(reinterpret_cast<const uint8_t*>(a.zv) + row * a.v_row, (uint32_t)(a.P * a.v_row));
+      };
+      for (int k = 0; k < kPrefetch; ++k) prefetch_page(k);
+      int zs = 0, vs = 0;
+      uint32_t zph = 0, vph = 0;
+      // z_v of a tile is needed only after its scores: stream it one tile behind
+      // z_k, so the two rings fill in the order the MMAs consume them
+      auto push_zv = [&](int k) -> bool {
+        int pg = page_of(a, b, pg0 + k);
+        if (pg < 0) pg = 0;   // reported with the keys
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(a.zv) + (size_t)(pg * a.G + g) * a.P * a.v_row;
+        for (int cb = 0; cb < 2 * NRV; ++cb) {
+          if (!mbar_wait(bar(BAR_ZV_EMPTY + vs), vph ^ 1, abort_flag, st, 11)) return false;
+          mbar_expect_tx(bar(BAR_ZV_FULL + vs), kStageBytes);
+          bulk_load(base + L.zv + vs * kStageBytes, src + (size_t)cb * a.P * 128, kStageBytes, bar(BAR_ZV_FULL + vs));
+          if (++vs == kNZV) { vs = 0; vph ^= 1; }
+        }
+        return true;
+      };
+      bool ok = true;
+      for (int k = 0; k < ntiles && ok && !*abort_flag; ++k) {
+        prefetch_page(k + kPrefetch);
+        int pg = page_of(a, b, pg0 + k);
+        if (pg < 0) {
+          report(st, PALU_ERR_DEVICE_BOUNDS, 2000000 + b);
+          pg = 0;   // keep the pipeline fed from a valid page; the status says the result is void
+        }
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(a.zk) + (size_t)(pg * a.G + g) * a.P * a.k_row;
+        for (int c = 0; c < nkc; ++c) {
+          if (!mbar_wait(bar(BAR_ZK_EMPTY + zs), zph ^ 1, abort_flag, st, 10)) { ok = false; break; }
+          mbar_expect_tx(bar(BAR_ZK_FULL + zs), kStageBytes);
+          bulk_load(base + L.zk + zs * kStageBytes, src + (size_t)c * kStageBytes, kStageBytes, bar(BAR_ZK_FULL + zs));
+          if (++zs == kNZK) { zs = 0; zph ^= 1; }
+        }
+        if (ok && k >= 1 && k - 1 < nvt) ok = push_zv(k - 1);
+      }
+      if (ok && ntiles >= 1 && ntiles - 1 < nvt) push_zv(ntiles - 1);
+    }
+  } else if (warp == 1) {
+    // ============================================================ MMA issuer
+    if (lane == 0) {
+      constexpr int kBf = ACT == PALU_BF16 ? 1 : 0;
+      const uint32_t idesc_s = idesc_f16(kBf, 0, 0, 16, 128);    // z_k K-major, q̃ K-major
+      const uint32_t idesc_pv = idesc_f16(kBf, 1, 0, 16, 128);   // z_vᵀ MN-major, Pᵀ K-major
+      int zs = 0, vs = 0;
+      uint32_t zph = 0, vph = 0;
+      bool ok = true;
+      auto issue_pv = [&](int j) -> bool {
+        const uint32_t a_tmem = tmem + 32 + (uint32_t)(j & 1) * 32;
+        const uint32_t p_base = base + L.p + (uint32_t)(j & 1) * kPBytes;
+        if (!mbar_wait(bar(BAR_P_FULL + (j & 1)), (j >> 1) & 1, abort_flag, st, 21)) return false;
+        if (!mbar_wait(bar(BAR_AT_EMPTY + (j & 1)), ((j >> 1) & 1) ^ 1, abort_flag, st, 22)) return false;
+        tc_fence_after();
+        for (int mb = 0; mb < NRV; ++mb) {
+          for (int cb = 0; cb < 2; ++cb)
+            if (!mbar_wait(bar(BAR_ZV_FULL + vs + cb), vph, abort_flag, st, 23)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk) {
+            const uint64_t ad = sdesc(base + L.zv + vs * kStageBytes + kk * 16 * 128, kStageBytes, 1024, kSw128);
+            const uint64_t bd = sdesc(p_base + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024, kSw128);
+            umma_f16(a_tmem + mb * 16, ad, bd, idesc_pv, kk != 0);
+          }
+          umma_commit(bar(BAR_ZV_EMPTY + vs));
+          umma_commit(bar(BAR_ZV_EMPTY + vs + 1));
+          vs += 2;
+          if (vs == kNZV) { vs = 0; vph ^= 1; }
+        }
+        umma_commit(bar(BAR_AT_FULL + (j & 1)));
+        return true;
+      };
+      for (int k = 0; k < ntiles && ok; ++k) {
+        const int slot = k & 1;
+        if (!mbar_wait(bar(BAR_D_EMPTY + slot), ((k >> 1) & 1) ^ 1, abort_flag, st, 24)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + (uint32_t)slot * 16;
+        for (int c = 0; c < nkc; ++c) {
+          if (!mbar_wait(bar(BAR_ZK_FULL + zs), zph, abort_flag, st, 25)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < kChunk / 16; ++kk) {
+            const uint64_t ad = sdesc(base + L.zk + zs * kStageBytes + kk * 32, 16, 1024, kSw128);
+            const uint64_t bd = sdesc(base + L.qt + c * 2048 + kk * 32, 16, 1024, kSw128);
+            umma_f16(d_tmem, ad, bd, idesc_s, (c | kk) != 0);
+          }
+          umma_commit(bar(BAR_ZK_EMPTY + zs));
+          if (++zs == kNZK) { zs = 0; zph ^= 1; }
+        }
+        if (!ok) break;
+        umma_commit(bar(BAR_D_FULL + slot));
+        // the previous tile's value MMA, once its P is written
+        if (k >= 1 && k - 1 < nvt && !issue_pv(k - 1)) { ok = false; break; }
+      }
+      if (ok && ntiles >= 1 && ntiles - 1 < nvt) issue_pv(ntiles - 1);
+      umma_commit(bar(BAR_TEARDOWN));
+      mbar_wait(bar(BAR_TEARDOWN), 0, abort_flag, st, 26);
+    }
+  } else {
+    // ============================================================ epilogue (warps 2-5)
+    const int q4 = warp & 3;                 // TMEM lane quarter this warp may access
+    const int row = q4 * 32 + lane;          // token row of the tile / latent row of aᵀ
+    const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
+    float* red = reinterpret_cast<float*>(sbase + L.red);
+    uint32_t epi_phase = 0;
+    auto ep_sync = [&](int where) -> bool {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(BAR_EPI));
+      const bool r = mbar_wait(bar(BAR_EPI), epi_phase, abort_flag, st, where);
+      epi_phase ^= 1;
+      return r;
+    };
+    float m_run[kMaxG], l_part[kMaxG], prev_scale[kMaxG];
+    float acc[NRV][kMaxG];
+#pragma unroll
+    for (int h = 0; h < kMaxG; ++h) {
+      m_run[h] = -INFINITY;
+      l_part[h] = 0.f;
+      prev_scale[h] = 0.f;
+#pragma unroll
+      for (int mb = 0; mb < NRV; ++mb) acc[mb][h] = 0.f;
+    }
+    auto fold_at = [&](int j) -> bool {
+      if (!mbar_wait(bar(BAR_AT_FULL + (j & 1)), (j >> 1) & 1, abort_flag, st, 30)) return false;
+      tc_fence_after();
+#pragma unroll
+      for (int mb = 0; mb < NRV; ++mb) {
+        float v[4];
+        tmem_ld2(tmem + lane_addr + 32 + (uint32_t)(j & 1) * 32 + mb * 16, v);
+        tmem_ld2(tmem + lane_addr + 32 + (uint32_t)(j & 1) * 32 + mb * 16 + 2, v + 2);
+        tmem_wait_ld();
+#pragma unroll
+        for (int h = 0; h < kMaxG; ++h)
+          if (h < gs) acc[mb][h] = fmaf(acc[mb][h], prev_scale[h], v[h]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(BAR_AT_EMPTY + (j & 1)));
+      return true;
+    };
+    bool ok = true;
+    for (int k = 0; k < ntiles && ok; ++k) {
+      const int slot = k & 1;
+      const int t0 = (pg0 + k) * kTile;
+      const bool valid = t0 + row < t_end;
+      if (!mbar_wait(bar(BAR_D_FULL + slot), (k >> 1) & 1, abort_flag, st, 31)) { ok = false; break; }
+      tc_fence_after();
+      float d[8];
+      tmem_ld2(tmem + lane_addr + slot * 16, d);
+      tmem_ld2(tmem + lane_addr + slot * 16 + 2, d + 2);
+      tmem_ld2(tmem + lane_addr + slot * 16 + 4, d + 4);
+      tmem_ld2(tmem + lane_addr + slot * 16 + 6, d + 6);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(BAR_D_EMPTY + slot));
+      // the previous tile's latent sums are ready by now (its value MMA went
+      // in behind this tile's scores)
+      if (k >= 1 && !fold_at(k - 1)) { ok = false; break; }
+      float sc[kMaxG];
+#pragma unroll
+      for (int h = 0; h < kMaxG; ++h) {
+        sc[h] = (valid && h < gs) ? d[h] + d[kMaxG + h] : -INFINITY;   // hi and lo parts of q̃
+        float m = sc[h];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+        if (lane == 0) red[((k & 1) * 4 + q4) * kMaxG + h] = m;
+      }
+      if (!ep_sync(33)) { ok = false; break; }
+#pragma unroll
+      for (int h = 0; h < kMaxG; ++h) {
+        if (h >= gs) continue;
+        const float* rr = red + (k & 1) * 4 * kMaxG + h;
+        const float mt = fmaxf(fmaxf(rr[0], rr[kMaxG]), fmaxf(rr[2 * kMaxG], rr[3 * kMaxG]));
+        const float m_new = fmaxf(m_run[h], mt);
+        const float scale = m_new == -INFINITY ? 1.f : exp2f(m_run[h] - m_new);
+        const uint16_t pb = to_bits<ACT>(valid ? exp2f(sc[h] - m_new) : 0.f);
+        *reinterpret_cast<uint16_t*>(sbase + L.p + slot * kPBytes + p_offset(h, row)) = pb;
+        l_part[h] = fmaf(l_part[h], scale, from_bits<ACT>(pb));
+        m_run[h] = m_new;
+        prev_scale[h] = scale;
+      }
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(BAR_P_FULL + slot));
+    }
+    if (ok && ntiles > 0) {
+      const int kl = ntiles - 1;
+      if (!ragged_last) {
+        ok = fold_at(kl);
+      } else {
+        // partial last page: a += Σ_{valid tokens} p · z_v on CUDA cores from the
+        // valid rows only
+        ok = ep_sync(34);   // every P entry of the tile is written
+        const int t0 = (pg0 + kl) * kTile;
+        const int nvalid = t_end - t0;
+        const int pg = page_of(a, b, pg0 + kl);
+        float at[NRV][kMaxG];
+#pragma unroll
+        for (int mb = 0; mb < NRV; ++mb)
+#pragma unroll
+          for (int h = 0; h < kMaxG; ++h) at[mb][h] = 0.f;
+        if (pg >= 0) {
+          const uint8_t* zv = reinterpret_cast<const uint8_t*>(a.zv) + (size_t)(pg * a.G + g) * a.P * a.v_row;
+          const uint8_t* pbuf = sbase + L.p + (kl & 1) * kPBytes;
+          for (int t = 0; t < nvalid; ++t) {
+            float z[NRV];
+#pragma unroll
+            for (int mb = 0; mb < NRV; ++mb) z[mb] = load_latent<ACT, ACT>(zv, t, a.P, nullptr, mb * 128 + row);
+#pragma unroll
+            for (int h = 0; h < kMaxG; ++h) {
+              if (h >= gs) continue;
+              const float pv = from_bits<ACT>(*reinterpret_cast<const uint16_t*>(pbuf + p_offset(h, t)));
+#pragma unroll
+              for (int mb = 0; mb < NRV; ++mb) at[mb][h] = fmaf(pv, z[mb], at[mb][h]);
+            }
+          }
+        }
+#pragma unroll
+        for (int mb = 0; mb < NRV; ++mb)
+#pragma unroll
+          for (int h = 0; h < kMaxG; ++h) acc[mb][h] = fmaf(acc[mb][h], prev_scale[h], at[mb][h]);
+      }
+    }
+    // l per head: sum of the per-thread partials
+    float* lred = reinterpret_cast<float*>(sbase + L.lred);
+#pragma unroll
+    for (int h = 0; h < kMaxG; ++h) {
+      float v = l_part[h];
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+      if (lane == 0) lred[q4 * kMaxG + h] = v;
+    }
+    ok = ep_sync(35) && ok;
+    float lsum[kMaxG];
+#pragma unroll
+    for (int h = 0; h < kMaxG; ++h)
+      lsum[h] = (lred[h] + lred[kMaxG + h]) + (lred[2 * kMaxG + h] + lred[3 * kMaxG + h]);
+    if (ok && !*abort_flag) {
+      constexpr float kLn2 = 0.6931471805599453f;
+#pragma unroll
+      for (int h = 0; h < kMaxG; ++h) {
+        if (h >= gs) continue;
+        float* out = a.part + (((size_t)b * a.H + g * gs + h) * a.S + s) * (a.r_v + 2);
+        if (row == 0) {
+          out[0] = ntiles > 0 ? m_run[h] * kLn2 : -INFINITY;
+          out[1] = lsum[h];
+        }
+#pragma unroll
+        for (int mb = 0; mb < NRV; ++mb) out[2 + mb * 128 + row] = acc[mb][h];
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <int ACT, int NRV>
+cudaError_t launch_t(const DecodeArgs& a, cudaStream_t st) {
+  void* qt = a.fused_q;
+  fold_query_kernel<ACT><<<dim3(a.G, a.batch), 256, 0, st>>>(a, qt);
+  count_launch();
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const Smem L = smem_layout(a.r_k);
+  const size_t smem = L.total + 1024;
+  auto kern = decode_fused_kernel<ACT, NRV>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<dim3(a.S, a.G, a.batch), kThreads, smem, st>>>(a, qt);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool fused_decode_supported(const palu_config* c) {
+  if (c->rope_base != 0.f) return false;
+  if (c->page_size != kTile || c->head_dim > 128 || c->group_size > kMaxG) return false;
+  if (c->act_dtype != PALU_F16 && c->act_dtype != PALU_BF16) return false;
+  if (c->latent_dtype != c->act_dtype) return false;
+  if (c->rank_k % 64 != 0 || c->rank_k > 512) return false;
+  if (c->rank_v != 128 && c->rank_v != 256) return false;
+  return smem_layout(c->rank_k).total + 1024 <= 227 * 1024;
+}
+
+size_t fused_query_bytes(const palu_config* c, int batch) {
+  const size_t G = (size_t)(c->num_heads / c->group_size);
+  return (size_t)batch * G * 2 * kMaxG * c->rank_k * 2;
+}
+
+cudaError_t launch_decode_fused(const DecodeArgs& a, cudaStream_t st) {
+  if (a.act == PALU_BF16) return a.r_v == 256 ? launch_t<PALU_BF16, 2>(a, st) : launch_t<PALU_BF16, 1>(a, st);
+  return a.r_v == 256 ? launch_t<PALU_F16, 2>(a, st) : launch_t<PALU_F16, 1>(a, st);
+}
+
+}  // namespace palu

@@ -74,9 +74,10 @@ size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
 int auto_splits(const palu_config* c, int batch, int max_pages, int kind) {
   const int sms = 148;
-  const long long units = kind == 2 ? (long long)batch * (c->num_heads / c->group_size) *
-                                          palu::tc_head_blocks(c)
-                                    : (long long)batch * c->num_heads;
+  const long long groups = (long long)batch * (c->num_heads / c->group_size);
+  const long long units = kind == 3   ? groups
+                          : kind == 2 ? groups * palu::tc_head_blocks(c)
+                                      : (long long)batch * c->num_heads;
   // enough CTAs for ~4 waves of one CTA per SM, but never more splits than pages
   long long S = (4LL * sms + units - 1) / units;
   if (kind == 2) {
@@ -91,6 +92,7 @@ int auto_splits(const palu_config* c, int batch, int max_pages, int kind) {
 
 int kernel_kind(const palu_config* c) {
   if (check_config(c) != PALU_OK) return 0;
+  if (palu::fused_decode_supported(c)) return 3;
   if (palu::tc_decode_supported(c)) return 2;
   return 1;
 }
@@ -220,6 +222,7 @@ palu_status palu_decode_workspace_size(const palu_config* cfg, int batch, int ma
   const int S = num_splits == 0 ? auto_splits(cfg, batch, max_pages, kernel_kind(cfg)) : num_splits;
   const size_t part = (size_t)batch * cfg->num_heads * S * (cfg->rank_v + 2) * sizeof(float);
   *bytes = kStatusBytes + align256(part);
+  if (kernel_kind(cfg) == 3) *bytes += align256(palu::fused_query_bytes(cfg, batch));
   return PALU_OK;
 }
 
@@ -281,6 +284,8 @@ palu_status palu_decode_attn(const palu_config* cfg, int batch, const void* q, c
   a.lse = lse;
   a.status = workspace;
   a.part = reinterpret_cast<float*>(static_cast<char*>(workspace) + kStatusBytes);
+  a.fused_q = static_cast<char*>(workspace) + kStatusBytes +
+              align256((size_t)batch * cfg->num_heads * S * (cfg->rank_v + 2) * sizeof(float));
   a.k_row = palu::latent_row_bytes(a.lat, a.r_k);
   a.v_row = palu::latent_row_bytes(a.lat, a.r_v);
   a.ks_row = palu::scale_row_bytes(a.lat, a.r_k);
@@ -288,7 +293,9 @@ palu_status palu_decode_attn(const palu_config* cfg, int batch, const void* q, c
   fill_omega(cfg, a.omega);
 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = (kind == 2) ? palu::launch_decode_tc(a, st) : palu::launch_decode_simt(a, st);
+  cudaError_t e = kind == 3   ? palu::launch_decode_fused(a, st)
+                  : kind == 2 ? palu::launch_decode_tc(a, st)
+                              : palu::launch_decode_simt(a, st);
   if (e != cudaSuccess) return cuda_status(e);
   return cuda_status(palu::launch_combine(a, st));
 }

@@ -33,6 +33,7 @@ struct DecodeArgs {
   void* out;
   float* lse;
   float* part;         // [batch][H][S][r_v + 2] float32
+  void* fused_q;       // fused (no-RoPE) path: folded queries [batch][G][2·gs][r_k], act dtype
   void* status;        // DevStatus*
   long long k_row, v_row, ks_row, vs_row;  // bytes per latent / scale row
   uint64_t omega[kMaxHalfDim];             // RoPE frequencies as 64-bit fixed-point turns

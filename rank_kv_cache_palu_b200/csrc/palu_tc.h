@@ -13,6 +13,13 @@ bool tc_decode_supported(const palu_config* c);
 int tc_head_blocks(const palu_config* c);
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st);
 
+// Decode without RoPE: the key up-projection folded into the query, scores
+// taken on the cached latents (no key is rebuilt).  Its workspace adds the
+// folded queries after the split partials.
+bool fused_decode_supported(const palu_config* c);
+size_t fused_query_bytes(const palu_config* c, int batch);
+cudaError_t launch_decode_fused(const DecodeArgs& a, cudaStream_t st);
+
 // Compress: shapes the tensor-core GEMM takes, and the scratch it needs.
 bool tc_compress_supported(const palu_config* c, int n_tokens, int d_model);
 size_t tc_compress_scratch_bytes(const palu_config* c, int n_tokens, int d_model);

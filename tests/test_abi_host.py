@@ -139,11 +139,22 @@ def test_product_path_does_not_import_oracle():
 
 def test_tensor_core_kernel_fits_every_7b_workload():
     # host-side check (no GPU): the tensor-core split kernel's shared-memory
-    # layout fits for every 7B-shaped workload, int4 latents included
+    # layout fits for every 7B-shaped workload, int4 latents included (the
+    # fused kernel for the workloads without RoPE)
     from rank_kv_cache_palu_b200.synth import WORKLOADS
     for w in WORKLOADS.values():
         if w.head_dim != 128:
             continue
         c = P.make_config(w.num_heads, w.head_dim, w.group_size, w.rank_k, w.rank_v, w.page_size,
                           w.rope_base, w.act_dtype, w.latent_dtype)
-        assert P.palu_decode_kernel_kind(c) == 2, w.name
+        assert P.palu_decode_kernel_kind(c) == (3 if w.rope_base == 0 else 2), w.name
+
+
+def test_fused_path_selected_without_rope():
+    # host-side: attention without RoPE takes the fused (latent-space) kernel,
+    # whose workspace also holds the folded queries
+    c = cfg(rope_base=0.0)
+    assert P.palu_decode_kernel_kind(c) == 3
+    assert P.palu_decode_kernel_kind(cfg()) == 2
+    S = P.palu_decode_num_splits(c, 16, 128)
+    assert P.palu_decode_workspace_size(c, 16, 128, S) >= 256 + 16 * 32 * S * 130 * 4 + 16 * 8 * 8 * 256 * 2

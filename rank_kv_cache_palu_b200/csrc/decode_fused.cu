@@ -45,7 +45,6 @@ constexpr int kNZK = 6;             // z_k ring stages
 constexpr int kNZV = 4;             // z_v ring stages (pairs of column blocks)
 constexpr int kStageBytes = kTile * kChunk * 2;   // 16 KB: one column block of a page
 constexpr int kPBytes = 16 * kTile * 2;           // P tile: 16 rows (heads, padded) × 128 tokens
-constexpr int kPrefetch = 4;        // pages pulled into L2 ahead of the copies
 constexpr int kTmemCols = 128;      // D: 2 × 16 columns; aᵀ: 2 × 32 columns
 
 struct Smem {
@@ -108,32 +107,49 @@ __device__ __forceinline__ float from_bits(uint16_t u) {
 
 // q̃ = B_k,h q_h (scaled) for the heads of one group, as hi + lo 16-bit rows:
 // out[b][g][h] = hi, out[b][g][4 + h] = lo (h < gs; other rows zero), each r_k
-// long.  One thread per latent entry j; the B_k row j of the group serves all
-// its heads.
+// long.  CTA (g, 64 latent entries, 4 sequences); thread (entry j, head h)
+// holds the B_k row segment B_k[g][j][h·d_h, +d_h) in registers and takes its
+// dot product with the query of each of the 4 sequences.
+constexpr int kFoldSeqs = 4;
 template <int ACT>
 __global__ void __launch_bounds__(256) fold_query_kernel(const DecodeArgs a, void* qt) {
   using TA = typename Dt<ACT>::T;
-  __shared__ float qs[kMaxG * 128];
-  const int g = blockIdx.x, b = blockIdx.y;
+  __shared__ float qs[kFoldSeqs][kMaxG][128];
+  const int g = blockIdx.x, jb = blockIdx.y, b0 = blockIdx.z * kFoldSeqs;
   const int gs = a.gs, d_h = a.d_h;
-  for (int i = threadIdx.x; i < gs * d_h; i += blockDim.x)
-    qs[i] = Dt<ACT>::to_f(reinterpret_cast<const TA*>(a.q)[((size_t)b * a.H + g * gs) * d_h + i]);
+  for (int i = threadIdx.x; i < kFoldSeqs * kMaxG * 128; i += blockDim.x) {
+    const int bb = i / (kMaxG * 128), h = (i / 128) % kMaxG, d = i % 128;
+    float v = 0.f;
+    if (b0 + bb < a.batch && h < gs && d < d_h)
+      v = Dt<ACT>::to_f(reinterpret_cast<const TA*>(a.q)[((size_t)(b0 + bb) * a.H + g * gs + h) * d_h + d]);
+    qs[bb][h][d] = v;
+  }
   __syncthreads();
+  const int jl = threadIdx.x >> 2, h = threadIdx.x & 3;
+  const int j = jb * 64 + jl;
+  if (j >= a.r_k) return;
+  // the row segment as 8-element vectors (d_h is a multiple of 8 here)
+  uint4 bseg[16];
+  const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const TA*>(a.Bk) +
+                                                    ((size_t)g * a.r_k + j) * a.W + (size_t)h * d_h);
+#pragma unroll
+  for (int v = 0; v < 16; ++v) bseg[v] = (h < gs && v * 8 < d_h) ? __ldg(src + v) : make_uint4(0, 0, 0, 0);
   constexpr float kLog2e = 1.4426950408889634f;
   const float sc = a.sm_scale * kLog2e;
-  TA* out = reinterpret_cast<TA*>(qt) + ((size_t)b * a.G + g) * 2 * kMaxG * a.r_k;
-  for (int j = threadIdx.x; j < a.r_k; j += blockDim.x) {
-    const TA* brow = reinterpret_cast<const TA*>(a.Bk) + ((size_t)g * a.r_k + j) * a.W;
-    for (int h = 0; h < kMaxG; ++h) {
-      float acc = 0.f;
-      if (h < gs)
-        for (int d = 0; d < d_h; ++d) acc = fmaf(Dt<ACT>::to_f(brow[h * d_h + d]), qs[h * d_h + d], acc);
-      acc *= sc;
-      const TA hi = Dt<ACT>::from_f(acc);
-      const TA lo = Dt<ACT>::from_f(acc - Dt<ACT>::to_f(hi));
-      out[(size_t)h * a.r_k + j] = hi;
-      out[(size_t)(kMaxG + h) * a.r_k + j] = lo;
+  for (int bb = 0; bb < kFoldSeqs && b0 + bb < a.batch; ++bb) {
+    float acc = 0.f;
+#pragma unroll
+    for (int v = 0; v < 16; ++v) {
+      const TA* e = reinterpret_cast<const TA*>(&bseg[v]);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) acc = fmaf(Dt<ACT>::to_f(e[u]), qs[bb][h][v * 8 + u], acc);
     }
+    acc *= sc;
+    const TA hi = Dt<ACT>::from_f(acc);
+    const TA lo = Dt<ACT>::from_f(acc - Dt<ACT>::to_f(hi));
+    TA* out = reinterpret_cast<TA*>(qt) + ((size_t)(b0 + bb) * a.G + g) * 2 * kMaxG * a.r_k;
+    out[(size_t)h * a.r_k + j] = hi;
+    out[(size_t)(kMaxG + h) * a.r_k + j] = lo;
   }
 }
 
@@ -215,16 +231,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ============================================================ producer (bulk copies)
+    // The rings hold 160 KB, enough bytes in flight to cover HBM latency; a
+    // bulk L2 prefetch of later pages on top of them measured slower here
+    // (lines evicted before use: 1.44x the algorithmic DRAM bytes).
     if (lane == 0) {
-      auto prefetch_page = [&](int k) {
-        if (k >= ntiles) return;
-        const int pg = page_of(a, b, pg0 + k);
-        if (pg < 0) return;
-        const size_t row = (size_t)(pg * a.G + g) * a.P;
-        prefetch_l2(reinterpret_cast<const uint8_t*>(a.zk) + row * a.k_row, (uint32_t)(a.P * a.k_row));
-        prefetch_l2(reinterpret_cast<const uint8_t*>(a.zv) + row * a.v_row, (uint32_t)(a.P * a.v_row));
-      };
-      for (int k = 0; k < kPrefetch; ++k) prefetch_page(k);
       int zs = 0, vs = 0;
       uint32_t zph = 0, vph = 0;
       // z_v of a tile is needed only after its scores: stream it one tile behind
@@ -243,7 +253,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       bool ok = true;
       for (int k = 0; k < ntiles && ok && !*abort_flag; ++k) {
-        prefetch_page(k + kPrefetch);
         int pg = page_of(a, b, pg0 + k);
         if (pg < 0) {
           report(st, PALU_ERR_DEVICE_BOUNDS, 2000000 + b);
@@ -487,7 +496,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int ACT, int NRV>
 cudaError_t launch_t(const DecodeArgs& a, cudaStream_t st) {
   void* qt = a.fused_q;
-  fold_query_kernel<ACT><<<dim3(a.G, a.batch), 256, 0, st>>>(a, qt);
+  fold_query_kernel<ACT><<<dim3(a.G, (a.r_k + 63) / 64, (a.batch + kFoldSeqs - 1) / kFoldSeqs), 256, 0, st>>>(a, qt);
   count_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -505,7 +514,7 @@ cudaError_t launch_t(const DecodeArgs& a, cudaStream_t st) {
 
 bool fused_decode_supported(const palu_config* c) {
   if (c->rope_base != 0.f) return false;
-  if (c->page_size != kTile || c->head_dim > 128 || c->group_size > kMaxG) return false;
+  if (c->page_size != kTile || c->head_dim > 128 || c->head_dim % 8 != 0 || c->group_size > kMaxG) return false;
   if (c->act_dtype != PALU_F16 && c->act_dtype != PALU_BF16) return false;
   if (c->latent_dtype != c->act_dtype) return false;
   if (c->rank_k % 64 != 0 || c->rank_k > 512) return false;

@@ -47,6 +47,9 @@ def parse_args():
     ap.add_argument("--num-splits", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU oracle sample budget")
+    ap.add_argument("--prefill", type=int, default=None,
+                    help="also time palu_compress_append of this many prompt tokens (default: 8192 for "
+                         "the batch-32 prefill + decode workload, else off)")
     return ap.parse_args()
 
 
@@ -407,6 +410,40 @@ def run_ours(args):
     e2e_ms = D.max_over_ranks(e0.elapsed_time(e1), dev)
     e2e_value = D.sum_over_ranks(e2e_units, dev) / (e2e_ms / 1e3)
 
+    # ---- prefill: palu_compress_append of a prompt (x·A for n tokens into fresh pages)
+    prefill = None
+    n_pre = args.prefill if args.prefill is not None else (8192 if w.name == "7b_bf16_r256_b32_t16k" else 0)
+    if n_pre > 0 and world >= 1:
+        pre_pages = (n_pre + Pz - 1) // Pz
+        pcache = P.LatentCache.allocate(cfg, pre_pages, device=dev)
+        xp = torch.randn((n_pre, d_model), device=dev, generator=gen).to(act)
+        pslots = torch.arange(n_pre, dtype=torch.int32, device=dev)
+        ws_p = torch.zeros(P.palu_compress_workspace_size(cfg, n_pre, d_model), dtype=torch.uint8, device=dev)
+        def pre():
+            P.palu_compress_append(cfg, xp, A_k, A_v, pslots, None, pcache.zk, pcache.zv, pcache.zks,
+                                   pcache.zvs, None, pre_pages, ws_p, stream)
+        for _ in range(3):
+            pre()
+        torch.cuda.synchronize(dev)
+        p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 10
+        p0.record(stream)
+        for _ in range(reps):
+            pre()
+        p1.record(stream)
+        torch.cuda.synchronize(dev)
+        pre_ms = p0.elapsed_time(p1) / reps
+        st_p, det_p = P.palu_get_device_status(ws_p)
+        if st_p:
+            raise RuntimeError(f"device status prefill={st_p}({det_p})")
+        pre_flops = 2.0 * n_pre * d_model * G * (w.rank_k + w.rank_v)
+        pk = measured_peaks()
+        prefill = {"tokens": n_pre, "ms": pre_ms, "tflops": pre_flops / pre_ms / 1e9,
+                   "frac_of_sustained_bf16": pre_flops / pre_ms / 1e9 / pk["bf16_tflops_sustained"],
+                   "kernel": "compress_tc_kernel (x·[A_k | A_v], tcgen05) + page scatter",
+                   "flops": pre_flops}
+        del pcache, xp, ws_p
+
     # ---- roofline of the dominant kernel (the decode step: split + combine)
     peaks = measured_peaks()
     mean_lens = [T0 + (first_step + args.steps / 2) + 0.5] * b
@@ -452,6 +489,7 @@ def run_ours(args):
         "clocks": clk.summary(),
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches,
+        **({"prefill": prefill} if prefill else {}),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, desc, threads, _ = oracle_sample(w, args.cpu_seconds)

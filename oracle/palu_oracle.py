@@ -56,6 +56,7 @@ __all__ = [
     "decode_attention_latent",
     "split_partials",
     "lse_combine",
+    "decode_attention_multi",
     "quantize_int4",
     "dequantize_int4",
     "cache_bytes_per_token",
@@ -186,6 +187,32 @@ def decode_attention(q, q_pos, z_k, z_v, pos, B_k, B_v, group_size, rope_base):
     for h in range(H):
         out[h], lse[h] = decode_attention_head(h, q, q_pos, z_k, z_v, pos, B_k, B_v,
                                                group_size, rope_base)
+    return out, lse
+
+
+def decode_attention_multi(q, q_pos, z_k, z_v, pos, B_k, B_v, group_size, rope_base):
+    """Several query tokens of one sequence in one step (multi-token decode).
+
+    q: [Q, H, d_h]; q_pos: [Q].  Query j attends to the cached tokens whose
+    position is at most its own, q_pos[j] (causal among the appended tokens;
+    [EXPL] §推理流程 Prefill / Decode 阶段 consume the same latent cache, and a
+    step that scores several new tokens at once is the same attention with a
+    per-query causal bound).  With one query at q_pos = T-1 this is
+    ``decode_attention``.  Returns (out [Q, H, d_h], lse [Q, H]); a query that
+    sees no token gives zeros and -inf.
+    """
+    q = np.asarray(q)
+    Q, H, d_h = q.shape
+    pos = np.asarray(pos)
+    out = np.zeros((Q, H, d_h))
+    lse = np.full((Q, H), -math.inf)
+    for j in range(Q):
+        keep = pos <= int(q_pos[j])
+        if not keep.any():
+            continue
+        zk_j, zv_j = z_k[:, keep], z_v[:, keep]
+        out[j], lse[j] = decode_attention(q[j], int(q_pos[j]), zk_j, zv_j, pos[keep], B_k, B_v,
+                                          group_size, rope_base)
     return out, lse
 
 

@@ -237,6 +237,48 @@ def test_brute_force_loops():
     np.testing.assert_allclose(out, brute_force_decode(c), rtol=0, atol=1e-12)
 
 
+def brute_force_multi(c, q, q_pos):
+    """Causal multi-query step by plain loops: each query over the tokens at or before it."""
+    outs = []
+    for j in range(len(q_pos)):
+        keep = [t for t in range(len(c["pos"])) if c["pos"][t] <= q_pos[j]]
+        cj = dict(c, q=q[j], q_pos=q_pos[j], z_k=c["z_k"][:, keep], z_v=c["z_v"][:, keep],
+                  pos=[c["pos"][t] for t in keep])
+        outs.append(brute_force_decode(cj) if keep else np.zeros(q[j].shape))
+    return np.array(outs)
+
+
+def test_multi_query_brute_force_and_causal_mask():
+    c = make_seq(31, H=4, d_h=4, g=2, r_k=3, r_v=2, T=7)
+    c["pos"] = np.array([0, 3, 1, 7, 2, 9, 5])
+    q = rng(32).standard_normal((3, 4, 4))
+    q_pos = np.array([4, 9, 1])
+    out, lse = O.decode_attention_multi(q, q_pos, c["z_k"], c["z_v"], c["pos"], c["B_k"], c["B_v"],
+                                        c["group_size"], c["rope_base"])
+    np.testing.assert_allclose(out, brute_force_multi(c, q, q_pos), rtol=0, atol=1e-12)
+    # a token after a query's position has no influence on it
+    zk2 = c["z_k"].copy()
+    zk2[:, 5] += 100.0                              # the token at position 9
+    out2, _ = O.decode_attention_multi(q, q_pos, zk2, c["z_v"], c["pos"], c["B_k"], c["B_v"],
+                                       c["group_size"], c["rope_base"])
+    np.testing.assert_array_equal(out2[0], out[0])
+    np.testing.assert_array_equal(out2[2], out[2])
+    assert np.abs(out2[1] - out[1]).max() > 1e-6
+    # a query before every token sees nothing
+    o3, l3 = O.decode_attention_multi(q[:1], np.array([-1]), c["z_k"], c["z_v"], c["pos"], c["B_k"],
+                                      c["B_v"], c["group_size"], c["rope_base"])
+    assert np.all(o3 == 0) and np.all(np.isneginf(l3))
+
+
+def test_multi_query_single_query_is_the_decode_step():
+    c = make_seq(33, T=29)
+    out, lse = O.decode_attention_multi(c["q"][None], np.array([c["q_pos"]]), c["z_k"], c["z_v"],
+                                        np.arange(29), c["B_k"], c["B_v"], c["group_size"], c["rope_base"])
+    ref, ref_lse = O.decode_attention(**dict(c, pos=np.arange(29)))
+    np.testing.assert_allclose(out[0], ref, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse[0], ref_lse, rtol=0, atol=1e-12)
+
+
 def test_latent_formulation_matches_materialised():
     c = make_seq(14, T=53)
     a, la = O.decode_attention(**c)

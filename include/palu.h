@@ -171,6 +171,32 @@ palu_status palu_decode_attn(const palu_config* cfg, int batch, const void* q, c
                              void* workspace, size_t workspace_bytes, int num_splits,
                              palu_stream_t stream);
 
+/* Multi-token decode step: num_queries (1..PALU_MAX_QUERIES) new tokens of
+ * every sequence query the cache at once, as when a step scores several
+ * appended tokens together (a chunk of a prompt, or drafted tokens to verify).
+ * "PALU 论文低秩投影分解" §把它放进一次真实推理流程里看: prefill and decode consume
+ * the same latent cache; each query is the decode step above, restricted to
+ * the cached tokens whose position is at most its own (causal among the new
+ * tokens, which the caller appends to the cache first).
+ *   q      [batch][num_queries][H][head_dim]   act dtype, before RoPE
+ *   q_pos  [batch][num_queries] int32          each query's position
+ *   out    [batch][num_queries][H][head_dim]   act dtype (written)
+ *   lse    [batch][num_queries][H] float32 or NULL
+ *   workspace >= palu_decode_multi_workspace_size bytes, 256-byte aligned
+ * Every other argument is as in palu_decode_attn.  A query that sees no token
+ * gives out = 0 and lse = -inf.  H·head_dim·(element size) must be a multiple of
+ * 16 bytes when num_queries > 1 (PALU_ERR_ALIGNMENT otherwise). */
+#define PALU_MAX_QUERIES 16
+palu_status palu_decode_multi_workspace_size(const palu_config* cfg, int batch, int num_queries,
+                                             int max_pages, int num_splits, size_t* bytes);
+palu_status palu_decode_attn_multi(const palu_config* cfg, int batch, int num_queries, const void* q,
+                                   const int32_t* q_pos, const void* zk_pool, const void* zv_pool,
+                                   const void* zk_scales, const void* zv_scales, const int32_t* pos_pool,
+                                   const int32_t* page_table, int max_pages, const int32_t* seq_lens,
+                                   int num_pages, const void* B_k, const void* B_v, void* out, float* lse,
+                                   void* workspace, size_t workspace_bytes, int num_splits,
+                                   palu_stream_t stream);
+
 /* Allocation-free decode step (the paper has no counterpart: this is a
  * deployment convenience of this library).
  * Some callers cannot call cudaMalloc at all: plug-ins whose host framework

@@ -43,6 +43,11 @@ SIGNATURES = {
                                      c_int, c_void_p, c_size_t, c_void_p]),
     "palu_decode_num_splits": (c_int, [_CFG, c_int, c_int, _P(c_int)]),
     "palu_decode_workspace_size": (c_int, [_CFG, c_int, c_int, c_int, _P(c_size_t)]),
+    "palu_decode_multi_workspace_size": (c_int, [_CFG, c_int, c_int, c_int, c_int, _P(c_size_t)]),
+    "palu_decode_attn_multi": (c_int, [_CFG, c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                       c_void_p, c_void_p, c_void_p, c_int, c_void_p, c_int, c_void_p,
+                                       c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_int,
+                                       c_void_p]),
     "palu_decode_attn": (c_int, [_CFG, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                  c_void_p, c_void_p, c_void_p, c_int, c_void_p, c_int, c_void_p,
                                  c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_int, c_void_p]),

@@ -133,6 +133,32 @@ def palu_decode_attn(cfg: PaluConfig, q, q_pos, zk_pool, zv_pool, zk_scales, zv_
     _check(st, "palu_decode_attn")
 
 
+MAX_QUERIES = 16
+
+
+def palu_decode_multi_workspace_size(cfg: PaluConfig, batch: int, num_queries: int, max_pages: int,
+                                     num_splits: int = 0) -> int:
+    out = ctypes.c_size_t()
+    _check(load().palu_decode_multi_workspace_size(ctypes.byref(cfg), batch, num_queries, max_pages,
+                                                   num_splits, ctypes.byref(out)),
+           "palu_decode_multi_workspace_size")
+    return int(out.value)
+
+
+def palu_decode_attn_multi(cfg: PaluConfig, q, q_pos, zk_pool, zv_pool, zk_scales, zv_scales, pos_pool,
+                           page_table, seq_lens, num_pages: int, B_k, B_v, out, lse, workspace,
+                           num_splits: int = 0, stream=None):
+    """Several query tokens per sequence: q [batch][Q][H][d_h], q_pos [batch][Q]; causal by position."""
+    batch, nq = q.shape[0], q.shape[1]
+    max_pages = page_table.shape[1]
+    st = load().palu_decode_attn_multi(
+        ctypes.byref(cfg), batch, nq, _ptr(q), _ptr(q_pos), _ptr(zk_pool), _ptr(zv_pool),
+        _ptr(zk_scales), _ptr(zv_scales), _ptr(pos_pool), _ptr(page_table), max_pages,
+        _ptr(seq_lens), num_pages, _ptr(B_k), _ptr(B_v), _ptr(out), _ptr(lse), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), num_splits, _stream(stream))
+    _check(st, "palu_decode_attn_multi")
+
+
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
 

@@ -121,7 +121,7 @@ __global__ void __launch_bounds__(256) fold_query_kernel(const DecodeArgs a, voi
     const int bb = i / (kMaxG * 128), h = (i / 128) % kMaxG, d = i % 128;
     float v = 0.f;
     if (b0 + bb < a.batch && h < gs && d < d_h)
-      v = Dt<ACT>::to_f(reinterpret_cast<const TA*>(a.q)[((size_t)(b0 + bb) * a.H + g * gs + h) * d_h + d]);
+      v = Dt<ACT>::to_f(reinterpret_cast<const TA*>(a.q)[(size_t)(b0 + bb) * a.q_bstride + (size_t)(g * gs + h) * d_h + d]);
     qs[bb][h][d] = v;
   }
   __syncthreads();
@@ -374,7 +374,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int k = 0; k < ntiles && ok; ++k) {
       const int slot = k & 1;
       const int t0 = (pg0 + k) * kTile;
-      const bool valid = t0 + row < t_end;
+      bool valid = t0 + row < t_end;
+      if (a.causal) {
+        // several queries per step: a token after the query's position is masked
+        int pos = t0 + row;
+        if (a.pos_pool != nullptr) {
+          const int pg = page_of(a, b, pg0 + k);
+          pos = pg >= 0 ? a.pos_pool[(size_t)pg * a.P + row] : 0;
+        }
+        valid = valid && pos <= a.q_pos[(size_t)b * a.qpos_bstride];
+      }
       if (!mbar_wait(bar(BAR_D_FULL + slot), (k >> 1) & 1, abort_flag, st, 31)) { ok = false; break; }
       tc_fence_after();
       float d[8];

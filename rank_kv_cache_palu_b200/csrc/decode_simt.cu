@@ -65,8 +65,8 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const DecodeArgs a) {
   const SplitRange rg = split_range(T, a.P, a.S, s);
 
   // Rotated query, with the softmax scale folded in.
-  const TA* qh = reinterpret_cast<const TA*>(a.q) + ((size_t)b * a.H + h) * d_h;
-  const int qpos = a.q_pos[b];
+  const TA* qh = reinterpret_cast<const TA*>(a.q) + (size_t)b * a.q_bstride + (size_t)h * d_h;
+  const int qpos = a.q_pos[(size_t)b * a.qpos_bstride];
   for (int i = tid; i < half; i += kThreads) {
     const float x1 = Dt<ACT>::to_f(qh[i]), x2 = Dt<ACT>::to_f(qh[i + half]);
     float c = 1.f, sn = 0.f;
@@ -165,7 +165,7 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const DecodeArgs a) {
       }
 #pragma unroll
       for (int off = 4; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
-      if (lane8 == 0 && tt < kTT) sc[tt] = (tt < nt) ? part : -INFINITY;
+      if (lane8 == 0 && tt < kTT) sc[tt] = (tt < nt && (!a.causal || tpos[tt] <= qpos)) ? part : -INFINITY;
     }
     __syncthreads();
     // ---- online softmax and the latent value sum
@@ -177,7 +177,7 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const DecodeArgs a) {
     float p[kTT];
 #pragma unroll
     for (int tt = 0; tt < kTT; ++tt) {
-      p[tt] = (tt < nt) ? expf(sc[tt] - m_new) : 0.f;
+      p[tt] = (tt < nt && m_new != -INFINITY) ? expf(sc[tt] - m_new) : 0.f;   // all masked so far: nothing
       psum += p[tt];
     }
     l_run = l_run * resc + psum;
@@ -221,10 +221,10 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const DecodeArgs a) {
 
   float M = -INFINITY;
   for (int s = 0; s < a.S; ++s) M = fmaxf(M, part[(size_t)s * (a.r_v + 2)]);
-  TA* out = reinterpret_cast<TA*>(a.out) + ((size_t)b * a.H + h) * a.d_h;
+  TA* out = reinterpret_cast<TA*>(a.out) + (size_t)b * a.o_bstride + (size_t)h * a.d_h;
   if (M == -INFINITY) {
     for (int d = tid; d < a.d_h; d += kThreads) out[d] = Dt<ACT>::from_f(0.f);
-    if (tid == 0 && a.lse != nullptr) a.lse[(size_t)b * a.H + h] = -INFINITY;
+    if (tid == 0 && a.lse != nullptr) a.lse[(size_t)b * a.lse_bstride + h] = -INFINITY;
     return;
   }
   float L = 0.f;
@@ -251,7 +251,7 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const DecodeArgs a) {
     for (int r = 0; r < a.r_v; ++r) o = fmaf(av[r], Dt<ACT>::to_f(Bv[(size_t)r * a.W + d]), o);
     out[d] = Dt<ACT>::from_f(o);
   }
-  if (tid == 0 && a.lse != nullptr) a.lse[(size_t)b * a.H + h] = M + logf(L);
+  if (tid == 0 && a.lse != nullptr) a.lse[(size_t)b * a.lse_bstride + h] = M + logf(L);
 }
 
 template <int ACT, int LAT>

@@ -622,10 +622,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (wg == 0) {
       const int hh = row >> 6, i = row & 63;
       using TA = typename Dt<ACT>::T;
-      const TA* qh = reinterpret_cast<const TA*>(a.q) + ((size_t)b * a.H + head0 + hh) * 128;
+      const TA* qh = reinterpret_cast<const TA*>(a.q) + (size_t)b * a.q_bstride + (size_t)(head0 + hh) * 128;
       const float x1 = Dt<ACT>::to_f(qh[i]), x2 = Dt<ACT>::to_f(qh[i + 64]);
       float c = 1.f, s = 0.f;
-      if (a.rope) rope_cs_fast(a.q_pos[b], a.omega[i], c, s);
+      if (a.rope) rope_cs_fast(a.q_pos[(size_t)b * a.qpos_bstride], a.omega[i], c, s);
       const float sc = a.sm_scale * kLog2e;
       const float qa = (x1 * c - x2 * s) * sc, qb = (x2 * c + x1 * s) * sc;
       qr[hh * 192 + i] = qa;
@@ -761,14 +761,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         return true;
       };
 
+      // causal bound (several queries per step): tokens after the query's position are masked
+      const int qlim = a.causal ? a.q_pos[(size_t)b * a.qpos_bstride] : 0;
       for (int k = 0; k < tr.ntiles && ok; ++k) {
         const int t0 = tr.t_begin + k * kTile;
-        const bool valid = t0 + row < tr.t_end;
         int pos = t0 + row;
         if (a.pos_pool != nullptr) {
           const int pg = page_of(a, b, t0 / kTile);
           pos = pg >= 0 ? a.pos_pool[(size_t)pg * a.P + row] : 0;
         }
+        const bool valid = t0 + row < tr.t_end && (!a.causal || pos <= qlim);
         const int slot = k & 1;
         if (!mbar_wait(bar(BAR_D_FULL + slot), (k >> 1) & 1, abort_flag, st, 31)) { ok = false; break; }
         tc_fence_after();
@@ -800,7 +802,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float* rr = red + (k & 1) * 8 + wg * 4;
         const float mt = fmaxf(fmaxf(rr[0], rr[1]), fmaxf(rr[2], rr[3]));
         const float m_new = fmaxf(m_run, mt);
-        const float scale = exp2f(m_run - m_new);                 // 0 on the first tile
+        // 0 on the first tile; 1 while every token so far is masked
+        const float scale = m_new == -INFINITY ? 1.f : exp2f(m_run - m_new);
         const uint16_t pb = to_bits<ACT>(valid ? exp2f(sc - m_new) : 0.f);
         *reinterpret_cast<uint16_t*>(sbase + L.p + slot * kPBytes + p_offset(hw, row)) = pb;
         l_part = fmaf(l_part, scale, from_bits<ACT>(pb));

@@ -69,6 +69,7 @@ void fill_omega(const palu_config* c, uint64_t* omega) {
 }
 
 constexpr size_t kStatusBytes = sizeof(palu::DevStatus);
+constexpr int kMaxQueries = PALU_MAX_QUERIES;
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
@@ -226,16 +227,24 @@ palu_status palu_decode_workspace_size(const palu_config* cfg, int batch, int ma
   return PALU_OK;
 }
 
-palu_status palu_decode_attn(const palu_config* cfg, int batch, const void* q, const int32_t* q_pos,
-                             const void* zk_pool, const void* zv_pool, const void* zk_scales,
-                             const void* zv_scales, const int32_t* pos_pool,
-                             const int32_t* page_table, int max_pages, const int32_t* seq_lens,
-                             int num_pages, const void* B_k, const void* B_v, void* out, float* lse,
-                             void* workspace, size_t workspace_bytes, int num_splits,
-                             palu_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// One decode step for Q queries per sequence (Q = 1: palu_decode_attn).  The
+// queries run one after another on the stream, each through the split kernel
+// and the combine, sharing the workspace; with Q > 1 a query attends only to
+// the tokens at or before its own position.
+palu_status decode_steps(const palu_config* cfg, int batch, int Q, const void* q, const int32_t* q_pos,
+                         const void* zk_pool, const void* zv_pool, const void* zk_scales,
+                         const void* zv_scales, const int32_t* pos_pool, const int32_t* page_table,
+                         int max_pages, const int32_t* seq_lens, int num_pages, const void* B_k,
+                         const void* B_v, void* out, float* lse, void* workspace, size_t workspace_bytes,
+                         int num_splits, palu_stream_t stream) {
   palu_status s = check_config(cfg);
   if (s != PALU_OK) return s;
-  if (batch < 0 || max_pages <= 0 || num_pages < 0 || num_splits < 0) return PALU_ERR_INVALID_ARG;
+  if (batch < 0 || max_pages <= 0 || num_pages < 0 || num_splits < 0 || Q < 1 || Q > kMaxQueries)
+    return PALU_ERR_INVALID_ARG;
   const int kind = kernel_kind(cfg);
   const int S = num_splits == 0 ? auto_splits(cfg, batch, max_pages, kind) : num_splits;
   if (S > max_pages) return PALU_ERR_INVALID_ARG;
@@ -292,12 +301,63 @@ palu_status palu_decode_attn(const palu_config* cfg, int batch, const void* q, c
   a.vs_row = palu::scale_row_bytes(a.lat, a.r_v);
   fill_omega(cfg, a.omega);
 
+  const long long qrow = (long long)a.H * a.d_h;       // one query's elements per sequence
+  const size_t elt = cfg->act_dtype == PALU_F32 ? 4 : 2;
+  if (Q > 1 && (qrow * (long long)elt) % 16 != 0) return PALU_ERR_ALIGNMENT;
+  a.q_bstride = Q * qrow;
+  a.o_bstride = Q * qrow;
+  a.qpos_bstride = Q;
+  a.lse_bstride = Q * a.H;
+  a.causal = Q > 1;
+
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = kind == 3   ? palu::launch_decode_fused(a, st)
-                  : kind == 2 ? palu::launch_decode_tc(a, st)
-                              : palu::launch_decode_simt(a, st);
-  if (e != cudaSuccess) return cuda_status(e);
-  return cuda_status(palu::launch_combine(a, st));
+  for (int j = 0; j < Q; ++j) {
+    a.q = static_cast<const char*>(q) + (size_t)j * qrow * elt;
+    a.q_pos = q_pos + j;
+    a.out = static_cast<char*>(out) + (size_t)j * qrow * elt;
+    a.lse = lse != nullptr ? lse + (size_t)j * a.H : nullptr;
+    cudaError_t e = kind == 3   ? palu::launch_decode_fused(a, st)
+                    : kind == 2 ? palu::launch_decode_tc(a, st)
+                                : palu::launch_decode_simt(a, st);
+    if (e != cudaSuccess) return cuda_status(e);
+    e = palu::launch_combine(a, st);
+    if (e != cudaSuccess) return cuda_status(e);
+  }
+  return PALU_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+palu_status palu_decode_attn(const palu_config* cfg, int batch, const void* q, const int32_t* q_pos,
+                             const void* zk_pool, const void* zv_pool, const void* zk_scales,
+                             const void* zv_scales, const int32_t* pos_pool,
+                             const int32_t* page_table, int max_pages, const int32_t* seq_lens,
+                             int num_pages, const void* B_k, const void* B_v, void* out, float* lse,
+                             void* workspace, size_t workspace_bytes, int num_splits,
+                             palu_stream_t stream) {
+  return decode_steps(cfg, batch, 1, q, q_pos, zk_pool, zv_pool, zk_scales, zv_scales, pos_pool, page_table,
+                      max_pages, seq_lens, num_pages, B_k, B_v, out, lse, workspace, workspace_bytes, num_splits,
+                      stream);
+}
+
+palu_status palu_decode_multi_workspace_size(const palu_config* cfg, int batch, int num_queries, int max_pages,
+                                             int num_splits, size_t* bytes) {
+  if (num_queries < 1 || num_queries > kMaxQueries) return PALU_ERR_INVALID_ARG;
+  return palu_decode_workspace_size(cfg, batch, max_pages, num_splits, bytes);
+}
+
+palu_status palu_decode_attn_multi(const palu_config* cfg, int batch, int num_queries, const void* q,
+                                   const int32_t* q_pos, const void* zk_pool, const void* zv_pool,
+                                   const void* zk_scales, const void* zv_scales, const int32_t* pos_pool,
+                                   const int32_t* page_table, int max_pages, const int32_t* seq_lens,
+                                   int num_pages, const void* B_k, const void* B_v, void* out, float* lse,
+                                   void* workspace, size_t workspace_bytes, int num_splits,
+                                   palu_stream_t stream) {
+  return decode_steps(cfg, batch, num_queries, q, q_pos, zk_pool, zv_pool, zk_scales, zv_scales, pos_pool,
+                      page_table, max_pages, seq_lens, num_pages, B_k, B_v, out, lse, workspace, workspace_bytes,
+                      num_splits, stream);
 }
 
 palu_status palu_get_device_status(void* workspace, palu_stream_t stream, int32_t* detail) {

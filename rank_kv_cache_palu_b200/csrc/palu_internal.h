@@ -21,6 +21,12 @@ struct DecodeArgs {
   float sm_scale;      // 1/sqrt(d_h)
   const void* q;
   const int32_t* q_pos;
+  // Per-sequence strides of q / q_pos / out / lse (elements): H·d_h, 1, H·d_h,
+  // H for one query per sequence; Q times that when a step holds Q queries
+  // and one launch serves one of them.
+  long long q_bstride, o_bstride;
+  int qpos_bstride, lse_bstride;
+  int causal;          // 1: a token counts only if its position <= the query's position
   const void* zk;
   const void* zv;
   const void* zks;

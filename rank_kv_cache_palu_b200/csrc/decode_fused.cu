@@ -44,28 +44,11 @@ constexpr int kMaxG = 4;            // heads per group the fused kernel takes
 constexpr int kNZK = 6;             // z_k ring stages
 constexpr int kNZV = 4;             // z_v ring stages (pairs of column blocks)
 constexpr int kStageBytes = kTile * kChunk * 2;   // 16 KB: one column block of a page
-constexpr int kPBytes = 16 * kTile * 2;           // P tile: 16 rows (heads, padded) × 128 tokens
-constexpr int kTmemCols = 128;      // D: 2 × 16 columns; aᵀ: 2 × 32 columns
+constexpr int kFusedMaxQueries = 4;  // queries of one sequence that share a pass over the cache
 
 struct Smem {
   uint32_t qt, zk, zv, p, red, lred, bars, tmem_slot, abort, total;
 };
-
-__host__ __device__ inline Smem smem_layout(int r_k) {
-  Smem s{};
-  uint32_t o = 0;
-  s.qt = o;   o += (uint32_t)(r_k / kChunk) * 16 * 128;   // [K chunk][16 rows][128 B], 128-byte swizzle
-  s.zk = o;   o += kNZK * kStageBytes;
-  s.zv = o;   o += kNZV * kStageBytes;
-  s.p = o;    o += 2 * kPBytes;
-  s.red = o;  o += 2 * 4 * kMaxG * 4;                    // [tile parity][warp][head] maxima
-  s.lred = o; o += 4 * kMaxG * 4;                        // [warp][head] softmax denominators
-  s.bars = o; o += 32 * 8;
-  s.tmem_slot = o; o += 16;
-  s.abort = o;     o += 16;
-  s.total = o;
-  return s;
-}
 
 enum {
   BAR_ZK_FULL = 0,
@@ -88,13 +71,6 @@ __device__ __forceinline__ int page_of(const DecodeArgs& a, int b, int lp) {
   return (pg < 0 || pg >= a.num_pages) ? -1 : pg;
 }
 
-// P tile, K-major with the 128-byte swizzle: row n (head), token k; tokens
-// 0-63 and 64-127 sit in two 2 KB atoms of 16 rows.
-__device__ __forceinline__ uint32_t p_offset(int n, int k) {
-  const int region = k >> 6, kin = k & 63;
-  return (uint32_t)(region * 2048 + n * 128 + (((kin >> 3) ^ (n & 7)) << 4) + (kin & 7) * 2);
-}
-
 template <int ACT>
 __device__ __forceinline__ uint16_t to_bits(float v) {
   const auto h = Dt<ACT>::from_f(v);
@@ -106,22 +82,29 @@ __device__ __forceinline__ float from_bits(uint16_t u) {
 }
 
 // q̃ = B_k,h q_h (scaled) for the heads of one group, as hi + lo 16-bit rows:
-// out[b][g][h] = hi, out[b][g][4 + h] = lo (h < gs; other rows zero), each r_k
-// long.  CTA (g, 64 latent entries, 4 sequences); thread (entry j, head h)
-// holds the B_k row segment B_k[g][j][h·d_h, +d_h) in registers and takes its
-// dot product with the query of each of the 4 sequences.
+// out[vb][g][h] = hi, out[vb][g][4 + h] = lo (h < gs; other rows zero), each
+// r_k long, for virtual sequence vb = b·qslots + jj (query jj of the pass; a
+// single query per step is qslots = 1).  CTA (g, 64 latent entries, 4 virtual
+// sequences); thread (entry j, head h) holds the B_k row segment
+// B_k[g][j][h·d_h, +d_h) in registers and takes its dot product with each
+// query.
 constexpr int kFoldSeqs = 4;
 template <int ACT>
-__global__ void __launch_bounds__(256) fold_query_kernel(const DecodeArgs a, void* qt) {
+__global__ void __launch_bounds__(256) fold_query_kernel(const DecodeArgs a, int qslots, void* qt) {
   using TA = typename Dt<ACT>::T;
   __shared__ float qs[kFoldSeqs][kMaxG][128];
-  const int g = blockIdx.x, jb = blockIdx.y, b0 = blockIdx.z * kFoldSeqs;
+  const int g = blockIdx.x, jb = blockIdx.y, v0 = blockIdx.z * kFoldSeqs;
   const int gs = a.gs, d_h = a.d_h;
+  const int nvb = a.batch * qslots;
+  auto live = [&](int vb) { return vb < nvb && vb % qslots < a.qn; };
   for (int i = threadIdx.x; i < kFoldSeqs * kMaxG * 128; i += blockDim.x) {
     const int bb = i / (kMaxG * 128), h = (i / 128) % kMaxG, d = i % 128;
+    const int vb = v0 + bb;
     float v = 0.f;
-    if (b0 + bb < a.batch && h < gs && d < d_h)
-      v = Dt<ACT>::to_f(reinterpret_cast<const TA*>(a.q)[(size_t)(b0 + bb) * a.q_bstride + (size_t)(g * gs + h) * d_h + d]);
+    if (live(vb) && h < gs && d < d_h)
+      v = Dt<ACT>::to_f(reinterpret_cast<const TA*>(a.q)[(size_t)(vb / qslots) * a.q_bstride +
+                                                          (size_t)(vb % qslots) * a.H * d_h +
+                                                          (size_t)(g * gs + h) * d_h + d]);
     qs[bb][h][d] = v;
   }
   __syncthreads();
@@ -136,7 +119,8 @@ __global__ void __launch_bounds__(256) fold_query_kernel(const DecodeArgs a, voi
   for (int v = 0; v < 16; ++v) bseg[v] = (h < gs && v * 8 < d_h) ? __ldg(src + v) : make_uint4(0, 0, 0, 0);
   constexpr float kLog2e = 1.4426950408889634f;
   const float sc = a.sm_scale * kLog2e;
-  for (int bb = 0; bb < kFoldSeqs && b0 + bb < a.batch; ++bb) {
+  for (int bb = 0; bb < kFoldSeqs; ++bb) {
+    if (!live(v0 + bb)) continue;
     float acc = 0.f;
 #pragma unroll
     for (int v = 0; v < 16; ++v) {
@@ -147,20 +131,62 @@ __global__ void __launch_bounds__(256) fold_query_kernel(const DecodeArgs a, voi
     acc *= sc;
     const TA hi = Dt<ACT>::from_f(acc);
     const TA lo = Dt<ACT>::from_f(acc - Dt<ACT>::to_f(hi));
-    TA* out = reinterpret_cast<TA*>(qt) + ((size_t)(b0 + bb) * a.G + g) * 2 * kMaxG * a.r_k;
+    TA* out = reinterpret_cast<TA*>(qt) + ((size_t)(v0 + bb) * a.G + g) * 2 * kMaxG * a.r_k;
     out[(size_t)h * a.r_k + j] = hi;
     out[(size_t)(kMaxG + h) * a.r_k + j] = lo;
   }
 }
 
-template <int ACT, int NRV>
+// Shape of one pass: QN queries of a sequence share each streamed tile.
+//   score MMA:  N = 8·QN rows of q̃ (query jj, hi/lo part, head h -> row 8jj + 4·lo + h)
+//   value MMA:  N = 4·QN rows of P (query jj, head h -> row 4jj + h), padded to 16
+template <int QN>
+struct Pass {
+  static constexpr int kN = 8 * QN < 16 ? 16 : 8 * QN;
+  static constexpr int kPC = kMaxG * QN;                 // (query, head) pairs
+  static constexpr int kNP = (kPC + 15) / 16 * 16;
+  static constexpr int kPBytes = kNP * kTile * 2;         // P tile: kNP rows × 128 tokens
+  static constexpr int kPRegion = kNP * 128;              // bytes per 64 tokens of P
+  static constexpr int kAt = 2 * kN;                      // first aᵀ column
+  static constexpr int kTmem = 2 * kN + 2 * 2 * kNP <= 128 ? 128 : 256;
+};
+
+template <int QN>
+__host__ __device__ inline Smem smem_layout(int r_k) {
+  using PS = Pass<QN>;
+  Smem s{};
+  uint32_t o = 0;
+  s.qt = o;   o += (uint32_t)(r_k / kChunk) * PS::kN * 128;   // [K chunk][kN rows][128 B], 128-byte swizzle
+  s.zk = o;   o += kNZK * kStageBytes;
+  s.zv = o;   o += kNZV * kStageBytes;
+  s.p = o;    o += 2 * PS::kPBytes;
+  s.red = o;  o += 2 * 4 * PS::kPC * 4;                  // [tile parity][warp][pair] maxima
+  s.lred = o; o += 4 * PS::kPC * 4;                      // [warp][pair] softmax denominators
+  s.bars = o; o += 32 * 8;
+  s.tmem_slot = o; o += 16;
+  s.abort = o;     o += 16;
+  s.total = o;
+  return s;
+}
+
+// P tile, K-major with the 128-byte swizzle: row n ((query, head) pair), token
+// k; tokens 0-63 and 64-127 sit in two atoms of kNP rows.
+template <int QN>
+__device__ __forceinline__ uint32_t p_offset(int n, int k) {
+  const int region = k >> 6, kin = k & 63;
+  return (uint32_t)(region * Pass<QN>::kPRegion + n * 128 + (((kin >> 3) ^ (n & 7)) << 4) + (kin & 7) * 2);
+}
+
+template <int ACT, int NRV, int QN>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_fused_kernel(const DecodeArgs a, const void* qt) {
+  using PS = Pass<QN>;
+  constexpr int kN = PS::kN, kNP = PS::kNP, kPC = PS::kPC, kPB = PS::kPBytes;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* sbase = smem_raw + (base - raw);
-  const Smem L = smem_layout(a.r_k);
+  const Smem L = smem_layout<QN>(a.r_k);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   DevStatus* st = reinterpret_cast<DevStatus*>(a.status);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sbase + L.abort);
@@ -168,6 +194,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int gs = a.gs;
+  const int nq = a.qn;                  // queries of this pass (<= QN)
   const int nkc = a.r_k / kChunk;
   int T = a.seq_lens[b];
   const int cap = a.max_pages * a.P;
@@ -206,22 +233,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(base + L.tmem_slot, kTmemCols);
+    tmem_alloc(base + L.tmem_slot, PS::kTmem);
     tmem_relinquish();
   }
-  // P padding rows stay zero; q̃ rows 2·gs..15 stay zero
-  for (int i = threadIdx.x; i < 2 * kPBytes / 4; i += kThreads) reinterpret_cast<uint32_t*>(sbase + L.p)[i] = 0u;
-  for (int i = threadIdx.x; i < nkc * 16 * 32; i += kThreads) reinterpret_cast<uint32_t*>(sbase + L.qt)[i] = 0u;   // rows 8-15
+  // P padding rows stay zero; q̃ rows of absent queries stay zero
+  for (int i = threadIdx.x; i < 2 * kPB / 4; i += kThreads) reinterpret_cast<uint32_t*>(sbase + L.p)[i] = 0u;
+  for (int i = threadIdx.x; i < nkc * kN * 32; i += kThreads) reinterpret_cast<uint32_t*>(sbase + L.qt)[i] = 0u;
   __syncthreads();
-  // q̃ into the K-major swizzled B operand: row n (hi/lo head), entry j
-  {
-    const uint16_t* src = reinterpret_cast<const uint16_t*>(qt) + ((size_t)b * a.G + g) * 2 * kMaxG * a.r_k;
-    for (int i = threadIdx.x; i < 2 * kMaxG * a.r_k; i += kThreads) {
-      const int n = i / a.r_k, j = i % a.r_k;
-      const int c = j / kChunk, kin = j % kChunk;
-      *reinterpret_cast<uint16_t*>(sbase + L.qt + c * 2048 + n * 128 + ((((kin >> 3) ^ (n & 7))) << 4) + (kin & 7) * 2) =
-          src[i];
-    }
+  // q̃ into the K-major swizzled B operand: row n = 8·jj + r of query jj, entry j
+  for (int i = threadIdx.x; i < nq * 2 * kMaxG * a.r_k; i += kThreads) {
+    const int n = i / a.r_k, j = i % a.r_k;
+    const int jj = n >> 3, r = n & 7;
+    const uint16_t* src = reinterpret_cast<const uint16_t*>(qt) +
+                          ((((size_t)b * QN + jj) * a.G + g) * 2 * kMaxG + r) * a.r_k;
+    const int c = j / kChunk, kin = j % kChunk;
+    *reinterpret_cast<uint16_t*>(sbase + L.qt + c * (kN * 128) + n * 128 + (((kin >> 3) ^ (n & 7)) << 4) +
+                                 (kin & 7) * 2) = src[j];
   }
   fence_proxy_async();
   tc_fence_before();
@@ -273,14 +300,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ============================================================ MMA issuer
     if (lane == 0) {
       constexpr int kBf = ACT == PALU_BF16 ? 1 : 0;
-      const uint32_t idesc_s = idesc_f16(kBf, 0, 0, 16, 128);    // z_k K-major, q̃ K-major
-      const uint32_t idesc_pv = idesc_f16(kBf, 1, 0, 16, 128);   // z_vᵀ MN-major, Pᵀ K-major
+      const uint32_t idesc_s = idesc_f16(kBf, 0, 0, kN, 128);    // z_k K-major, q̃ K-major
+      const uint32_t idesc_pv = idesc_f16(kBf, 1, 0, kNP, 128);  // z_vᵀ MN-major, Pᵀ K-major
       int zs = 0, vs = 0;
       uint32_t zph = 0, vph = 0;
       bool ok = true;
       auto issue_pv = [&](int j) -> bool {
-        const uint32_t a_tmem = tmem + 32 + (uint32_t)(j & 1) * 32;
-        const uint32_t p_base = base + L.p + (uint32_t)(j & 1) * kPBytes;
+        const uint32_t a_tmem = tmem + PS::kAt + (uint32_t)(j & 1) * NRV * kNP;
+        const uint32_t p_base = base + L.p + (uint32_t)(j & 1) * kPB;
         if (!mbar_wait(bar(BAR_P_FULL + (j & 1)), (j >> 1) & 1, abort_flag, st, 21)) return false;
         if (!mbar_wait(bar(BAR_AT_EMPTY + (j & 1)), ((j >> 1) & 1) ^ 1, abort_flag, st, 22)) return false;
         tc_fence_after();
@@ -291,8 +318,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk) {
             const uint64_t ad = sdesc(base + L.zv + vs * kStageBytes + kk * 16 * 128, kStageBytes, 1024, kSw128);
-            const uint64_t bd = sdesc(p_base + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024, kSw128);
-            umma_f16(a_tmem + mb * 16, ad, bd, idesc_pv, kk != 0);
+            const uint64_t bd = sdesc(p_base + (kk >> 2) * PS::kPRegion + (kk & 3) * 32, 16, 1024, kSw128);
+            umma_f16(a_tmem + mb * kNP, ad, bd, idesc_pv, kk != 0);
           }
           umma_commit(bar(BAR_ZV_EMPTY + vs));
           umma_commit(bar(BAR_ZV_EMPTY + vs + 1));
@@ -306,14 +333,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int slot = k & 1;
         if (!mbar_wait(bar(BAR_D_EMPTY + slot), ((k >> 1) & 1) ^ 1, abort_flag, st, 24)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t d_tmem = tmem + (uint32_t)slot * 16;
+        const uint32_t d_tmem = tmem + (uint32_t)slot * kN;
         for (int c = 0; c < nkc; ++c) {
           if (!mbar_wait(bar(BAR_ZK_FULL + zs), zph, abort_flag, st, 25)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < kChunk / 16; ++kk) {
             const uint64_t ad = sdesc(base + L.zk + zs * kStageBytes + kk * 32, 16, 1024, kSw128);
-            const uint64_t bd = sdesc(base + L.qt + c * 2048 + kk * 32, 16, 1024, kSw128);
+            const uint64_t bd = sdesc(base + L.qt + c * (kN * 128) + kk * 32, 16, 1024, kSw128);
             umma_f16(d_tmem, ad, bd, idesc_s, (c | kk) != 0);
           }
           umma_commit(bar(BAR_ZK_EMPTY + zs));
@@ -330,6 +357,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ============================================================ epilogue (warps 2-5)
+    // One thread per token row (scores) and per latent row (value sums); the
+    // (query, head) pairs of the pass are p = 4·jj + h.
     const int q4 = warp & 3;                 // TMEM lane quarter this warp may access
     const int row = q4 * 32 + lane;          // token row of the tile / latent row of aᵀ
     const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
@@ -342,28 +371,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       epi_phase ^= 1;
       return r;
     };
-    float m_run[kMaxG], l_part[kMaxG], prev_scale[kMaxG];
-    float acc[NRV][kMaxG];
+    auto live = [&](int p) { return (p & 3) < gs && (p >> 2) < nq; };
+    int qlim[QN];
 #pragma unroll
-    for (int h = 0; h < kMaxG; ++h) {
-      m_run[h] = -INFINITY;
-      l_part[h] = 0.f;
-      prev_scale[h] = 0.f;
+    for (int jj = 0; jj < QN; ++jj) qlim[jj] = (a.causal && jj < nq) ? a.q_pos[(size_t)b * a.qpos_bstride + jj] : 0;
+    float m_run[kPC], l_part[kPC], prev_scale[kPC];
+    float acc[NRV][kPC];
 #pragma unroll
-      for (int mb = 0; mb < NRV; ++mb) acc[mb][h] = 0.f;
+    for (int p = 0; p < kPC; ++p) {
+      m_run[p] = -INFINITY;
+      l_part[p] = 0.f;
+      prev_scale[p] = 0.f;
+#pragma unroll
+      for (int mb = 0; mb < NRV; ++mb) acc[mb][p] = 0.f;
     }
     auto fold_at = [&](int j) -> bool {
       if (!mbar_wait(bar(BAR_AT_FULL + (j & 1)), (j >> 1) & 1, abort_flag, st, 30)) return false;
       tc_fence_after();
 #pragma unroll
       for (int mb = 0; mb < NRV; ++mb) {
-        float v[4];
-        tmem_ld2(tmem + lane_addr + 32 + (uint32_t)(j & 1) * 32 + mb * 16, v);
-        tmem_ld2(tmem + lane_addr + 32 + (uint32_t)(j & 1) * 32 + mb * 16 + 2, v + 2);
+        float v[kPC];
+#pragma unroll
+        for (int c = 0; c < kPC; c += 2)
+          tmem_ld2(tmem + lane_addr + PS::kAt + (uint32_t)(j & 1) * NRV * kNP + mb * kNP + c, v + c);
         tmem_wait_ld();
 #pragma unroll
-        for (int h = 0; h < kMaxG; ++h)
-          if (h < gs) acc[mb][h] = fmaf(acc[mb][h], prev_scale[h], v[h]);
+        for (int p = 0; p < kPC; ++p)
+          if (live(p)) acc[mb][p] = fmaf(acc[mb][p], prev_scale[p], v[p]);
       }
       tc_fence_before();
       __syncwarp();
@@ -374,23 +408,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int k = 0; k < ntiles && ok; ++k) {
       const int slot = k & 1;
       const int t0 = (pg0 + k) * kTile;
-      bool valid = t0 + row < t_end;
-      if (a.causal) {
-        // several queries per step: a token after the query's position is masked
-        int pos = t0 + row;
-        if (a.pos_pool != nullptr) {
-          const int pg = page_of(a, b, pg0 + k);
-          pos = pg >= 0 ? a.pos_pool[(size_t)pg * a.P + row] : 0;
-        }
-        valid = valid && pos <= a.q_pos[(size_t)b * a.qpos_bstride];
+      const bool in_seq = t0 + row < t_end;
+      int pos = t0 + row;
+      if (a.causal && a.pos_pool != nullptr) {
+        const int pg = page_of(a, b, pg0 + k);
+        pos = pg >= 0 ? a.pos_pool[(size_t)pg * a.P + row] : 0;
       }
       if (!mbar_wait(bar(BAR_D_FULL + slot), (k >> 1) & 1, abort_flag, st, 31)) { ok = false; break; }
       tc_fence_after();
-      float d[8];
-      tmem_ld2(tmem + lane_addr + slot * 16, d);
-      tmem_ld2(tmem + lane_addr + slot * 16 + 2, d + 2);
-      tmem_ld2(tmem + lane_addr + slot * 16 + 4, d + 4);
-      tmem_ld2(tmem + lane_addr + slot * 16 + 6, d + 6);
+      float d[8 * QN];
+#pragma unroll
+      for (int c = 0; c < 8 * QN; c += 2) tmem_ld2(tmem + lane_addr + slot * kN + c, d + c);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
@@ -398,28 +426,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the previous tile's latent sums are ready by now (its value MMA went
       // in behind this tile's scores)
       if (k >= 1 && !fold_at(k - 1)) { ok = false; break; }
-      float sc[kMaxG];
+      float sc[kPC];
+      bool valid[QN];
 #pragma unroll
-      for (int h = 0; h < kMaxG; ++h) {
-        sc[h] = (valid && h < gs) ? d[h] + d[kMaxG + h] : -INFINITY;   // hi and lo parts of q̃
-        float m = sc[h];
+      for (int jj = 0; jj < QN; ++jj)
+        valid[jj] = in_seq && jj < nq && (!a.causal || pos <= qlim[jj]);   // causal among the new tokens
+#pragma unroll
+      for (int p = 0; p < kPC; ++p) {
+        const int jj = p >> 2, h = p & 3;
+        sc[p] = (valid[jj] && h < gs) ? d[8 * jj + h] + d[8 * jj + 4 + h] : -INFINITY;   // hi and lo parts of q̃
+        float m = sc[p];
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-        if (lane == 0) red[((k & 1) * 4 + q4) * kMaxG + h] = m;
+        if (lane == 0) red[((k & 1) * 4 + q4) * kPC + p] = m;
       }
       if (!ep_sync(33)) { ok = false; break; }
 #pragma unroll
-      for (int h = 0; h < kMaxG; ++h) {
-        if (h >= gs) continue;
-        const float* rr = red + (k & 1) * 4 * kMaxG + h;
-        const float mt = fmaxf(fmaxf(rr[0], rr[kMaxG]), fmaxf(rr[2 * kMaxG], rr[3 * kMaxG]));
-        const float m_new = fmaxf(m_run[h], mt);
-        const float scale = m_new == -INFINITY ? 1.f : exp2f(m_run[h] - m_new);
-        const uint16_t pb = to_bits<ACT>(valid ? exp2f(sc[h] - m_new) : 0.f);
-        *reinterpret_cast<uint16_t*>(sbase + L.p + slot * kPBytes + p_offset(h, row)) = pb;
-        l_part[h] = fmaf(l_part[h], scale, from_bits<ACT>(pb));
-        m_run[h] = m_new;
-        prev_scale[h] = scale;
+      for (int p = 0; p < kPC; ++p) {
+        if (!live(p)) continue;
+        const float* rr = red + (k & 1) * 4 * kPC + p;
+        const float mt = fmaxf(fmaxf(rr[0], rr[kPC]), fmaxf(rr[2 * kPC], rr[3 * kPC]));
+        const float m_new = fmaxf(m_run[p], mt);
+        const float scale = m_new == -INFINITY ? 1.f : exp2f(m_run[p] - m_new);   // 1 while all masked
+        const uint16_t pb = to_bits<ACT>(sc[p] != -INFINITY ? exp2f(sc[p] - m_new) : 0.f);
+        *reinterpret_cast<uint16_t*>(sbase + L.p + slot * kPB + p_offset<QN>(p, row)) = pb;
+        l_part[p] = fmaf(l_part[p], scale, from_bits<ACT>(pb));
+        m_run[p] = m_new;
+        prev_scale[p] = scale;
       }
       fence_proxy_async();
       __syncwarp();
@@ -436,59 +469,57 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int t0 = (pg0 + kl) * kTile;
         const int nvalid = t_end - t0;
         const int pg = page_of(a, b, pg0 + kl);
-        float at[NRV][kMaxG];
+        float at[NRV][kPC];
 #pragma unroll
         for (int mb = 0; mb < NRV; ++mb)
 #pragma unroll
-          for (int h = 0; h < kMaxG; ++h) at[mb][h] = 0.f;
+          for (int p = 0; p < kPC; ++p) at[mb][p] = 0.f;
         if (pg >= 0) {
           const uint8_t* zv = reinterpret_cast<const uint8_t*>(a.zv) + (size_t)(pg * a.G + g) * a.P * a.v_row;
-          const uint8_t* pbuf = sbase + L.p + (kl & 1) * kPBytes;
+          const uint8_t* pbuf = sbase + L.p + (kl & 1) * kPB;
           for (int t = 0; t < nvalid; ++t) {
             float z[NRV];
 #pragma unroll
             for (int mb = 0; mb < NRV; ++mb) z[mb] = load_latent<ACT, ACT>(zv, t, a.P, nullptr, mb * 128 + row);
 #pragma unroll
-            for (int h = 0; h < kMaxG; ++h) {
-              if (h >= gs) continue;
-              const float pv = from_bits<ACT>(*reinterpret_cast<const uint16_t*>(pbuf + p_offset(h, t)));
+            for (int p = 0; p < kPC; ++p) {
+              if (!live(p)) continue;
+              const float pv = from_bits<ACT>(*reinterpret_cast<const uint16_t*>(pbuf + p_offset<QN>(p, t)));
 #pragma unroll
-              for (int mb = 0; mb < NRV; ++mb) at[mb][h] = fmaf(pv, z[mb], at[mb][h]);
+              for (int mb = 0; mb < NRV; ++mb) at[mb][p] = fmaf(pv, z[mb], at[mb][p]);
             }
           }
         }
 #pragma unroll
         for (int mb = 0; mb < NRV; ++mb)
 #pragma unroll
-          for (int h = 0; h < kMaxG; ++h) acc[mb][h] = fmaf(acc[mb][h], prev_scale[h], at[mb][h]);
+          for (int p = 0; p < kPC; ++p) acc[mb][p] = fmaf(acc[mb][p], prev_scale[p], at[mb][p]);
       }
     }
-    // l per head: sum of the per-thread partials
+    // l per pair: sum of the per-thread partials
     float* lred = reinterpret_cast<float*>(sbase + L.lred);
 #pragma unroll
-    for (int h = 0; h < kMaxG; ++h) {
-      float v = l_part[h];
+    for (int p = 0; p < kPC; ++p) {
+      float v = l_part[p];
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-      if (lane == 0) lred[q4 * kMaxG + h] = v;
+      if (lane == 0) lred[q4 * kPC + p] = v;
     }
     ok = ep_sync(35) && ok;
-    float lsum[kMaxG];
-#pragma unroll
-    for (int h = 0; h < kMaxG; ++h)
-      lsum[h] = (lred[h] + lred[kMaxG + h]) + (lred[2 * kMaxG + h] + lred[3 * kMaxG + h]);
     if (ok && !*abort_flag) {
       constexpr float kLn2 = 0.6931471805599453f;
 #pragma unroll
-      for (int h = 0; h < kMaxG; ++h) {
-        if (h >= gs) continue;
-        float* out = a.part + (((size_t)b * a.H + g * gs + h) * a.S + s) * (a.r_v + 2);
+      for (int p = 0; p < kPC; ++p) {
+        if (!live(p)) continue;
+        const int jj = p >> 2, h = p & 3;
+        // partials of virtual sequence b·QN + jj (the combine maps it back)
+        float* out = a.part + ((((size_t)b * QN + jj) * a.H + g * gs + h) * a.S + s) * (a.r_v + 2);
         if (row == 0) {
-          out[0] = ntiles > 0 ? m_run[h] * kLn2 : -INFINITY;
-          out[1] = lsum[h];
+          out[0] = ntiles > 0 ? m_run[p] * kLn2 : -INFINITY;
+          out[1] = (lred[p] + lred[kPC + p]) + (lred[2 * kPC + p] + lred[3 * kPC + p]);
         }
 #pragma unroll
-        for (int mb = 0; mb < NRV; ++mb) out[2 + mb * 128 + row] = acc[mb][h];
+        for (int mb = 0; mb < NRV; ++mb) out[2 + mb * 128 + row] = acc[mb][p];
       }
     }
   }
@@ -498,25 +529,36 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc(tmem, PS::kTmem);
   }
 }
 
-template <int ACT, int NRV>
+template <int ACT, int NRV, int QN>
 cudaError_t launch_t(const DecodeArgs& a, cudaStream_t st) {
   void* qt = a.fused_q;
-  fold_query_kernel<ACT><<<dim3(a.G, (a.r_k + 63) / 64, (a.batch + kFoldSeqs - 1) / kFoldSeqs), 256, 0, st>>>(a, qt);
+  const int vb = a.batch * QN;   // one folded query per (sequence, query slot of the pass)
+  fold_query_kernel<ACT><<<dim3(a.G, (a.r_k + 63) / 64, (vb + kFoldSeqs - 1) / kFoldSeqs), 256, 0, st>>>(a, QN, qt);
   count_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const Smem L = smem_layout(a.r_k);
+  const Smem L = smem_layout<QN>(a.r_k);
   const size_t smem = L.total + 1024;
-  auto kern = decode_fused_kernel<ACT, NRV>;
+  auto kern = decode_fused_kernel<ACT, NRV, QN>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   kern<<<dim3(a.S, a.G, a.batch), kThreads, smem, st>>>(a, qt);
   count_launch();
   return cudaGetLastError();
+}
+
+// A pass serves exactly 1, 2 or 4 queries of every sequence (the caller splits
+// a step's queries into such passes).
+template <int ACT, int NRV>
+cudaError_t launch_q(const DecodeArgs& a, cudaStream_t st) {
+  if (a.qn == 1) return launch_t<ACT, NRV, 1>(a, st);
+  if (a.qn == 2) return launch_t<ACT, NRV, 2>(a, st);
+  if (a.qn == 4) return launch_t<ACT, NRV, 4>(a, st);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace
@@ -528,8 +570,10 @@ bool fused_decode_supported(const palu_config* c) {
   if (c->latent_dtype != c->act_dtype) return false;
   if (c->rank_k % 64 != 0 || c->rank_k > 512) return false;
   if (c->rank_v != 128 && c->rank_v != 256) return false;
-  return smem_layout(c->rank_k).total + 1024 <= 227 * 1024;
+  return smem_layout<kFusedMaxQueries>(c->rank_k).total + 1024 <= 227 * 1024;
 }
+
+int fused_queries_per_pass() { return kFusedMaxQueries; }
 
 size_t fused_query_bytes(const palu_config* c, int batch) {
   const size_t G = (size_t)(c->num_heads / c->group_size);
@@ -537,8 +581,8 @@ size_t fused_query_bytes(const palu_config* c, int batch) {
 }
 
 cudaError_t launch_decode_fused(const DecodeArgs& a, cudaStream_t st) {
-  if (a.act == PALU_BF16) return a.r_v == 256 ? launch_t<PALU_BF16, 2>(a, st) : launch_t<PALU_BF16, 1>(a, st);
-  return a.r_v == 256 ? launch_t<PALU_F16, 2>(a, st) : launch_t<PALU_F16, 1>(a, st);
+  if (a.act == PALU_BF16) return a.r_v == 256 ? launch_q<PALU_BF16, 2>(a, st) : launch_q<PALU_BF16, 1>(a, st);
+  return a.r_v == 256 ? launch_q<PALU_F16, 2>(a, st) : launch_q<PALU_F16, 1>(a, st);
 }
 
 }  // namespace palu

@@ -214,17 +214,19 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const DecodeArgs a) {
   extern __shared__ float smem[];
   float* av = smem;             // [r_v]
   float* wgt = av + a.r_v;      // [S]
-  const int h = blockIdx.x, b = blockIdx.y;
+  // virtual sequence vb = b·qn + j: query j of sequence b (qn = 1: one query per sequence)
+  const int h = blockIdx.x, vb = blockIdx.y;
+  const int b = vb / a.qn, jq = vb % a.qn;
   const int tid = threadIdx.x;
   const int g = h / a.gs, jh = h % a.gs;
-  const float* part = a.part + ((size_t)b * a.H + h) * a.S * (a.r_v + 2);
+  const float* part = a.part + ((size_t)vb * a.H + h) * a.S * (a.r_v + 2);
 
   float M = -INFINITY;
   for (int s = 0; s < a.S; ++s) M = fmaxf(M, part[(size_t)s * (a.r_v + 2)]);
-  TA* out = reinterpret_cast<TA*>(a.out) + (size_t)b * a.o_bstride + (size_t)h * a.d_h;
+  TA* out = reinterpret_cast<TA*>(a.out) + (size_t)b * a.o_bstride + ((size_t)jq * a.H + h) * a.d_h;
   if (M == -INFINITY) {
     for (int d = tid; d < a.d_h; d += kThreads) out[d] = Dt<ACT>::from_f(0.f);
-    if (tid == 0 && a.lse != nullptr) a.lse[(size_t)b * a.lse_bstride + h] = -INFINITY;
+    if (tid == 0 && a.lse != nullptr) a.lse[(size_t)b * a.lse_bstride + (size_t)jq * a.H + h] = -INFINITY;
     return;
   }
   float L = 0.f;
@@ -251,7 +253,7 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const DecodeArgs a) {
     for (int r = 0; r < a.r_v; ++r) o = fmaf(av[r], Dt<ACT>::to_f(Bv[(size_t)r * a.W + d]), o);
     out[d] = Dt<ACT>::from_f(o);
   }
-  if (tid == 0 && a.lse != nullptr) a.lse[(size_t)b * a.lse_bstride + h] = M + logf(L);
+  if (tid == 0 && a.lse != nullptr) a.lse[(size_t)b * a.lse_bstride + (size_t)jq * a.H + h] = M + logf(L);
 }
 
 template <int ACT, int LAT>
@@ -281,7 +283,7 @@ cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t st) {
 
 cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t st) {
   const size_t smem = sizeof(float) * (a.r_v + a.S);
-  dim3 grid(a.H, a.batch);
+  dim3 grid(a.H, a.batch * a.qn);
   if (a.act == PALU_F32) combine_kernel<PALU_F32><<<grid, kThreads, smem, st>>>(a);
   else if (a.act == PALU_F16) combine_kernel<PALU_F16><<<grid, kThreads, smem, st>>>(a);
   else if (a.act == PALU_BF16) combine_kernel<PALU_BF16><<<grid, kThreads, smem, st>>>(a);

@@ -73,6 +73,26 @@ constexpr int kMaxQueries = PALU_MAX_QUERIES;
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
+// Queries of each sequence one launch serves: the fused kernel takes passes
+// of 4, 2 or 1 queries; the other kernels one query per launch.
+int pass_queries(int kind, int remaining) {
+  if (kind != 3) return 1;
+  const int m = palu::fused_queries_per_pass();
+  return remaining >= m ? m : remaining >= 2 ? 2 : 1;
+}
+
+// Workspace layout: status word, partials [vb][H][S][r_v + 2] for vb virtual
+// sequences (sequence × query slot of a pass), then (fused kernel) the folded
+// queries.  Returns the total; *fused_off receives the offset of the queries.
+size_t workspace_layout(const palu_config* c, int kind, int vb, int S, size_t* fused_off) {
+  const size_t part = (size_t)vb * c->num_heads * S * (c->rank_v + 2) * sizeof(float);
+  size_t total = kStatusBytes + align256(part);
+  if (fused_off) *fused_off = total;
+  if (kind == 3) total += align256(palu::fused_query_bytes(c, vb));
+  return total;
+}
+
+
 int auto_splits(const palu_config* c, int batch, int max_pages, int kind) {
   const int sms = 148;
   const long long groups = (long long)batch * (c->num_heads / c->group_size);
@@ -96,6 +116,11 @@ int kernel_kind(const palu_config* c) {
   if (palu::fused_decode_supported(c)) return 3;
   if (palu::tc_decode_supported(c)) return 2;
   return 1;
+}
+
+// The split count a call runs (num_splits = 0: automatic).
+int run_S(const palu_config* c, int kind, int batch, int max_pages, int num_splits) {
+  return num_splits == 0 ? auto_splits(c, batch, max_pages, kind) : num_splits;
 }
 
 }  // namespace
@@ -217,14 +242,7 @@ palu_status palu_decode_num_splits(const palu_config* cfg, int batch, int max_pa
 
 palu_status palu_decode_workspace_size(const palu_config* cfg, int batch, int max_pages,
                                        int num_splits, size_t* bytes) {
-  palu_status s = check_config(cfg);
-  if (s != PALU_OK) return s;
-  if (bytes == nullptr || batch < 0 || max_pages <= 0 || num_splits < 0) return PALU_ERR_INVALID_ARG;
-  const int S = num_splits == 0 ? auto_splits(cfg, batch, max_pages, kernel_kind(cfg)) : num_splits;
-  const size_t part = (size_t)batch * cfg->num_heads * S * (cfg->rank_v + 2) * sizeof(float);
-  *bytes = kStatusBytes + align256(part);
-  if (kernel_kind(cfg) == 3) *bytes += align256(palu::fused_query_bytes(cfg, batch));
-  return PALU_OK;
+  return palu_decode_multi_workspace_size(cfg, batch, 1, max_pages, num_splits, bytes);
 }
 
 }  // extern "C"
@@ -246,10 +264,10 @@ palu_status decode_steps(const palu_config* cfg, int batch, int Q, const void* q
   if (batch < 0 || max_pages <= 0 || num_pages < 0 || num_splits < 0 || Q < 1 || Q > kMaxQueries)
     return PALU_ERR_INVALID_ARG;
   const int kind = kernel_kind(cfg);
-  const int S = num_splits == 0 ? auto_splits(cfg, batch, max_pages, kind) : num_splits;
+  const int S = run_S(cfg, kind, batch, max_pages, num_splits);
   if (S > max_pages) return PALU_ERR_INVALID_ARG;
-  size_t need = 0;
-  palu_decode_workspace_size(cfg, batch, max_pages, S, &need);
+  size_t fused_off = 0;
+  const size_t need = workspace_layout(cfg, kind, batch * pass_queries(kind, Q), S, &fused_off);
   if (workspace == nullptr || workspace_bytes < need) return PALU_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return PALU_ERR_ALIGNMENT;
   if (batch == 0) return PALU_OK;
@@ -293,8 +311,7 @@ palu_status decode_steps(const palu_config* cfg, int batch, int Q, const void* q
   a.lse = lse;
   a.status = workspace;
   a.part = reinterpret_cast<float*>(static_cast<char*>(workspace) + kStatusBytes);
-  a.fused_q = static_cast<char*>(workspace) + kStatusBytes +
-              align256((size_t)batch * cfg->num_heads * S * (cfg->rank_v + 2) * sizeof(float));
+  a.fused_q = static_cast<char*>(workspace) + fused_off;
   a.k_row = palu::latent_row_bytes(a.lat, a.r_k);
   a.v_row = palu::latent_row_bytes(a.lat, a.r_v);
   a.ks_row = palu::scale_row_bytes(a.lat, a.r_k);
@@ -311,7 +328,8 @@ palu_status decode_steps(const palu_config* cfg, int batch, int Q, const void* q
   a.causal = Q > 1;
 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  for (int j = 0; j < Q; ++j) {
+  for (int j = 0; j < Q; j += a.qn) {
+    a.qn = pass_queries(kind, Q - j);   // queries j .. j + qn - 1 of every sequence
     a.q = static_cast<const char*>(q) + (size_t)j * qrow * elt;
     a.q_pos = q_pos + j;
     a.out = static_cast<char*>(out) + (size_t)j * qrow * elt;
@@ -344,8 +362,15 @@ palu_status palu_decode_attn(const palu_config* cfg, int batch, const void* q, c
 
 palu_status palu_decode_multi_workspace_size(const palu_config* cfg, int batch, int num_queries, int max_pages,
                                              int num_splits, size_t* bytes) {
-  if (num_queries < 1 || num_queries > kMaxQueries) return PALU_ERR_INVALID_ARG;
-  return palu_decode_workspace_size(cfg, batch, max_pages, num_splits, bytes);
+  palu_status s = check_config(cfg);
+  if (s != PALU_OK) return s;
+  if (bytes == nullptr || batch < 0 || max_pages <= 0 || num_splits < 0 || num_queries < 1 ||
+      num_queries > kMaxQueries)
+    return PALU_ERR_INVALID_ARG;
+  const int kind = kernel_kind(cfg);
+  const int S = run_S(cfg, kind, batch, max_pages, num_splits);
+  *bytes = workspace_layout(cfg, kind, batch * pass_queries(kind, num_queries), S, nullptr);
+  return PALU_OK;
 }
 
 palu_status palu_decode_attn_multi(const palu_config* cfg, int batch, int num_queries, const void* q,

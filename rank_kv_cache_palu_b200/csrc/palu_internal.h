@@ -27,6 +27,8 @@ struct DecodeArgs {
   long long q_bstride, o_bstride;
   int qpos_bstride, lse_bstride;
   int causal;          // 1: a token counts only if its position <= the query's position
+  int qn;              // queries of each sequence this launch serves (the fused kernel takes
+                       // several per pass; their partials sit at virtual sequence b·qn + j)
   const void* zk;
   const void* zv;
   const void* zks;

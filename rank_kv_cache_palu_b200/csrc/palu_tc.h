@@ -18,6 +18,9 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st);
 // folded queries after the split partials.
 bool fused_decode_supported(const palu_config* c);
 size_t fused_query_bytes(const palu_config* c, int batch);
+// Queries of one sequence the fused kernel serves in one pass over the cache
+// (a pass takes 1, 2 or this many; DecodeArgs::qn).
+int fused_queries_per_pass();
 cudaError_t launch_decode_fused(const DecodeArgs& a, cudaStream_t st);
 
 // Compress: shapes the tensor-core GEMM takes, and the scratch it needs.

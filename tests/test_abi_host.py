@@ -158,3 +158,16 @@ def test_fused_path_selected_without_rope():
     assert P.palu_decode_kernel_kind(cfg()) == 2
     S = P.palu_decode_num_splits(c, 16, 128)
     assert P.palu_decode_workspace_size(c, 16, 128, S) >= 256 + 16 * 32 * S * 130 * 4 + 16 * 8 * 8 * 256 * 2
+
+
+def test_multi_query_workspace():
+    # fused path: up to four queries share a pass, so their partials and folded
+    # queries sit side by side; other paths run one query per launch
+    c = cfg(rope_base=0.0)
+    one = P.palu_decode_workspace_size(c, 16, 128, 4)
+    assert P.palu_decode_multi_workspace_size(c, 16, 1, 128, 4) == one
+    assert P.palu_decode_multi_workspace_size(c, 16, 8, 128, 4) > 3 * one
+    r = cfg()
+    assert P.palu_decode_multi_workspace_size(r, 16, 8, 128, 4) == P.palu_decode_workspace_size(r, 16, 128, 4)
+    with pytest.raises(P.PaluError):
+        P.palu_decode_multi_workspace_size(c, 16, P.MAX_QUERIES + 1, 128, 4)

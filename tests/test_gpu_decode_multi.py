@@ -72,10 +72,18 @@ def test_multi_tensor_core_rope(nq):
     check_multi(case, nq, num_splits=3)
 
 
-def test_multi_fused_no_rope():
+@pytest.mark.parametrize("nq", [2, 3, 5, 8])
+def test_multi_fused_no_rope(nq):
+    # the fused kernel serves 4, 2 or 1 queries per pass over the cache
     case = make_decode_case(bf16_7b(rope_base=0.0), [300, 130, 1000, 5])
     assert P.palu_decode_kernel_kind(case.cfg) == 3
-    check_multi(case, 8)
+    check_multi(case, nq)
+    check_multi(case, nq, num_splits=3)
+
+
+def test_multi_fused_rank_v_256_explicit_positions():
+    w = dataclasses.replace(bf16_7b(rope_base=0.0), rank_v=256, act_dtype="f16", latent_dtype="f16")
+    check_multi(make_decode_case(w, [700, 129], explicit_positions=True), 4)
 
 
 def test_multi_int4():

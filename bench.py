@@ -47,6 +47,9 @@ def parse_args():
     ap.add_argument("--num-splits", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU oracle sample budget")
+    ap.add_argument("--queries", type=int, default=1,
+                    help="query tokens per sequence per step (multi-token decode: appended together, "
+                         "each attends causally; palu_decode_attn_multi)")
     ap.add_argument("--prefill", type=int, default=None,
                     help="also time palu_compress_append of this many prompt tokens (default: 8192 for "
                          "the batch-32 prefill + decode workload, else off)")
@@ -274,8 +277,9 @@ def run_ours(args):
                         w.rope_base, w.act_dtype, w.latent_dtype)
     b, T0, G, W = w.batch, w.context, w.groups, w.width
     Pz = w.page_size
+    Q = args.queries
     steps_total = 2 * (args.warmup + args.steps) + 2
-    max_tokens = T0 + steps_total
+    max_tokens = T0 + steps_total * Q
     max_pages = (max_tokens + Pz - 1) // Pz
     num_pages = b * max_pages
     gen = torch.Generator(device=dev)
@@ -306,30 +310,42 @@ def run_ours(args):
     B_k = (torch.randn((G, w.rank_k, W), device=dev, generator=gen) / math.sqrt(w.rank_k)).to(act)
     B_v = (torch.randn((G, w.rank_v, W), device=dev, generator=gen) / math.sqrt(w.rank_v)).to(act)
     ring = 4
-    xs = [torch.randn((b, d_model), device=dev, generator=gen).to(act) for _ in range(ring)]
-    qs = [torch.randn((b, w.num_heads, w.head_dim), device=dev, generator=gen).to(act) for _ in range(ring)]
+    xs = [torch.randn((b * Q, d_model), device=dev, generator=gen).to(act) for _ in range(ring)]
+    qshape = (b, w.num_heads, w.head_dim) if Q == 1 else (b, Q, w.num_heads, w.head_dim)
+    qs = [torch.randn(qshape, device=dev, generator=gen).to(act) for _ in range(ring)]
 
-    # per-step metadata, all on the device before timing
+    # per-step metadata, all on the device before timing: the step appends Q
+    # tokens per sequence at positions base .. base + Q - 1, then queries them
     def meta(step):
-        pos = T0 + step
-        slots = np.array([pt_host[i, pos // Pz] * Pz + pos % Pz for i in range(b)], np.int32)
-        return (torch.from_numpy(slots).to(dev), torch.full((b,), pos, dtype=torch.int32, device=dev),
-                torch.full((b,), pos + 1, dtype=torch.int32, device=dev))
+        base = T0 + step * Q
+        slots = np.array([pt_host[i, (base + j) // Pz] * Pz + (base + j) % Pz for i in range(b) for j in range(Q)],
+                         np.int32)
+        qpos = np.array([[base + j for j in range(Q)] for _ in range(b)], np.int32)
+        return (torch.from_numpy(slots).to(dev), torch.from_numpy(qpos.reshape(b) if Q == 1 else qpos).to(dev),
+                torch.full((b,), base + Q, dtype=torch.int32, device=dev))
     metas = [meta(s) for s in range(steps_total)]
 
+    def step_units(s):
+        base = T0 + s * Q
+        return b * w.num_heads * sum(base + j + 1 for j in range(Q))
+
     S = args.num_splits or P.palu_decode_num_splits(cfg, b, max_pages)
-    ws_d = torch.zeros(P.palu_decode_workspace_size(cfg, b, max_pages, S), dtype=torch.uint8, device=dev)
-    ws_c = torch.zeros(P.palu_compress_workspace_size(cfg, b, d_model), dtype=torch.uint8, device=dev)
-    out = torch.empty((b, w.num_heads, w.head_dim), dtype=act, device=dev)
+    ws_d = torch.zeros(P.palu_decode_multi_workspace_size(cfg, b, Q, max_pages, S), dtype=torch.uint8,
+                       device=dev)
+    ws_c = torch.zeros(P.palu_compress_workspace_size(cfg, b * Q, d_model), dtype=torch.uint8, device=dev)
+    out = torch.empty(qshape, dtype=act, device=dev)
     stream = torch.cuda.current_stream(dev)
+
+    def decode(q, qpos, lens):
+        fn = P.palu_decode_attn if Q == 1 else P.palu_decode_attn_multi
+        fn(cfg, q, qpos, cache.zk, cache.zv, cache.zks, cache.zvs, None, page_table, lens, num_pages, B_k, B_v,
+           out, None, ws_d, S, stream)
 
     def step(s, x=None, q=None):
         slots, qpos, lens = metas[s]
         P.palu_compress_append(cfg, xs[s % ring] if x is None else x, A_k, A_v, slots, None,
                                cache.zk, cache.zv, cache.zks, cache.zvs, None, num_pages, ws_c, stream)
-        P.palu_decode_attn(cfg, qs[s % ring] if q is None else q, qpos, cache.zk, cache.zv, cache.zks,
-                           cache.zvs, None, page_table, lens, num_pages, B_k, B_v, out, None, ws_d, S,
-                           stream)
+        decode(qs[s % ring] if q is None else q, qpos, lens)
 
     # ---- device-resident timing
     s_idx = 0
@@ -352,8 +368,7 @@ def run_ours(args):
             P.palu_compress_append(cfg, xs[s_idx % ring], A_k, A_v, slots, None, cache.zk, cache.zv,
                                    cache.zks, cache.zvs, None, num_pages, ws_c, stream)
             ev[k][1].record(stream)
-            P.palu_decode_attn(cfg, qs[s_idx % ring], qpos, cache.zk, cache.zv, cache.zks, cache.zvs,
-                               None, page_table, lens, num_pages, B_k, B_v, out, None, ws_d, S, stream)
+            decode(qs[s_idx % ring], qpos, lens)
             ev[k][2].record(stream)
             s_idx += 1
         end.record(stream)
@@ -367,8 +382,7 @@ def run_ours(args):
     el_ms = D.max_over_ranks(start.elapsed_time(end), dev)
     dec_ms = [e[1].elapsed_time(e[2]) for e in ev]
     cmp_ms = [e[0].elapsed_time(e[1]) for e in ev]
-    lens_timed = [[T0 + s + 1] * b for s in range(first_step, first_step + args.steps)]
-    units = sum(sum(l) for l in lens_timed) * w.num_heads
+    units = sum(step_units(s) for s in range(first_step, first_step + args.steps))
     value = D.sum_over_ranks(units, dev) / (el_ms / 1e3)
 
     # ---- end to end through the public API: pinned host inputs -> H2D -> step -> D2H
@@ -389,8 +403,7 @@ def run_ours(args):
             dst.copy_(src, non_blocking=True)
         P.palu_compress_append(cfg, x_d, A_k, A_v, m_d[0], None, cache.zk, cache.zv, cache.zks,
                                cache.zvs, None, num_pages, ws_c, stream)
-        P.palu_decode_attn(cfg, q_d, m_d[1], cache.zk, cache.zv, cache.zks, cache.zvs, None, page_table,
-                           m_d[2], num_pages, B_k, B_v, out, None, ws_d, S, stream)
+        decode(q_d, m_d[1], m_d[2])
         outh.copy_(out, non_blocking=True)
 
     for _ in range(min(args.warmup, 3)):
@@ -403,7 +416,7 @@ def run_ours(args):
     e0.record(stream)
     for _ in range(args.steps):
         e2e_step(s_idx)
-        e2e_units += (T0 + s_idx + 1) * b * w.num_heads
+        e2e_units += step_units(s_idx)
         s_idx += 1
     e1.record(stream)
     torch.cuda.synchronize(dev)
@@ -446,8 +459,10 @@ def run_ours(args):
 
     # ---- roofline of the dominant kernel (the decode step: split + combine)
     peaks = measured_peaks()
-    mean_lens = [T0 + (first_step + args.steps / 2) + 0.5] * b
-    dbytes, dflops = step_work(w, mean_lens)
+    # the step's algorithmic work: the cache read once, every query's flops
+    mean_T = T0 + (first_step + args.steps / 2) * Q + Q
+    dbytes, dflops = step_work(w, [mean_T] * b)
+    dflops *= Q
     dec_avg_s = statistics.mean(dec_ms) / 1e3
     gbs = dbytes / dec_avg_s / 1e9
     tfs = dflops / dec_avg_s / 1e12
@@ -480,7 +495,7 @@ def run_ours(args):
                    "context_at_first_timed_step": T0 + first_step + 1, "heads": w.num_heads,
                    "head_dim": w.head_dim, "group_size": w.group_size, "rank_k": w.rank_k,
                    "rank_v": w.rank_v, "latent_dtype": w.latent_dtype, "page_size": Pz,
-                   "num_splits": S, "decode_kernel_kind": kind,
+                   "num_splits": S, "decode_kernel_kind": kind, "queries_per_step": Q,
                    "l2": "inputs larger than L2 (latent cache %.2f GB vs 126 MB L2)" %
                          ((cache.zk.numel() + cache.zv.numel()) / 1e9),
                    "parallelism": f"dp{world} replicas (independent sequences per GPU)"},

@@ -57,6 +57,7 @@ __all__ = [
     "split_partials",
     "lse_combine",
     "decode_attention_multi",
+    "decode_attention_ranked",
     "quantize_int4",
     "dequantize_int4",
     "cache_bytes_per_token",
@@ -213,6 +214,30 @@ def decode_attention_multi(q, q_pos, z_k, z_v, pos, B_k, B_v, group_size, rope_b
         zk_j, zv_j = z_k[:, keep], z_v[:, keep]
         out[j], lse[j] = decode_attention(q[j], int(q_pos[j]), zk_j, zv_j, pos[keep], B_k, B_v,
                                           group_size, rope_base)
+    return out, lse
+
+
+def decode_attention_ranked(q, q_pos, z_k, z_v, pos, B_k, B_v, group_size, rope_base):
+    """The multi-query step of a layer whose head groups have their own ranks.
+
+    The rank is chosen by a search, per layer and per group of heads, rather
+    than cut to one value everywhere ([EXPL] §为什么还能保精度; §怎么落地, 路线 B;
+    §风险、边界和别踩的坑, 风险 1).  z_k, z_v, B_k, B_v are length-G sequences:
+    z_k[g] [T, r_k,g], z_v[g] [T, r_v,g], B_k[g] [r_k,g, G_w], B_v[g] [r_v,g, G_w].
+    In the group-head decomposition ([ABS2]) the heads of group g read only
+    group g's latents and B, so each group is the step above on its own.
+    q: [Q, H, d_h]; q_pos: [Q].  Returns (out [Q, H, d_h], lse [Q, H]).
+    """
+    q = np.asarray(q)
+    Q, H, d_h = q.shape
+    G = H // group_size
+    out = np.zeros((Q, H, d_h))
+    lse = np.full((Q, H), -math.inf)
+    for g in range(G):
+        heads = slice(g * group_size, (g + 1) * group_size)
+        out[:, heads], lse[:, heads] = decode_attention_multi(
+            q[:, heads], q_pos, np.asarray(z_k[g])[None], np.asarray(z_v[g])[None], pos,
+            np.asarray(B_k[g])[None], np.asarray(B_v[g])[None], group_size, rope_base)
     return out, lse
 
 

@@ -279,6 +279,59 @@ def test_multi_query_single_query_is_the_decode_step():
     np.testing.assert_allclose(lse[0], ref_lse, rtol=0, atol=1e-12)
 
 
+def make_ranked(seed, ranks_k, ranks_v, H=8, d_h=8, g=2, T=23, base=10000.0):
+    r = rng(seed)
+    W = g * d_h
+    return dict(
+        z_k=[r.standard_normal((T, rk)) for rk in ranks_k],
+        z_v=[r.standard_normal((T, rv)) for rv in ranks_v],
+        B_k=[r.standard_normal((rk, W)) / math.sqrt(rk) for rk in ranks_k],
+        B_v=[r.standard_normal((rv, W)) / math.sqrt(rv) for rv in ranks_v],
+        pos=np.arange(T) * 2 + 1, group_size=g, rope_base=base,
+    ), r.standard_normal((3, H, d_h)), np.array([2 * T - 1, 17, 6])
+
+
+def test_ranked_equals_zero_padded_uniform():
+    # z·B is unchanged when z gains zero columns and B gains rows (any rows):
+    # padding every group to the largest rank gives the uniform step
+    ranks_k, ranks_v = [3, 7, 1, 5], [2, 6, 4, 4]
+    c, q, q_pos = make_ranked(41, ranks_k, ranks_v)
+    out, lse = O.decode_attention_ranked(q, q_pos, **c)
+    T = len(c["pos"])
+    rk, rv = max(ranks_k), max(ranks_v)
+    fill = rng(42)
+    zk = np.zeros((4, T, rk))
+    zv = np.zeros((4, T, rv))
+    Bk = fill.standard_normal((4, rk, 16))          # the padded rows are junk on purpose
+    Bv = fill.standard_normal((4, rv, 16))
+    for gi in range(4):
+        zk[gi, :, : ranks_k[gi]] = c["z_k"][gi]
+        zv[gi, :, : ranks_v[gi]] = c["z_v"][gi]
+        Bk[gi, : ranks_k[gi]] = c["B_k"][gi]
+        Bv[gi, : ranks_v[gi]] = c["B_v"][gi]
+    ref, ref_lse = O.decode_attention_multi(q, q_pos, zk, zv, c["pos"], Bk, Bv, 2, 10000.0)
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, ref_lse, rtol=0, atol=1e-12)
+
+
+def test_ranked_brute_force_and_group_independence():
+    ranks_k, ranks_v = [3, 1], [2, 4]
+    c, q, q_pos = make_ranked(43, ranks_k, ranks_v, H=4, d_h=4, g=2, T=6)
+    out, _ = O.decode_attention_ranked(q, q_pos, **c)
+    # brute force, one group at a time, each with its own rank
+    for gi in range(2):
+        cg = dict(q=None, q_pos=None, z_k=np.asarray(c["z_k"][gi])[None], z_v=np.asarray(c["z_v"][gi])[None],
+                  pos=c["pos"], B_k=np.asarray(c["B_k"][gi])[None], B_v=np.asarray(c["B_v"][gi])[None],
+                  group_size=2, rope_base=10000.0)
+        bf = brute_force_multi(cg, q[:, 2 * gi: 2 * gi + 2], q_pos)
+        np.testing.assert_allclose(out[:, 2 * gi: 2 * gi + 2], bf, rtol=0, atol=1e-12)
+    # changing one group's latents leaves the other group's heads untouched
+    c2 = dict(c, z_k=[c["z_k"][0] + 5.0, c["z_k"][1]])
+    out2, _ = O.decode_attention_ranked(q, q_pos, **c2)
+    np.testing.assert_array_equal(out2[:, 2:], out[:, 2:])
+    assert np.abs(out2[:, :2] - out[:, :2]).max() > 1e-6
+
+
 def test_latent_formulation_matches_materialised():
     c = make_seq(14, T=53)
     a, la = O.decode_attention(**c)

@@ -19,8 +19,8 @@
  *     G = num_heads / group_size groups, group width W = group_size·head_dim.
  *   - All tensors are dense, row-major, in DEVICE memory owned by the caller.
  *     The library allocates nothing, keeps no per-call state, and never frees
- *     what it is given.  It caches CUDA tensor-map descriptors keyed by pointer
- *     and shape; that cache is thread-safe.
+ *     what it is given.  Tensor-map descriptors are encoded on the host for
+ *     each launch and passed by value; no state survives a call.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
  *     default stream).  Argument checks are synchronous and return a status
  *     before anything is launched.  Faults found by the kernels themselves
@@ -80,7 +80,8 @@ typedef enum palu_dtype {
 typedef struct palu_config {
   int32_t num_heads;    /* H query heads (= KV heads) */
   int32_t head_dim;     /* d_h, even */
-  int32_t group_size;   /* g heads share one latent (medium-grained decomposition) */
+  int32_t group_size;   /* g heads share one latent (medium-grained decomposition);
+                           num_heads / group_size <= 64 groups */
   int32_t rank_k;       /* r_k latent width per group for keys */
   int32_t rank_v;       /* r_v latent width per group for values */
   int32_t page_size;    /* tokens per cache page */
@@ -197,6 +198,59 @@ palu_status palu_decode_attn_multi(const palu_config* cfg, int batch, int num_qu
                                    void* workspace, size_t workspace_bytes, int num_splits,
                                    palu_stream_t stream);
 
+/* Layers whose head groups carry different ranks: the output of Palu's rank
+ * search.  "PALU 论文低秩投影分解" §为什么还能保精度 (the rank is searched rather
+ * than cut uniformly everywhere), §怎么落地 路线 B (ranks found offline per layer
+ * and per group of heads, then served from the compressed cache) and
+ * §风险、边界和别踩的坑 风险 1 (one rank for every layer loses accuracy or gain).
+ * A per-layer rank needs nothing new: each layer has its own config.  These
+ * calls take a rank pair per group instead of cfg->rank_k / cfg->rank_v:
+ *   ranks_k, ranks_v  [G] int32, HOST memory, read during the call only.  Each
+ *            pair must be valid in a config of its own (the rank rules of
+ *            palu_config).  NULL for both = every group uses cfg's ranks, and
+ *            the call is exactly its uniform counterpart.
+ * Layout, with r_k,g the key rank of group g (V and the int4 scale pools the
+ * same way, with their own row sizes):
+ *   K pool  page p holds every group's block back to back: group g's block of
+ *           page_size rows of row_k,g bytes starts at
+ *           p·k_page_bytes + Σ_{g'<g} page_size·row_k,g'
+ *           (palu_cache_strides_ranked gives k_page_bytes and those offsets);
+ *           inside the block the swizzled layout above applies unchanged.
+ *   A_k     [d_model][Σ_g r_k,g]: group g's columns start at Σ_{g'<g} r_k,g'
+ *   B_k     [Σ_g r_k,g][W]: group g's rows start at Σ_{g'<g} r_k,g'
+ * With equal ranks this is byte for byte the uniform layout.  Groups that share
+ * a rank pair are served by one launch of each kernel; the calls run the rank
+ * classes one after another on `stream`.  Every other argument, rule and
+ * status is that of the uniform call named in each comment. */
+/* as palu_cache_strides; k_group_offsets / v_group_offsets [G] (optional)
+ * receive the byte offset of each group's block within a K / V page.  In an
+ * int4 scale page, group g's block starts at Σ_{g'<g} page_size·srow_g'. */
+palu_status palu_cache_strides_ranked(const palu_config* cfg, const int32_t* ranks_k, const int32_t* ranks_v,
+                                      size_t* k_page_bytes, size_t* v_page_bytes, size_t* k_scale_page_bytes,
+                                      size_t* v_scale_page_bytes, size_t* k_group_offsets,
+                                      size_t* v_group_offsets);
+/* as palu_compress_workspace_size / palu_compress_append */
+palu_status palu_compress_ranked_workspace_size(const palu_config* cfg, const int32_t* ranks_k,
+                                                const int32_t* ranks_v, int n_tokens, int d_model, size_t* bytes);
+palu_status palu_compress_append_ranked(const palu_config* cfg, const int32_t* ranks_k, const int32_t* ranks_v,
+                                        int n_tokens, int d_model, const void* x, const void* A_k, const void* A_v,
+                                        const int32_t* slot_mapping, const int32_t* positions, void* zk_pool,
+                                        void* zv_pool, void* zk_scales, void* zv_scales, int32_t* pos_pool,
+                                        int num_pages, void* workspace, size_t workspace_bytes,
+                                        palu_stream_t stream);
+/* as palu_decode_multi_workspace_size / palu_decode_attn_multi (num_queries = 1
+ * is palu_decode_attn) */
+palu_status palu_decode_ranked_workspace_size(const palu_config* cfg, const int32_t* ranks_k,
+                                              const int32_t* ranks_v, int batch, int num_queries, int max_pages,
+                                              int num_splits, size_t* bytes);
+palu_status palu_decode_attn_ranked(const palu_config* cfg, const int32_t* ranks_k, const int32_t* ranks_v,
+                                    int batch, int num_queries, const void* q, const int32_t* q_pos,
+                                    const void* zk_pool, const void* zv_pool, const void* zk_scales,
+                                    const void* zv_scales, const int32_t* pos_pool, const int32_t* page_table,
+                                    int max_pages, const int32_t* seq_lens, int num_pages, const void* B_k,
+                                    const void* B_v, void* out, float* lse, void* workspace,
+                                    size_t workspace_bytes, int num_splits, palu_stream_t stream);
+
 /* Allocation-free decode step (the paper has no counterpart: this is a
  * deployment convenience of this library).
  * Some callers cannot call cudaMalloc at all: plug-ins whose host framework
@@ -244,7 +298,9 @@ const char* palu_status_string(palu_status status);
 const char* palu_last_cuda_error(void);
 
 /* Which kernel family a decode call with this config would launch:
- * 0 = none (unsupported), 1 = CUDA-core kernels, 2 = tcgen05/TMA kernels. */
+ * 0 = none (unsupported), 1 = CUDA-core kernels, 2 = tcgen05/TMA kernels,
+ * 3 = the fused no-RoPE kernel (query folded through B_k, scores straight
+ * from z_k). */
 int palu_decode_kernel_kind(const palu_config* cfg);
 
 /* Phase tracing of the tensor-core decode kernel, for performance analysis.

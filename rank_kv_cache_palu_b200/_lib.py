@@ -55,6 +55,19 @@ SIGNATURES = {
                                          c_void_p, c_void_p, c_void_p, c_int, c_void_p, c_int,
                                          c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_void_p,
                                          _P(c_int32)]),
+    "palu_cache_strides_ranked": (c_int, [_CFG, _P(c_int32), _P(c_int32), _P(c_size_t), _P(c_size_t),
+                                          _P(c_size_t), _P(c_size_t), _P(c_size_t), _P(c_size_t)]),
+    "palu_compress_ranked_workspace_size": (c_int, [_CFG, _P(c_int32), _P(c_int32), c_int, c_int,
+                                                    _P(c_size_t)]),
+    "palu_compress_append_ranked": (c_int, [_CFG, _P(c_int32), _P(c_int32), c_int, c_int, c_void_p, c_void_p,
+                                            c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                            c_void_p, c_void_p, c_int, c_void_p, c_size_t, c_void_p]),
+    "palu_decode_ranked_workspace_size": (c_int, [_CFG, _P(c_int32), _P(c_int32), c_int, c_int, c_int, c_int,
+                                                  _P(c_size_t)]),
+    "palu_decode_attn_ranked": (c_int, [_CFG, _P(c_int32), _P(c_int32), c_int, c_int, c_void_p, c_void_p,
+                                        c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int,
+                                        c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                        c_size_t, c_int, c_void_p]),
     "palu_get_device_status": (c_int, [c_void_p, c_void_p, _P(c_int32)]),
     "palu_status_string": (ctypes.c_char_p, [c_int]),
     "palu_last_cuda_error": (ctypes.c_char_p, []),

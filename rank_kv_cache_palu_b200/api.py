@@ -159,6 +159,67 @@ def palu_decode_attn_multi(cfg: PaluConfig, q, q_pos, zk_pool, zv_pool, zk_scale
     _check(st, "palu_decode_attn_multi")
 
 
+def _ranks(r):
+    """Host int32 array of per-group ranks (None: the config's uniform ranks)."""
+    return None if r is None else (ctypes.c_int32 * len(r))(*[int(v) for v in r])
+
+
+def palu_cache_strides_ranked(cfg: PaluConfig, ranks_k, ranks_v):
+    """(k_page, v_page, k_scale_page, v_scale_page, k_group_offsets, v_group_offsets) in bytes."""
+    G = cfg.num_heads // cfg.group_size
+    out = [ctypes.c_size_t() for _ in range(4)]
+    ko, vo = (ctypes.c_size_t * G)(), (ctypes.c_size_t * G)()
+    _check(load().palu_cache_strides_ranked(ctypes.byref(cfg), _ranks(ranks_k), _ranks(ranks_v),
+                                            *[ctypes.byref(o) for o in out], ko, vo),
+           "palu_cache_strides_ranked")
+    return (*[o.value for o in out], list(ko), list(vo))
+
+
+def palu_compress_ranked_workspace_size(cfg: PaluConfig, ranks_k, ranks_v, n_tokens: int, d_model: int) -> int:
+    out = ctypes.c_size_t()
+    _check(load().palu_compress_ranked_workspace_size(ctypes.byref(cfg), _ranks(ranks_k), _ranks(ranks_v),
+                                                      n_tokens, d_model, ctypes.byref(out)),
+           "palu_compress_ranked_workspace_size")
+    return int(out.value)
+
+
+def palu_compress_append_ranked(cfg: PaluConfig, ranks_k, ranks_v, x, A_k, A_v, slot_mapping, positions,
+                                zk_pool, zv_pool, zk_scales, zv_scales, pos_pool, num_pages: int, workspace,
+                                stream=None):
+    """palu_compress_append for a layer with a rank pair per group (A columns stacked by group)."""
+    n, d_model = x.shape
+    st = load().palu_compress_append_ranked(
+        ctypes.byref(cfg), _ranks(ranks_k), _ranks(ranks_v), n, d_model, _ptr(x), _ptr(A_k), _ptr(A_v),
+        _ptr(slot_mapping), _ptr(positions), _ptr(zk_pool), _ptr(zv_pool), _ptr(zk_scales), _ptr(zv_scales),
+        _ptr(pos_pool), num_pages, _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream))
+    _check(st, "palu_compress_append_ranked")
+
+
+def palu_decode_ranked_workspace_size(cfg: PaluConfig, ranks_k, ranks_v, batch: int, num_queries: int,
+                                      max_pages: int, num_splits: int = 0) -> int:
+    out = ctypes.c_size_t()
+    _check(load().palu_decode_ranked_workspace_size(ctypes.byref(cfg), _ranks(ranks_k), _ranks(ranks_v), batch,
+                                                    num_queries, max_pages, num_splits, ctypes.byref(out)),
+           "palu_decode_ranked_workspace_size")
+    return int(out.value)
+
+
+def palu_decode_attn_ranked(cfg: PaluConfig, ranks_k, ranks_v, q, q_pos, zk_pool, zv_pool, zk_scales, zv_scales,
+                            pos_pool, page_table, seq_lens, num_pages: int, B_k, B_v, out, lse, workspace,
+                            num_splits: int = 0, stream=None):
+    """Decode step of a layer with a rank pair per group: q [batch][Q][H][d_h], q_pos [batch][Q]
+    (Q = 1 is the single-query step); B_k / B_v rows stacked by group."""
+    batch, nq = q.shape[0], q.shape[1]
+    max_pages = page_table.shape[1]
+    st = load().palu_decode_attn_ranked(
+        ctypes.byref(cfg), _ranks(ranks_k), _ranks(ranks_v), batch, nq, _ptr(q), _ptr(q_pos), _ptr(zk_pool),
+        _ptr(zv_pool), _ptr(zk_scales), _ptr(zv_scales), _ptr(pos_pool), _ptr(page_table), max_pages,
+        _ptr(seq_lens), num_pages, _ptr(B_k), _ptr(B_v), _ptr(out), _ptr(lse), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), num_splits, _stream(stream))
+    _check(st, "palu_decode_attn_ranked")
+
+
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
 

@@ -14,7 +14,7 @@ namespace {
 constexpr int kBM = 64, kBN = 64, kBK = 32, kThreads = 256;
 
 template <int ACT, int LAT>
-__global__ void __launch_bounds__(kThreads) compress_kernel(const CompressArgs a) {
+__global__ void __launch_bounds__(kThreads) compress_kernel(const __grid_constant__ CompressArgs a) {
   using TA = typename Dt<ACT>::T;
   __shared__ float xs[kBK][kBM + 1];
   __shared__ float as_[kBK][kBN + 1];
@@ -23,7 +23,9 @@ __global__ void __launch_bounds__(kThreads) compress_kernel(const CompressArgs a
 
   const bool is_v = blockIdx.z == 1;
   const int r = is_v ? a.r_v : a.r_k;
-  const int N = a.G * r;
+  const int N = a.gm.n * r;                 // output columns: entry gc / r, latent entry gc % r
+  const long long acols = is_v ? a.a_vcols : a.a_kcols;
+  const int* col0s = is_v ? a.gm.v_row0 : a.gm.k_row0;
   const int row0 = blockIdx.x * kBM, col0 = blockIdx.y * kBN;
   if (col0 >= N) return;
   const TA* X = reinterpret_cast<const TA*>(a.x);
@@ -40,7 +42,7 @@ __global__ void __launch_bounds__(kThreads) compress_kernel(const CompressArgs a
     for (int e = tid; e < kBK * kBN; e += kThreads) {
       const int k = e / kBN, c = e % kBN;
       const int gk = k0 + k, gc = col0 + c;
-      as_[k][c] = (gk < a.d_model && gc < N) ? Dt<ACT>::to_f(A[(size_t)gk * N + gc]) : 0.f;
+      as_[k][c] = (gk < a.d_model && gc < N) ? Dt<ACT>::to_f(A[(size_t)gk * acols + col0s[gc / r] + gc % r]) : 0.f;
     }
     __syncthreads();
 #pragma unroll 8
@@ -65,13 +67,12 @@ __global__ void __launch_bounds__(kThreads) compress_kernel(const CompressArgs a
   __syncthreads();
 
   const long long cap = (long long)a.num_pages * a.P;
-  uint8_t* pool = reinterpret_cast<uint8_t*>(is_v ? a.zv : a.zk);
-  const long long row_bytes = is_v ? a.v_row : a.k_row;
+  const long long page_bytes = is_v ? a.gm.v_page : a.gm.k_page;
 
   if constexpr (LAT == PALU_INT4) {
     // one thread per (token row, 32-entry block)
-    uint8_t* spool = reinterpret_cast<uint8_t*>(is_v ? a.zvs : a.zks);
     const long long srow = is_v ? a.vs_row : a.ks_row;
+    const long long spage = is_v ? a.gm.vs_page : a.gm.ks_page;
     if (tid < kBM * 2) {
       const int i = tid / 2, blk = tid % 2;
       const int gi = row0 + i, gc = col0 + blk * 32;
@@ -81,10 +82,10 @@ __global__ void __launch_bounds__(kThreads) compress_kernel(const CompressArgs a
           if (slot >= cap) {
             report(st, PALU_ERR_DEVICE_BOUNDS, 3000000 + gi);
           } else {
-            const int g = gc / r, j0 = gc % r;
-            const long long pgb = (long long)(slot / a.P) * a.G + g;   // (page, group) block
+            const int e = gc / r, j0 = gc % r;
             const int tok = slot % a.P;
-            const long long prow = pgb * a.P + tok;
+            uint8_t* pblk = const_cast<uint8_t*>(is_v ? a.gm.zv[e] : a.gm.zk[e]) + (long long)(slot / a.P) * page_bytes;
+            uint8_t* sblk = const_cast<uint8_t*>(is_v ? a.gm.zvs[e] : a.gm.zks[e]) + (long long)(slot / a.P) * spage;
             float amax = 0.f;
             for (int u = 0; u < 32; ++u) amax = fmaxf(amax, fabsf(ct[i][blk * 32 + u]));
             const __half s16 = __float2half_rn(__fdiv_rn(amax, 7.0f));
@@ -100,9 +101,9 @@ __global__ void __launch_bounds__(kThreads) compress_kernel(const CompressArgs a
               words[u / 8] |= (uint32_t)(code & 0xF) << (4 * (u % 8));
             }
             // 32 codes = one 16-byte unit of the swizzled page block
-            uint4* dst = reinterpret_cast<uint4*>(pool + pgb * a.P * row_bytes + swz_offset(tok, j0 / 2, a.P));
+            uint4* dst = reinterpret_cast<uint4*>(pblk + swz_offset(tok, j0 / 2, a.P));
             *dst = make_uint4(words[0], words[1], words[2], words[3]);
-            reinterpret_cast<__half*>(spool + prow * srow)[j0 / 32] = s16;
+            reinterpret_cast<__half*>(sblk + tok * srow)[j0 / 32] = s16;
           }
         }
       }
@@ -123,9 +124,9 @@ __global__ void __launch_bounds__(kThreads) compress_kernel(const CompressArgs a
       for (int v = 0; v < 4; ++v) {
         const int gc = col0 + tx * 4 + v;
         if (gc >= N) continue;
-        const int g = gc / r, j = gc % r;
-        const long long pgb = (long long)(slot / a.P) * a.G + g;   // (page, group) block
-        *reinterpret_cast<TL*>(pool + pgb * a.P * row_bytes + swz_offset(slot % a.P, (long long)j * sizeof(TL), a.P)) =
+        const int e = gc / r, j = gc % r;
+        uint8_t* blk = const_cast<uint8_t*>(is_v ? a.gm.zv[e] : a.gm.zk[e]) + (long long)(slot / a.P) * page_bytes;
+        *reinterpret_cast<TL*>(blk + swz_offset(slot % a.P, (long long)j * sizeof(TL), a.P)) =
             Dt<LAT>::from_f(ct[i][tx * 4 + v]);
       }
     }
@@ -143,7 +144,7 @@ __global__ void __launch_bounds__(kThreads) compress_kernel(const CompressArgs a
 
 template <int ACT, int LAT>
 cudaError_t launch_t(const CompressArgs& a, cudaStream_t st) {
-  const int ncol = a.G * (a.r_k > a.r_v ? a.r_k : a.r_v);
+  const int ncol = a.gm.n * (a.r_k > a.r_v ? a.r_k : a.r_v);
   dim3 grid((a.n + kBM - 1) / kBM, (ncol + kBN - 1) / kBN, 2);
   compress_kernel<ACT, LAT><<<grid, kThreads, 0, st>>>(a);
   count_launch();

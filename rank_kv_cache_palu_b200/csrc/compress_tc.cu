@@ -75,14 +75,21 @@ struct TcArgs {
   float* partials;
 };
 
-// Write one latent column `j` (of group g) for token row i of the tile.
+// Column of A holding column lc of this launch (group entry lc / r, latent
+// entry lc % r).  Past the last entry it continues from the last one, so a TMA
+// box that runs off the end still has a valid start (those columns are
+// computed and dropped).
+__device__ __forceinline__ int a_column(const GroupMap& gm, const int* row0, int r, int lc) {
+  int e = lc / r;
+  if (e >= gm.n) e = gm.n - 1;
+  return row0[e] + (lc - e * r);
+}
+
+// Write latent entry j of one token into its (page, group) block.
 template <int LAT>
-__device__ __forceinline__ void store_latent(const CompressArgs& a, uint8_t* pool, long long row_bytes, int g,
-                                             int j, int slot, float v) {
+__device__ __forceinline__ void store_latent(const CompressArgs& a, uint8_t* blk, int j, int slot, float v) {
   using TL = typename Dt<LAT>::T;
-  const long long pgb = (long long)(slot / a.P) * a.G + g;
-  *reinterpret_cast<TL*>(pool + pgb * a.P * row_bytes + swz_offset(slot % a.P, (long long)j * sizeof(TL), a.P)) =
-      Dt<LAT>::from_f(v);
+  *reinterpret_cast<TL*>(blk + swz_offset(slot % a.P, (long long)j * sizeof(TL), a.P)) = Dt<LAT>::from_f(v);
 }
 
 template <int ACT, int LAT>
@@ -113,7 +120,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int ctile = is_v ? blockIdx.x - p.tk : blockIdx.x;
   const int c0 = ctile * kM;
   const int r = is_v ? a.r_v : a.r_k;
-  const int ncols = a.G * r;
+  const int ncols = a.gm.n * r;
   const int t0 = blockIdx.y * p.NT;
   const int kst = a.d_model / kKStage;
   const int split = blockIdx.z;
@@ -149,8 +156,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(empty(s), ph ^ 1, abort_flag, st, 50)) break;
         mbar_expect_tx(full(s), (uint32_t)stage_bytes);
         const uint32_t dst = base + (uint32_t)s * stage_bytes;
-        tma_load_2d(dst, tm_a, c0, kb * kKStage, full(s));
-        tma_load_2d(dst + kABytes / 2, tm_a, c0 + 64, kb * kKStage, full(s));
+        const int* row0 = is_v ? a.gm.v_row0 : a.gm.k_row0;
+        tma_load_2d(dst, tm_a, a_column(a.gm, row0, r, c0), kb * kKStage, full(s));
+        tma_load_2d(dst + kABytes / 2, tm_a, a_column(a.gm, row0, r, c0 + 64), kb * kKStage, full(s));
         tma_load_2d(dst + kABytes, &tm_x, kb * kKStage, t0, full(s));
         if (++s == p.stages) { s = 0; ph ^= 1; }
       }
@@ -221,11 +229,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (finalize) __threadfence();
     }
     if (ok && finalize) {
-      uint8_t* pool = reinterpret_cast<uint8_t*>(is_v ? a.zv : a.zk);
-      const long long row_bytes = is_v ? a.v_row : a.k_row;
       const long long cap = (long long)a.num_pages * a.P;
-      const int g = gc / r, j = gc % r;
       const bool col_ok = gc < ncols;
+      const int e = col_ok ? gc / r : 0, j = gc % r;   // group entry and latent entry of this column
+      uint8_t* pool = const_cast<uint8_t*>(is_v ? a.gm.zv[e] : a.gm.zk[e]);
+      const long long page_bytes = is_v ? a.gm.v_page : a.gm.k_page;
       const int ntok = min(p.NT, a.n - t0);
       for (int j0 = 0; j0 < ntok; j0 += 16) {
         float v[16];
@@ -267,19 +275,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             int code = 0;
             if (s != 0.f) code = (int)fminf(fmaxf(rintf(__fdiv_rn(v[u], s)), -7.f), 7.f);
             const int hi = __shfl_down_sync(0xffffffffu, code, 1);
-            if (col_ok && (lane & 1) == 0) {
-              const long long pgb = (long long)(slot / a.P) * a.G + g;
-              pool[pgb * a.P * row_bytes + swz_offset(slot % a.P, j >> 1, a.P)] =
+            if (col_ok && (lane & 1) == 0)
+              pool[(long long)(slot / a.P) * page_bytes + swz_offset(slot % a.P, j >> 1, a.P)] =
                   (uint8_t)((code & 0xF) | ((hi & 0xF) << 4));
-            }
             if (col_ok && lane == 0) {
-              uint8_t* spool = reinterpret_cast<uint8_t*>(is_v ? a.zvs : a.zks);
+              const uint8_t* spool = is_v ? a.gm.zvs[e] : a.gm.zks[e];
               const long long srow = is_v ? a.vs_row : a.ks_row;
-              const long long prow = ((long long)(slot / a.P) * a.G + g) * a.P + slot % a.P;
-              reinterpret_cast<__half*>(spool + prow * srow)[j >> 5] = s16;
+              const long long spage = is_v ? a.gm.vs_page : a.gm.ks_page;
+              reinterpret_cast<__half*>(const_cast<uint8_t*>(spool) + (long long)(slot / a.P) * spage +
+                                        (slot % a.P) * srow)[j >> 5] = s16;
             }
           } else {
-            if (col_ok) store_latent<LAT>(a, pool, row_bytes, g, j, slot, v[u]);
+            if (col_ok) store_latent<LAT>(a, pool + (long long)(slot / a.P) * page_bytes, j, slot, v[u]);
           }
         }
       }
@@ -331,11 +338,11 @@ bool map2d(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, uint64_t inn
 
 template <int ACT, int LAT>
 cudaError_t launch_t(const CompressArgs& a, cudaStream_t st) {
-  const Plan p = make_plan(a.n, a.d_model, a.G, a.r_k, a.r_v);
+  const Plan p = make_plan(a.n, a.d_model, a.gm.n, a.r_k, a.r_v);
   const CUtensorMapDataType dt = ACT == PALU_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   CUtensorMap tm_ak, tm_av, tm_x;
-  if (!map2d(&tm_ak, a.Ak, dt, (uint64_t)a.G * a.r_k, a.d_model, (uint64_t)a.G * a.r_k * 2, 64, kKStage) ||
-      !map2d(&tm_av, a.Av, dt, (uint64_t)a.G * a.r_v, a.d_model, (uint64_t)a.G * a.r_v * 2, 64, kKStage) ||
+  if (!map2d(&tm_ak, a.Ak, dt, (uint64_t)a.a_kcols, a.d_model, (uint64_t)a.a_kcols * 2, 64, kKStage) ||
+      !map2d(&tm_av, a.Av, dt, (uint64_t)a.a_vcols, a.d_model, (uint64_t)a.a_vcols * 2, 64, kKStage) ||
       !map2d(&tm_x, a.x, dt, a.d_model, a.n, (uint64_t)a.d_model * 2, 64, p.NT))
     return cudaErrorInvalidValue;
   TcArgs t{};

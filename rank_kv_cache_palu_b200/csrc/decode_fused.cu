@@ -90,10 +90,12 @@ __device__ __forceinline__ float from_bits(uint16_t u) {
 // query.
 constexpr int kFoldSeqs = 4;
 template <int ACT>
-__global__ void __launch_bounds__(256) fold_query_kernel(const DecodeArgs a, int qslots, void* qt) {
+__global__ void __launch_bounds__(256) fold_query_kernel(const __grid_constant__ DecodeArgs a, int qslots, void* qt) {
   using TA = typename Dt<ACT>::T;
   __shared__ float qs[kFoldSeqs][kMaxG][128];
-  const int g = blockIdx.x, jb = blockIdx.y, v0 = blockIdx.z * kFoldSeqs;
+  // blockIdx.x: entry gi of the group map (model group g)
+  const int gi = blockIdx.x, jb = blockIdx.y, v0 = blockIdx.z * kFoldSeqs;
+  const int g = a.gm.g[gi];
   const int gs = a.gs, d_h = a.d_h;
   const int nvb = a.batch * qslots;
   auto live = [&](int vb) { return vb < nvb && vb % qslots < a.qn; };
@@ -114,7 +116,7 @@ __global__ void __launch_bounds__(256) fold_query_kernel(const DecodeArgs a, int
   // the row segment as 8-element vectors (d_h is a multiple of 8 here)
   uint4 bseg[16];
   const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const TA*>(a.Bk) +
-                                                    ((size_t)g * a.r_k + j) * a.W + (size_t)h * d_h);
+                                                    ((size_t)a.gm.k_row0[gi] + j) * a.W + (size_t)h * d_h);
 #pragma unroll
   for (int v = 0; v < 16; ++v) bseg[v] = (h < gs && v * 8 < d_h) ? __ldg(src + v) : make_uint4(0, 0, 0, 0);
   constexpr float kLog2e = 1.4426950408889634f;
@@ -131,7 +133,7 @@ __global__ void __launch_bounds__(256) fold_query_kernel(const DecodeArgs a, int
     acc *= sc;
     const TA hi = Dt<ACT>::from_f(acc);
     const TA lo = Dt<ACT>::from_f(acc - Dt<ACT>::to_f(hi));
-    TA* out = reinterpret_cast<TA*>(qt) + ((size_t)(v0 + bb) * a.G + g) * 2 * kMaxG * a.r_k;
+    TA* out = reinterpret_cast<TA*>(qt) + ((size_t)(v0 + bb) * a.gm.n + gi) * 2 * kMaxG * a.r_k;
     out[(size_t)h * a.r_k + j] = hi;
     out[(size_t)(kMaxG + h) * a.r_k + j] = lo;
   }
@@ -179,7 +181,7 @@ __device__ __forceinline__ uint32_t p_offset(int n, int k) {
 
 template <int ACT, int NRV, int QN>
 __global__ void __launch_bounds__(kThreads, 1)
-    decode_fused_kernel(const DecodeArgs a, const void* qt) {
+    decode_fused_kernel(const __grid_constant__ DecodeArgs a, const void* qt) {
   using PS = Pass<QN>;
   constexpr int kN = PS::kN, kNP = PS::kNP, kPC = PS::kPC, kPB = PS::kPBytes;
   extern __shared__ uint8_t smem_raw[];
@@ -192,7 +194,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sbase + L.abort);
   auto bar = [&](int i) { return base + L.bars + 8u * i; };
 
-  const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  // blockIdx.y: entry gi of the group map (model group gm.g[gi])
+  const int s = blockIdx.x, gi = blockIdx.y, b = blockIdx.z;
+  const GroupMap& gm = a.gm;
   const int gs = a.gs;
   const int nq = a.qn;                  // queries of this pass (<= QN)
   const int nkc = a.r_k / kChunk;
@@ -245,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int n = i / a.r_k, j = i % a.r_k;
     const int jj = n >> 3, r = n & 7;
     const uint16_t* src = reinterpret_cast<const uint16_t*>(qt) +
-                          ((((size_t)b * QN + jj) * a.G + g) * 2 * kMaxG + r) * a.r_k;
+                          ((((size_t)b * QN + jj) * gm.n + gi) * 2 * kMaxG + r) * a.r_k;
     const int c = j / kChunk, kin = j % kChunk;
     *reinterpret_cast<uint16_t*>(sbase + L.qt + c * (kN * 128) + n * 128 + (((kin >> 3) ^ (n & 7)) << 4) +
                                  (kin & 7) * 2) = src[j];
@@ -269,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto push_zv = [&](int k) -> bool {
         int pg = page_of(a, b, pg0 + k);
         if (pg < 0) pg = 0;   // reported with the keys
-        const uint8_t* src = reinterpret_cast<const uint8_t*>(a.zv) + (size_t)(pg * a.G + g) * a.P * a.v_row;
+        const uint8_t* src = gm.zv[gi] + (size_t)pg * gm.v_page;
         for (int cb = 0; cb < 2 * NRV; ++cb) {
           if (!mbar_wait(bar(BAR_ZV_EMPTY + vs), vph ^ 1, abort_flag, st, 11)) return false;
           mbar_expect_tx(bar(BAR_ZV_FULL + vs), kStageBytes);
@@ -285,7 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           report(st, PALU_ERR_DEVICE_BOUNDS, 2000000 + b);
           pg = 0;   // keep the pipeline fed from a valid page; the status says the result is void
         }
-        const uint8_t* src = reinterpret_cast<const uint8_t*>(a.zk) + (size_t)(pg * a.G + g) * a.P * a.k_row;
+        const uint8_t* src = gm.zk[gi] + (size_t)pg * gm.k_page;
         for (int c = 0; c < nkc; ++c) {
           if (!mbar_wait(bar(BAR_ZK_EMPTY + zs), zph ^ 1, abort_flag, st, 10)) { ok = false; break; }
           mbar_expect_tx(bar(BAR_ZK_FULL + zs), kStageBytes);
@@ -475,7 +479,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int p = 0; p < kPC; ++p) at[mb][p] = 0.f;
         if (pg >= 0) {
-          const uint8_t* zv = reinterpret_cast<const uint8_t*>(a.zv) + (size_t)(pg * a.G + g) * a.P * a.v_row;
+          const uint8_t* zv = gm.zv[gi] + (size_t)pg * gm.v_page;
           const uint8_t* pbuf = sbase + L.p + (kl & 1) * kPB;
           for (int t = 0; t < nvalid; ++t) {
             float z[NRV];
@@ -513,7 +517,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!live(p)) continue;
         const int jj = p >> 2, h = p & 3;
         // partials of virtual sequence b·QN + jj (the combine maps it back)
-        float* out = a.part + ((((size_t)b * QN + jj) * a.H + g * gs + h) * a.S + s) * (a.r_v + 2);
+        float* out = a.part + ((((size_t)b * QN + jj) * gm.n * gs + gi * gs + h) * a.S + s) * (a.r_v + 2);
         if (row == 0) {
           out[0] = ntiles > 0 ? m_run[p] * kLn2 : -INFINITY;
           out[1] = (lred[p] + lred[kPC + p]) + (lred[2 * kPC + p] + lred[3 * kPC + p]);
@@ -537,7 +541,7 @@ template <int ACT, int NRV, int QN>
 cudaError_t launch_t(const DecodeArgs& a, cudaStream_t st) {
   void* qt = a.fused_q;
   const int vb = a.batch * QN;   // one folded query per (sequence, query slot of the pass)
-  fold_query_kernel<ACT><<<dim3(a.G, (a.r_k + 63) / 64, (vb + kFoldSeqs - 1) / kFoldSeqs), 256, 0, st>>>(a, QN, qt);
+  fold_query_kernel<ACT><<<dim3(a.gm.n, (a.r_k + 63) / 64, (vb + kFoldSeqs - 1) / kFoldSeqs), 256, 0, st>>>(a, QN, qt);
   count_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -546,7 +550,7 @@ cudaError_t launch_t(const DecodeArgs& a, cudaStream_t st) {
   auto kern = decode_fused_kernel<ACT, NRV, QN>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<dim3(a.S, a.G, a.batch), kThreads, smem, st>>>(a, qt);
+  kern<<<dim3(a.S, a.gm.n, a.batch), kThreads, smem, st>>>(a, qt);
   count_launch();
   return cudaGetLastError();
 }

@@ -45,12 +45,14 @@ __device__ __forceinline__ SplitRange split_range(int T, int P, int S, int s) {
 }
 
 template <int ACT, int LAT>
-__global__ void __launch_bounds__(kThreads) split_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(kThreads) split_kernel(const __grid_constant__ DecodeArgs a) {
   using TA = typename Dt<ACT>::T;
   extern __shared__ float smem[];
-  const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  // blockIdx.y: head hl of this launch; entry i = hl / gs of the group map
+  const int s = blockIdx.x, hl = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x;
-  const int g = h / a.gs, jh = h % a.gs;
+  const int gi = hl / a.gs, jh = hl % a.gs;
+  const int h = a.gm.g[gi] * a.gs + jh;   // model head
   const int d_h = a.d_h, half = d_h / 2;
   DevStatus* st = reinterpret_cast<DevStatus*>(a.status);
 
@@ -81,11 +83,11 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const DecodeArgs a) {
   for (int k = 0; k < kMaxRv / kThreads; ++k) acc_v[k] = 0.f;
   float m_run = -INFINITY, l_run = 0.f;
 
-  const TA* Bk = reinterpret_cast<const TA*>(a.Bk) + (size_t)g * a.r_k * a.W + jh * d_h;
-  const uint8_t* zk_base = reinterpret_cast<const uint8_t*>(a.zk);
-  const uint8_t* zv_base = reinterpret_cast<const uint8_t*>(a.zv);
-  const uint8_t* zks_base = reinterpret_cast<const uint8_t*>(a.zks);
-  const uint8_t* zvs_base = reinterpret_cast<const uint8_t*>(a.zvs);
+  const TA* Bk = reinterpret_cast<const TA*>(a.Bk) + (size_t)a.gm.k_row0[gi] * a.W + jh * d_h;
+  const uint8_t* zk_base = a.gm.zk[gi];
+  const uint8_t* zv_base = a.gm.zv[gi];
+  const uint8_t* zks_base = a.gm.zks[gi];
+  const uint8_t* zvs_base = a.gm.zvs[gi];
   const int32_t* ptab = a.page_table + (size_t)b * a.max_pages;
 
   for (int t0 = rg.t_begin; t0 < rg.t_end; t0 += kTT) {
@@ -111,10 +113,11 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const DecodeArgs a) {
         if (page < 0 || page >= a.num_pages) {
           report(st, PALU_ERR_DEVICE_BOUNDS, 2000000 + b);
         } else {
-          const size_t blk = (size_t)page * a.G + g;
-          const size_t row = blk * a.P + t % a.P;
-          v = load_latent<LAT, ACT>(zk_base + blk * a.P * a.k_row, t % a.P, a.P,
-                                    LAT == PALU_INT4 ? zks_base + row * a.ks_row : nullptr, j);
+          v = load_latent<LAT, ACT>(zk_base + (size_t)page * a.gm.k_page, t % a.P, a.P,
+                                    LAT == PALU_INT4 ? zks_base + (size_t)page * a.gm.ks_page +
+                                                           (size_t)(t % a.P) * a.ks_row
+                                                     : nullptr,
+                                    j);
         }
       }
       zk_t[e] = v;
@@ -126,10 +129,11 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const DecodeArgs a) {
         const int t = t0 + tt;
         const int page = ptab[t / a.P];
         if (page >= 0 && page < a.num_pages) {
-          const size_t blk = (size_t)page * a.G + g;
-          const size_t row = blk * a.P + t % a.P;
-          v = load_latent<LAT, ACT>(zv_base + blk * a.P * a.v_row, t % a.P, a.P,
-                                    LAT == PALU_INT4 ? zvs_base + row * a.vs_row : nullptr, j);
+          v = load_latent<LAT, ACT>(zv_base + (size_t)page * a.gm.v_page, t % a.P, a.P,
+                                    LAT == PALU_INT4 ? zvs_base + (size_t)page * a.gm.vs_page +
+                                                           (size_t)(t % a.P) * a.vs_row
+                                                     : nullptr,
+                                    j);
         }
       }
       zv_t[e] = v;
@@ -194,7 +198,7 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const DecodeArgs a) {
     }
   }
 
-  float* out = a.part + (((size_t)b * a.H + h) * a.S + s) * (a.r_v + 2);
+  float* out = a.part + (((size_t)b * a.gm.n * a.gs + hl) * a.S + s) * (a.r_v + 2);
   if (tid == 0) {
     out[0] = m_run;
     out[1] = l_run;
@@ -209,17 +213,19 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const DecodeArgs a) {
 // Log-sum-exp merge of the split partials, then the value up-projection
 // out_h = a_h · B_v[g][:, cols_h] (a GEMV per (sequence, head)).
 template <int ACT>
-__global__ void __launch_bounds__(kThreads) combine_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(kThreads) combine_kernel(const __grid_constant__ DecodeArgs a) {
   using TA = typename Dt<ACT>::T;
   extern __shared__ float smem[];
   float* av = smem;             // [r_v]
   float* wgt = av + a.r_v;      // [S]
   // virtual sequence vb = b·qn + j: query j of sequence b (qn = 1: one query per sequence)
-  const int h = blockIdx.x, vb = blockIdx.y;
+  // blockIdx.x: head hl of this launch (entry hl / gs of the group map)
+  const int hl = blockIdx.x, vb = blockIdx.y;
   const int b = vb / a.qn, jq = vb % a.qn;
   const int tid = threadIdx.x;
-  const int g = h / a.gs, jh = h % a.gs;
-  const float* part = a.part + ((size_t)vb * a.H + h) * a.S * (a.r_v + 2);
+  const int gi = hl / a.gs, jh = hl % a.gs;
+  const int h = a.gm.g[gi] * a.gs + jh;   // model head
+  const float* part = a.part + ((size_t)vb * a.gm.n * a.gs + hl) * a.S * (a.r_v + 2);
 
   float M = -INFINITY;
   for (int s = 0; s < a.S; ++s) M = fmaxf(M, part[(size_t)s * (a.r_v + 2)]);
@@ -247,7 +253,7 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const DecodeArgs a) {
     av[r] = v * invL;
   }
   __syncthreads();
-  const TA* Bv = reinterpret_cast<const TA*>(a.Bv) + (size_t)g * a.r_v * a.W + jh * a.d_h;
+  const TA* Bv = reinterpret_cast<const TA*>(a.Bv) + (size_t)a.gm.v_row0[gi] * a.W + jh * a.d_h;
   for (int d = tid; d < a.d_h; d += kThreads) {
     float o = 0.f;
     for (int r = 0; r < a.r_v; ++r) o = fmaf(av[r], Dt<ACT>::to_f(Bv[(size_t)r * a.W + d]), o);
@@ -264,7 +270,7 @@ cudaError_t launch_split_t(const DecodeArgs& a, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  dim3 grid(a.S, a.H, a.batch);
+  dim3 grid(a.S, a.gm.n * a.gs, a.batch);
   kern<<<grid, kThreads, smem, st>>>(a);
   count_launch();
   return cudaGetLastError();
@@ -283,7 +289,7 @@ cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t st) {
 
 cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t st) {
   const size_t smem = sizeof(float) * (a.r_v + a.S);
-  dim3 grid(a.H, a.batch * a.qn);
+  dim3 grid(a.gm.n * a.gs, a.batch * a.qn);
   if (a.act == PALU_F32) combine_kernel<PALU_F32><<<grid, kThreads, smem, st>>>(a);
   else if (a.act == PALU_F16) combine_kernel<PALU_F16><<<grid, kThreads, smem, st>>>(a);
   else if (a.act == PALU_BF16) combine_kernel<PALU_BF16><<<grid, kThreads, smem, st>>>(a);

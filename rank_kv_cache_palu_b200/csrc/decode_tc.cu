@@ -238,7 +238,7 @@ __device__ __forceinline__ void trace_record(const DecodeArgs& a, int ev, int k,
 
 template <int ACT, int NRV, int LAT>
 __global__ void __launch_bounds__(kThreads, 1)
-    decode_tc_kernel(const __grid_constant__ CUtensorMap tm_bk, const DecodeArgs a) {
+    decode_tc_kernel(const __grid_constant__ CUtensorMap tm_bk, const __grid_constant__ DecodeArgs a) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -254,7 +254,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int b = blockIdx.z;
   const int nhp = a.gs / 2;                         // head pairs per group
-  const int g = blockIdx.y / nhp, hp = blockIdx.y % nhp;
+  const int gi = blockIdx.y / nhp, hp = blockIdx.y % nhp;   // entry gi of the group map
+  const GroupMap& gm = a.gm;
   const int nkc = a.r_k / kChunk;
   const TileRange tr = tile_range(a, b, st, threadIdx.x == 0);
   const long long t_start = clock64();
@@ -308,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     mbar_expect_tx(bar(BAR_B), (uint32_t)a.r_k * 256 * 2);
     for (int nb = 0; nb < 4; ++nb)
-      tma_load_2d(base + L.b + (uint32_t)nb * a.r_k * 128, &tm_bk, hp * 256 + nb * 64, g * a.r_k, bar(BAR_B));
+      tma_load_2d(base + L.b + (uint32_t)nb * a.r_k * 128, &tm_bk, hp * 256 + nb * 64, gm.k_row0[gi], bar(BAR_B));
   }
   if (kInt4 && (warp == 0 || warp == 3)) {
     // ============================================================ int4 key codes (warps 0, 3)
@@ -334,16 +335,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = (k == 0 ? 1 : k + kPrefetch); kk <= k + kPrefetch && kk < tr.ntiles; ++kk) {
           const int ppg = page_of(a, b, tr.t_begin / kTile + kk);
           if (ppg < 0) continue;
-          const size_t prow = (size_t)(ppg * a.G + g) * a.P;
-          prefetch_l2(reinterpret_cast<const uint8_t*>(a.zk) + prow * a.k_row, (uint32_t)(a.P * a.k_row));
-          prefetch_l2(reinterpret_cast<const uint8_t*>(a.zks) + prow * a.ks_row, (uint32_t)(a.P * a.ks_row));
-          prefetch_l2(reinterpret_cast<const uint8_t*>(a.zv) + prow * a.v_row, (uint32_t)(a.P * a.v_row));
-          prefetch_l2(reinterpret_cast<const uint8_t*>(a.zvs) + prow * a.vs_row, (uint32_t)(a.P * a.vs_row));
+          prefetch_l2(gm.zk[gi] + (size_t)ppg * gm.k_page, (uint32_t)(a.P * a.k_row));
+          prefetch_l2(gm.zks[gi] + (size_t)ppg * gm.ks_page, (uint32_t)(a.P * a.ks_row));
+          prefetch_l2(gm.zv[gi] + (size_t)ppg * gm.v_page, (uint32_t)(a.P * a.v_row));
+          prefetch_l2(gm.zvs[gi] + (size_t)ppg * gm.vs_page, (uint32_t)(a.P * a.vs_row));
         }
       }
-      const size_t row0 = (size_t)(pg * a.G + g) * a.P;
-      const uint8_t* blk = reinterpret_cast<const uint8_t*>(a.zk) + row0 * 128;
-      const uint8_t* sblk = reinterpret_cast<const uint8_t*>(a.zks) + row0 * a.ks_row;
+      const uint8_t* blk = gm.zk[gi] + (size_t)pg * gm.k_page;
+      const uint8_t* sblk = gm.zks[gi] + (size_t)pg * gm.ks_page;
       const int u = 2 * (n & 3) + (zt & 1);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -399,10 +398,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto load_raw = [&](int k) {
       int pg = page_of(a, b, tr.t_begin / kTile + k);
       if (pg < 0) pg = 0;   // reported by the key producer
-      const size_t row0 = (size_t)(pg * a.G + g) * a.P;
       mbar_expect_tx(bar(BAR_VRAW), kVRawBytes);
-      bulk_load(vraw, reinterpret_cast<const uint8_t*>(a.zv) + row0 * 128, 128 * 128, bar(BAR_VRAW));
-      bulk_load(vraw + 128 * 128, reinterpret_cast<const uint8_t*>(a.zvs) + row0 * a.vs_row, 128 * 16,
+      bulk_load(vraw, gm.zv[gi] + (size_t)pg * gm.v_page, 128 * 128, bar(BAR_VRAW));
+      bulk_load(vraw + 128 * 128, gm.zvs[gi] + (size_t)pg * gm.vs_page, 128 * 16,
                 bar(BAR_VRAW));
     };
     if (lane == 0 && nv_tiles > 0) load_raw(0);
@@ -449,10 +447,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (kk >= tr.ntiles) return;
         const int ppg = page_of(a, b, tr.t_begin / kTile + kk);
         if (ppg < 0) return;
-        const size_t row = (size_t)(ppg * a.G + g) * a.P;
-        prefetch_l2(reinterpret_cast<const uint8_t*>(a.zk) + row * a.k_row, (uint32_t)(a.P * a.k_row));
+        prefetch_l2(gm.zk[gi] + (size_t)ppg * gm.k_page, (uint32_t)(a.P * a.k_row));
         if (!(tr.ragged_last && kk == tr.ntiles - 1))
-          prefetch_l2(reinterpret_cast<const uint8_t*>(a.zv) + row * a.v_row, (uint32_t)(a.P * a.v_row));
+          prefetch_l2(gm.zv[gi] + (size_t)ppg * gm.v_page, (uint32_t)(a.P * a.v_row));
       };
       for (int kk = 0; kk < kPrefetch; ++kk) prefetch_page(kk);
       for (int k = 0; k < tr.ntiles && !*abort_flag; ++k) {
@@ -465,7 +462,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // one (page, group) block is the shared-memory image of the tile: each
         // 128-byte column block (64 latent entries of all 128 tokens) is one copy
-        const uint8_t* src = reinterpret_cast<const uint8_t*>(a.zk) + (size_t)(pg * a.G + g) * a.P * a.k_row;
+        const uint8_t* src = gm.zk[gi] + (size_t)pg * gm.k_page;
         for (int c = 0; c < nkc; ++c) {
           if (!mbar_wait(bar(BAR_ZK_EMPTY + stage), phase ^ 1, abort_flag, st, 10)) break;
           mbar_expect_tx(bar(BAR_ZK_FULL + stage), kZkBytes);
@@ -485,7 +482,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int lp = tr.t_begin / kTile + k;
         int pg = page_of(a, b, lp);
         if (pg < 0) pg = 0;   // reported by the z_k producer
-        const uint8_t* src = reinterpret_cast<const uint8_t*>(a.zv) + (size_t)(pg * a.G + g) * a.P * a.v_row;
+        const uint8_t* src = gm.zv[gi] + (size_t)pg * gm.v_page;
         // one copy per 128-byte column block of the page (64 latent entries of
         // all 128 tokens); two consecutive blocks are the two MN-blocks of one
         // value-MMA operand
@@ -606,7 +603,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     float* qr = reinterpret_cast<float*>(sbase + L.qr);
     float* psc = reinterpret_cast<float*>(sbase + L.psc);   // [slot][head][128]
     const uint64_t* om = reinterpret_cast<const uint64_t*>(sbase + L.omega);
-    const int head0 = g * a.gs + hp * 2;
+    const int head0 = gm.g[gi] * a.gs + hp * 2;   // model head of the pair's first head
+    const int hl0 = gi * a.gs + hp * 2;           // the same head among this launch's heads
     constexpr float kLog2e = 1.4426950408889634f;
     // the 4 warps of one warpgroup meet here; a bounded wait (unlike bar.sync), so a thread that gave
     // up on a timed-out wait cannot strand the others.
@@ -830,9 +828,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int mb = 0; mb < NRV; ++mb) at[mb] = 0.f;
           if (pg >= 0) {
-            const size_t row0 = (size_t)(pg * a.G + g) * a.P;
-            const uint8_t* zv = reinterpret_cast<const uint8_t*>(a.zv) + row0 * a.v_row;
-            const uint8_t* zvs = kInt4 ? reinterpret_cast<const uint8_t*>(a.zvs) + row0 * a.vs_row : nullptr;
+            const uint8_t* zv = gm.zv[gi] + (size_t)pg * gm.v_page;
+            const uint8_t* zvs = kInt4 ? gm.zvs[gi] + (size_t)pg * gm.vs_page : nullptr;
             const uint8_t* pbuf = sbase + L.p + (kl & 1) * kPBytes;
             for (int t = 0; t < nvalid; ++t) {
               const float pv = from_bits<ACT>(*reinterpret_cast<const uint16_t*>(pbuf + p_offset(hw, t)));
@@ -856,7 +853,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = ep_sync(35) && ok;
       if (ok && !*abort_flag) {
         constexpr float kLn2 = 0.6931471805599453f;
-        float* out = a.part + (((size_t)b * a.H + head0 + hw) * a.S + blockIdx.x) * (a.r_v + 2);
+        float* out = a.part + (((size_t)b * gm.n * a.gs + hl0 + hw) * a.S + blockIdx.x) * (a.r_v + 2);
         if (row == 0) {
           out[0] = tr.ntiles > 0 ? m_run * kLn2 : -INFINITY;
           out[1] = (lred[wg * 4 + 0] + lred[wg * 4 + 1]) + (lred[wg * 4 + 2] + lred[wg * 4 + 3]);
@@ -911,7 +908,7 @@ template <int ACT, int NRV, int LAT>
 cudaError_t launch_t(const DecodeArgs& a, cudaStream_t st) {
   const CUtensorMapDataType dt = ACT == PALU_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   CUtensorMap tm_bk;
-  if (!make_map_2d(&tm_bk, a.Bk, dt, 2, a.W, (uint64_t)a.G * a.r_k, (uint64_t)a.W * 2, 64, a.r_k,
+  if (!make_map_2d(&tm_bk, a.Bk, dt, 2, a.W, (uint64_t)a.bk_rows, (uint64_t)a.W * 2, 64, a.r_k,
                    CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   const Smem L = smem_layout(a.r_k, LAT == PALU_INT4);
@@ -919,14 +916,14 @@ cudaError_t launch_t(const DecodeArgs& a, cudaStream_t st) {
   auto kern = decode_tc_kernel<ACT, NRV, LAT>;
   DecodeArgs args = a;
   const TraceSetting ts = trace_setting();
-  const size_t ctas = (size_t)a.S * a.G * (a.gs / 2) * a.batch;
+  const size_t ctas = (size_t)a.S * a.gm.n * (a.gs / 2) * a.batch;
   if (ts.buffer != nullptr && ctas * 8 * (size_t)ts.tiles * 8 <= ts.bytes) {
     args.trace = static_cast<long long*>(ts.buffer);
     args.trace_tiles = ts.tiles;
   }
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(a.S, a.G * (a.gs / 2), a.batch);
+  dim3 grid(a.S, a.gm.n * (a.gs / 2), a.batch);
   kern<<<grid, kThreads, smem, st>>>(tm_bk, args);
   count_launch();
   return cudaGetLastError();

@@ -46,6 +46,7 @@ palu_status check_config(const palu_config* c) {
   if (!pair_ok) return PALU_ERR_UNSUPPORTED;
   if (c->head_dim > 2 * palu::kMaxHalfDim) return PALU_ERR_UNSUPPORTED;
   if (c->rank_k > 512 || c->rank_v > 512) return PALU_ERR_UNSUPPORTED;
+  if (c->num_heads / c->group_size > palu::kMaxGroups) return PALU_ERR_UNSUPPORTED;
   // latent rows are whole 128-byte column blocks (the swizzled page layout)
   if (palu::latent_row_bytes(c->latent_dtype, c->rank_k) % 128 != 0 ||
       palu::latent_row_bytes(c->latent_dtype, c->rank_v) % 128 != 0)
@@ -81,18 +82,6 @@ int pass_queries(int kind, int remaining) {
   return remaining >= m ? m : remaining >= 2 ? 2 : 1;
 }
 
-// Workspace layout: status word, partials [vb][H][S][r_v + 2] for vb virtual
-// sequences (sequence × query slot of a pass), then (fused kernel) the folded
-// queries.  Returns the total; *fused_off receives the offset of the queries.
-size_t workspace_layout(const palu_config* c, int kind, int vb, int S, size_t* fused_off) {
-  const size_t part = (size_t)vb * c->num_heads * S * (c->rank_v + 2) * sizeof(float);
-  size_t total = kStatusBytes + align256(part);
-  if (fused_off) *fused_off = total;
-  if (kind == 3) total += align256(palu::fused_query_bytes(c, vb));
-  return total;
-}
-
-
 int auto_splits(const palu_config* c, int batch, int max_pages, int kind) {
   const int sms = 148;
   const long long groups = (long long)batch * (c->num_heads / c->group_size);
@@ -121,6 +110,294 @@ int kernel_kind(const palu_config* c) {
 // The split count a call runs (num_splits = 0: automatic).
 int run_S(const palu_config* c, int kind, int batch, int max_pages, int num_splits) {
   return num_splits == 0 ? auto_splits(c, batch, max_pages, kind) : num_splits;
+}
+
+// One layer's head groups and where their latents live.  Group g has its own
+// rank pair (r_k,g, r_v,g) — one pair for all groups unless the caller gives a
+// rank per group.  A page of the K pool holds every group's block back to back,
+// group g's at byte Σ_{g'<g} P·row_k,g' (likewise V and the int4 scale pools);
+// B_k stacks the groups' [r_k,g × W] blocks, so group g's rows start at
+// Σ_{g'<g} r_k,g', and A_k's columns follow the same order.  With one rank pair
+// this is the layout pool[page][g][P rows].  Groups with equal rank pairs form
+// a class, which one launch of each kernel serves.
+struct Layer {
+  palu_config cfg;   // model shape and dtypes (rank fields: see rk / rv)
+  int G;
+  int rk[palu::kMaxGroups], rv[palu::kMaxGroups];
+  long long k_off[palu::kMaxGroups], v_off[palu::kMaxGroups];
+  long long ks_off[palu::kMaxGroups], vs_off[palu::kMaxGroups];
+  long long k_page, v_page, ks_page, vs_page;   // bytes per page of each pool
+  int k_row0[palu::kMaxGroups], v_row0[palu::kMaxGroups];
+  int bk_rows, bv_rows;                         // Σ r_k,g and Σ r_v,g
+  int nclass;
+  int cls[palu::kMaxGroups];                    // class of each group
+  int crk[palu::kMaxGroups], crv[palu::kMaxGroups], cn[palu::kMaxGroups];
+};
+
+palu_status make_layer(const palu_config* cfg, const int32_t* ranks_k, const int32_t* ranks_v, Layer* L) {
+  if (cfg == nullptr || (ranks_k == nullptr) != (ranks_v == nullptr)) return PALU_ERR_INVALID_ARG;
+  // the shape checks, with group 0's ranks standing in for cfg's when ranks are given
+  palu_config c0 = *cfg;
+  if (ranks_k != nullptr) {
+    c0.rank_k = ranks_k[0];
+    c0.rank_v = ranks_v[0];
+  }
+  palu_status s = check_config(&c0);
+  if (s != PALU_OK) return s;
+  L->cfg = *cfg;
+  const int G = cfg->num_heads / cfg->group_size;
+  const long long P = cfg->page_size;
+  const int lat = cfg->latent_dtype;
+  L->G = G;
+  L->nclass = 0;
+  long long ko = 0, vo = 0, kso = 0, vso = 0;
+  int kr = 0, vr = 0;
+  for (int g = 0; g < G; ++g) {
+    palu_config c = *cfg;
+    c.rank_k = ranks_k ? ranks_k[g] : cfg->rank_k;
+    c.rank_v = ranks_v ? ranks_v[g] : cfg->rank_v;
+    s = check_config(&c);
+    if (s != PALU_OK) return s;
+    L->rk[g] = c.rank_k;
+    L->rv[g] = c.rank_v;
+    L->k_off[g] = ko;
+    L->v_off[g] = vo;
+    L->ks_off[g] = kso;
+    L->vs_off[g] = vso;
+    ko += P * palu::latent_row_bytes(lat, c.rank_k);
+    vo += P * palu::latent_row_bytes(lat, c.rank_v);
+    kso += P * palu::scale_row_bytes(lat, c.rank_k);
+    vso += P * palu::scale_row_bytes(lat, c.rank_v);
+    L->k_row0[g] = kr;
+    L->v_row0[g] = vr;
+    kr += c.rank_k;
+    vr += c.rank_v;
+    int k = 0;
+    while (k < L->nclass && !(L->crk[k] == c.rank_k && L->crv[k] == c.rank_v)) ++k;
+    if (k == L->nclass) {
+      L->crk[k] = c.rank_k;
+      L->crv[k] = c.rank_v;
+      L->cn[k] = 0;
+      ++L->nclass;
+    }
+    L->cls[g] = k;
+    ++L->cn[k];
+  }
+  L->k_page = ko;
+  L->v_page = vo;
+  L->ks_page = kso;
+  L->vs_page = vso;
+  L->bk_rows = kr;
+  L->bv_rows = vr;
+  return PALU_OK;
+}
+
+// The config one class's launches see: its groups and its ranks.
+palu_config class_cfg(const Layer& L, int c) {
+  palu_config x = L.cfg;
+  x.num_heads = L.cn[c] * L.cfg.group_size;
+  x.rank_k = L.crk[c];
+  x.rank_v = L.crv[c];
+  return x;
+}
+
+void class_map(const Layer& L, int c, const void* zk, const void* zv, const void* zks, const void* zvs,
+               palu::GroupMap& m) {
+  auto at = [](const void* pool, long long off) {
+    return pool == nullptr ? nullptr : static_cast<const uint8_t*>(pool) + off;
+  };
+  m.n = 0;
+  m.k_page = L.k_page;
+  m.v_page = L.v_page;
+  m.ks_page = L.ks_page;
+  m.vs_page = L.vs_page;
+  for (int g = 0; g < L.G; ++g) {
+    if (L.cls[g] != c) continue;
+    const int i = m.n++;
+    m.g[i] = g;
+    m.zk[i] = at(zk, L.k_off[g]);
+    m.zv[i] = at(zv, L.v_off[g]);
+    m.zks[i] = at(zks, L.ks_off[g]);
+    m.zvs[i] = at(zvs, L.vs_off[g]);
+    m.k_row0[i] = L.k_row0[g];
+    m.v_row0[i] = L.v_row0[g];
+  }
+}
+
+// Decode workspace: the status word, then the partials of the largest class
+// ([vb][heads][S][r_v + 2] float32, vb = sequence × query slot of a pass),
+// then the folded queries of the largest fused-kernel class.  Classes run one
+// after another on the stream, so they share both regions.
+size_t decode_workspace(const Layer& L, int batch, int Q, int max_pages, int num_splits, size_t* fused_off) {
+  size_t part = 0, fq = 0;
+  for (int c = 0; c < L.nclass; ++c) {
+    const palu_config cc = class_cfg(L, c);
+    const int kind = kernel_kind(&cc);
+    const int S = run_S(&cc, kind, batch, max_pages, num_splits);
+    const int vb = batch * pass_queries(kind, Q);
+    const size_t pc = align256((size_t)vb * cc.num_heads * S * (cc.rank_v + 2) * sizeof(float));
+    if (pc > part) part = pc;
+    if (kind == 3) {
+      const size_t f = align256(palu::fused_query_bytes(&cc, vb));
+      if (f > fq) fq = f;
+    }
+  }
+  if (fused_off) *fused_off = kStatusBytes + part;
+  return kStatusBytes + part + fq;
+}
+
+size_t compress_workspace(const Layer& L, int n_tokens, int d_model) {
+  size_t sc = 0;
+  for (int c = 0; c < L.nclass; ++c) {
+    const palu_config cc = class_cfg(L, c);
+    const size_t b = palu::tc_compress_scratch_bytes(&cc, n_tokens, d_model);
+    if (b > sc) sc = b;
+  }
+  return kStatusBytes + sc;
+}
+
+palu_status compress_layer(const Layer& L, int n_tokens, int d_model, const void* x, const void* A_k,
+                           const void* A_v, const int32_t* slot_mapping, const int32_t* positions, void* zk_pool,
+                           void* zv_pool, void* zk_scales, void* zv_scales, int32_t* pos_pool, int num_pages,
+                           void* workspace, size_t workspace_bytes, palu_stream_t stream) {
+  const palu_config* cfg = &L.cfg;
+  if (n_tokens < 0 || d_model <= 0 || num_pages < 0) return PALU_ERR_INVALID_ARG;
+  if (d_model % 64 != 0) return PALU_ERR_UNSUPPORTED;
+  if (workspace == nullptr || workspace_bytes < compress_workspace(L, n_tokens, d_model)) return PALU_ERR_WORKSPACE;
+  if (n_tokens == 0) return PALU_OK;
+  if (!x || !A_k || !A_v || !slot_mapping || !zk_pool || !zv_pool) return PALU_ERR_INVALID_ARG;
+  const bool int4 = cfg->latent_dtype == PALU_INT4;
+  if (int4 && (!zk_scales || !zv_scales)) return PALU_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(A_k) || !aligned16(A_v) || !aligned16(zk_pool) ||
+      !aligned16(zv_pool) || (int4 && (!aligned16(zk_scales) || !aligned16(zv_scales))) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return PALU_ERR_ALIGNMENT;
+
+  palu::CompressArgs a{};
+  a.n = n_tokens;
+  a.d_model = d_model;
+  a.G = L.G;
+  a.P = cfg->page_size;
+  a.num_pages = num_pages;
+  a.act = cfg->act_dtype;
+  a.lat = cfg->latent_dtype;
+  a.x = x;
+  a.Ak = A_k;
+  a.Av = A_v;
+  a.slots = slot_mapping;
+  a.pos_pool = pos_pool;
+  a.status = workspace;
+  a.scratch = reinterpret_cast<float*>(static_cast<char*>(workspace) + kStatusBytes);
+  a.scratch_bytes = workspace_bytes - kStatusBytes;
+  a.a_kcols = L.bk_rows;
+  a.a_vcols = L.bv_rows;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  for (int c = 0; c < L.nclass; ++c) {
+    const palu_config cc = class_cfg(L, c);
+    a.r_k = cc.rank_k;
+    a.r_v = cc.rank_v;
+    a.k_row = palu::latent_row_bytes(a.lat, a.r_k);
+    a.v_row = palu::latent_row_bytes(a.lat, a.r_v);
+    a.ks_row = palu::scale_row_bytes(a.lat, a.r_k);
+    a.vs_row = palu::scale_row_bytes(a.lat, a.r_v);
+    class_map(L, c, zk_pool, zv_pool, zk_scales, zv_scales, a.gm);
+    a.positions = c == 0 ? positions : nullptr;   // once per token
+    const cudaError_t e = palu::tc_compress_supported(&cc, n_tokens, d_model) ? palu::launch_compress_tc(a, st)
+                                                                             : palu::launch_compress_simt(a, st);
+    if (e != cudaSuccess) return cuda_status(e);
+  }
+  return PALU_OK;
+}
+
+// One decode step for Q queries per sequence (Q = 1: palu_decode_attn).  Each
+// rank class runs its split kernel and combine over its own groups; within a
+// class, passes of queries run one after another on the stream, sharing the
+// workspace.  With Q > 1 a query attends only to the tokens at or before its
+// own position.
+palu_status decode_layer(const Layer& L, int batch, int Q, const void* q, const int32_t* q_pos,
+                         const void* zk_pool, const void* zv_pool, const void* zk_scales, const void* zv_scales,
+                         const int32_t* pos_pool, const int32_t* page_table, int max_pages, const int32_t* seq_lens,
+                         int num_pages, const void* B_k, const void* B_v, void* out, float* lse, void* workspace,
+                         size_t workspace_bytes, int num_splits, palu_stream_t stream) {
+  const palu_config* cfg = &L.cfg;
+  if (batch < 0 || max_pages <= 0 || num_pages < 0 || num_splits < 0 || Q < 1 || Q > kMaxQueries)
+    return PALU_ERR_INVALID_ARG;
+  if (num_splits > max_pages) return PALU_ERR_INVALID_ARG;
+  size_t fused_off = 0;
+  const size_t need = decode_workspace(L, batch, Q, max_pages, num_splits, &fused_off);
+  if (workspace == nullptr || workspace_bytes < need) return PALU_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return PALU_ERR_ALIGNMENT;
+  if (batch == 0) return PALU_OK;
+  if (!q || !q_pos || !zk_pool || !zv_pool || !page_table || !seq_lens || !B_k || !B_v || !out)
+    return PALU_ERR_INVALID_ARG;
+  const bool int4 = cfg->latent_dtype == PALU_INT4;
+  if (int4 && (!zk_scales || !zv_scales)) return PALU_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(zk_pool) || !aligned16(zv_pool) || !aligned16(B_k) ||
+      !aligned16(B_v) || (int4 && (!aligned16(zk_scales) || !aligned16(zv_scales))))
+    return PALU_ERR_ALIGNMENT;
+
+  palu::DecodeArgs a{};
+  a.H = cfg->num_heads;
+  a.d_h = cfg->head_dim;
+  a.gs = cfg->group_size;
+  a.G = L.G;
+  a.W = cfg->group_size * cfg->head_dim;
+  a.P = cfg->page_size;
+  a.batch = batch;
+  a.max_pages = max_pages;
+  a.num_pages = num_pages;
+  a.act = cfg->act_dtype;
+  a.lat = cfg->latent_dtype;
+  a.rope = cfg->rope_base != 0.f;
+  a.sm_scale = (float)(1.0 / sqrt((double)cfg->head_dim));
+  a.pos_pool = pos_pool;
+  a.page_table = page_table;
+  a.seq_lens = seq_lens;
+  a.Bk = B_k;
+  a.Bv = B_v;
+  a.bk_rows = L.bk_rows;
+  a.bv_rows = L.bv_rows;
+  a.status = workspace;
+  a.part = reinterpret_cast<float*>(static_cast<char*>(workspace) + kStatusBytes);
+  a.fused_q = static_cast<char*>(workspace) + fused_off;
+  fill_omega(cfg, a.omega);
+
+  const long long qrow = (long long)a.H * a.d_h;       // one query's elements per sequence
+  const size_t elt = cfg->act_dtype == PALU_F32 ? 4 : 2;
+  if (Q > 1 && (qrow * (long long)elt) % 16 != 0) return PALU_ERR_ALIGNMENT;
+  a.q_bstride = Q * qrow;
+  a.o_bstride = Q * qrow;
+  a.qpos_bstride = Q;
+  a.lse_bstride = Q * a.H;
+  a.causal = Q > 1;
+
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  for (int c = 0; c < L.nclass; ++c) {
+    const palu_config cc = class_cfg(L, c);
+    const int kind = kernel_kind(&cc);
+    a.S = run_S(&cc, kind, batch, max_pages, num_splits);
+    a.r_k = cc.rank_k;
+    a.r_v = cc.rank_v;
+    a.k_row = palu::latent_row_bytes(a.lat, a.r_k);
+    a.v_row = palu::latent_row_bytes(a.lat, a.r_v);
+    a.ks_row = palu::scale_row_bytes(a.lat, a.r_k);
+    a.vs_row = palu::scale_row_bytes(a.lat, a.r_v);
+    class_map(L, c, zk_pool, zv_pool, zk_scales, zv_scales, a.gm);
+    for (int j = 0; j < Q; j += a.qn) {
+      a.qn = pass_queries(kind, Q - j);   // queries j .. j + qn - 1 of every sequence
+      a.q = static_cast<const char*>(q) + (size_t)j * qrow * elt;
+      a.q_pos = q_pos + j;
+      a.out = static_cast<char*>(out) + (size_t)j * qrow * elt;
+      a.lse = lse != nullptr ? lse + (size_t)j * a.H : nullptr;
+      cudaError_t e = kind == 3   ? palu::launch_decode_fused(a, st)
+                      : kind == 2 ? palu::launch_decode_tc(a, st)
+                                  : palu::launch_decode_simt(a, st);
+      if (e != cudaSuccess) return cuda_status(e);
+      e = palu::launch_combine(a, st);
+      if (e != cudaSuccess) return cuda_status(e);
+    }
+  }
+  return PALU_OK;
 }
 
 }  // namespace
@@ -155,23 +432,40 @@ uint64_t palu_kernel_launches(void) { return palu::g_launches.load(std::memory_o
 
 palu_status palu_cache_strides(const palu_config* cfg, size_t* k_page_bytes, size_t* v_page_bytes,
                                size_t* k_scale_page_bytes, size_t* v_scale_page_bytes) {
-  palu_status s = check_config(cfg);
+  return palu_cache_strides_ranked(cfg, nullptr, nullptr, k_page_bytes, v_page_bytes, k_scale_page_bytes,
+                                   v_scale_page_bytes, nullptr, nullptr);
+}
+
+palu_status palu_cache_strides_ranked(const palu_config* cfg, const int32_t* ranks_k, const int32_t* ranks_v,
+                                      size_t* k_page_bytes, size_t* v_page_bytes, size_t* k_scale_page_bytes,
+                                      size_t* v_scale_page_bytes, size_t* k_group_offsets,
+                                      size_t* v_group_offsets) {
+  Layer L;
+  palu_status s = make_layer(cfg, ranks_k, ranks_v, &L);
   if (s != PALU_OK) return s;
-  const int G = cfg->num_heads / cfg->group_size;
-  const size_t per = (size_t)G * cfg->page_size;
-  if (k_page_bytes) *k_page_bytes = per * palu::latent_row_bytes(cfg->latent_dtype, cfg->rank_k);
-  if (v_page_bytes) *v_page_bytes = per * palu::latent_row_bytes(cfg->latent_dtype, cfg->rank_v);
-  if (k_scale_page_bytes) *k_scale_page_bytes = per * palu::scale_row_bytes(cfg->latent_dtype, cfg->rank_k);
-  if (v_scale_page_bytes) *v_scale_page_bytes = per * palu::scale_row_bytes(cfg->latent_dtype, cfg->rank_v);
+  if (k_page_bytes) *k_page_bytes = (size_t)L.k_page;
+  if (v_page_bytes) *v_page_bytes = (size_t)L.v_page;
+  if (k_scale_page_bytes) *k_scale_page_bytes = (size_t)L.ks_page;
+  if (v_scale_page_bytes) *v_scale_page_bytes = (size_t)L.vs_page;
+  for (int g = 0; g < L.G; ++g) {
+    if (k_group_offsets) k_group_offsets[g] = (size_t)L.k_off[g];
+    if (v_group_offsets) v_group_offsets[g] = (size_t)L.v_off[g];
+  }
   return PALU_OK;
 }
 
 palu_status palu_compress_workspace_size(const palu_config* cfg, int n_tokens, int d_model,
                                          size_t* bytes) {
-  palu_status s = check_config(cfg);
+  return palu_compress_ranked_workspace_size(cfg, nullptr, nullptr, n_tokens, d_model, bytes);
+}
+
+palu_status palu_compress_ranked_workspace_size(const palu_config* cfg, const int32_t* ranks_k,
+                                                const int32_t* ranks_v, int n_tokens, int d_model, size_t* bytes) {
+  Layer L;
+  palu_status s = make_layer(cfg, ranks_k, ranks_v, &L);
   if (s != PALU_OK) return s;
   if (bytes == nullptr || n_tokens < 0 || d_model <= 0) return PALU_ERR_INVALID_ARG;
-  *bytes = kStatusBytes + palu::tc_compress_scratch_bytes(cfg, n_tokens, d_model);
+  *bytes = compress_workspace(L, n_tokens, d_model);
   return PALU_OK;
 }
 
@@ -180,56 +474,22 @@ palu_status palu_compress_append(const palu_config* cfg, int n_tokens, int d_mod
                                  const int32_t* positions, void* zk_pool, void* zv_pool,
                                  void* zk_scales, void* zv_scales, int32_t* pos_pool, int num_pages,
                                  void* workspace, size_t workspace_bytes, palu_stream_t stream) {
-  palu_status s = check_config(cfg);
-  if (s != PALU_OK) return s;
-  if (n_tokens < 0 || d_model <= 0 || num_pages < 0) return PALU_ERR_INVALID_ARG;
-  if (d_model % 64 != 0) return PALU_ERR_UNSUPPORTED;
-  size_t need = 0;
-  palu_compress_workspace_size(cfg, n_tokens, d_model, &need);
-  if (workspace == nullptr || workspace_bytes < need) return PALU_ERR_WORKSPACE;
-  if (n_tokens == 0) return PALU_OK;
-  if (!x || !A_k || !A_v || !slot_mapping || !zk_pool || !zv_pool) return PALU_ERR_INVALID_ARG;
-  const bool int4 = cfg->latent_dtype == PALU_INT4;
-  if (int4 && (!zk_scales || !zv_scales)) return PALU_ERR_INVALID_ARG;
-  if (!aligned16(x) || !aligned16(A_k) || !aligned16(A_v) || !aligned16(zk_pool) ||
-      !aligned16(zv_pool) || (int4 && (!aligned16(zk_scales) || !aligned16(zv_scales))) ||
-      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
-    return PALU_ERR_ALIGNMENT;
+  return palu_compress_append_ranked(cfg, nullptr, nullptr, n_tokens, d_model, x, A_k, A_v, slot_mapping, positions,
+                                     zk_pool, zv_pool, zk_scales, zv_scales, pos_pool, num_pages, workspace,
+                                     workspace_bytes, stream);
+}
 
-  palu::CompressArgs a{};
-  a.n = n_tokens;
-  a.d_model = d_model;
-  a.G = cfg->num_heads / cfg->group_size;
-  a.r_k = cfg->rank_k;
-  a.r_v = cfg->rank_v;
-  a.P = cfg->page_size;
-  a.num_pages = num_pages;
-  a.act = cfg->act_dtype;
-  a.lat = cfg->latent_dtype;
-  a.x = x;
-  a.Ak = A_k;
-  a.Av = A_v;
-  a.slots = slot_mapping;
-  a.positions = positions;
-  a.zk = zk_pool;
-  a.zv = zv_pool;
-  a.zks = zk_scales;
-  a.zvs = zv_scales;
-  a.pos_pool = pos_pool;
-  a.status = workspace;
-  a.scratch = reinterpret_cast<float*>(static_cast<char*>(workspace) + kStatusBytes);
-  a.scratch_bytes = workspace_bytes - kStatusBytes;
-  a.k_row = palu::latent_row_bytes(a.lat, a.r_k);
-  a.v_row = palu::latent_row_bytes(a.lat, a.r_v);
-  a.ks_row = palu::scale_row_bytes(a.lat, a.r_k);
-  a.vs_row = palu::scale_row_bytes(a.lat, a.r_v);
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e;
-  if (palu::tc_compress_supported(cfg, n_tokens, d_model))
-    e = palu::launch_compress_tc(a, st);
-  else
-    e = palu::launch_compress_simt(a, st);
-  return cuda_status(e);
+palu_status palu_compress_append_ranked(const palu_config* cfg, const int32_t* ranks_k, const int32_t* ranks_v,
+                                        int n_tokens, int d_model, const void* x, const void* A_k, const void* A_v,
+                                        const int32_t* slot_mapping, const int32_t* positions, void* zk_pool,
+                                        void* zv_pool, void* zk_scales, void* zv_scales, int32_t* pos_pool,
+                                        int num_pages, void* workspace, size_t workspace_bytes,
+                                        palu_stream_t stream) {
+  Layer L;
+  palu_status s = make_layer(cfg, ranks_k, ranks_v, &L);
+  if (s != PALU_OK) return s;
+  return compress_layer(L, n_tokens, d_model, x, A_k, A_v, slot_mapping, positions, zk_pool, zv_pool, zk_scales,
+                        zv_scales, pos_pool, num_pages, workspace, workspace_bytes, stream);
 }
 
 palu_status palu_decode_num_splits(const palu_config* cfg, int batch, int max_pages, int* num_splits) {
@@ -242,111 +502,27 @@ palu_status palu_decode_num_splits(const palu_config* cfg, int batch, int max_pa
 
 palu_status palu_decode_workspace_size(const palu_config* cfg, int batch, int max_pages,
                                        int num_splits, size_t* bytes) {
-  return palu_decode_multi_workspace_size(cfg, batch, 1, max_pages, num_splits, bytes);
+  return palu_decode_ranked_workspace_size(cfg, nullptr, nullptr, batch, 1, max_pages, num_splits, bytes);
 }
 
-}  // extern "C"
+palu_status palu_decode_multi_workspace_size(const palu_config* cfg, int batch, int num_queries, int max_pages,
+                                             int num_splits, size_t* bytes) {
+  return palu_decode_ranked_workspace_size(cfg, nullptr, nullptr, batch, num_queries, max_pages, num_splits,
+                                           bytes);
+}
 
-namespace {
-
-// One decode step for Q queries per sequence (Q = 1: palu_decode_attn).  The
-// queries run one after another on the stream, each through the split kernel
-// and the combine, sharing the workspace; with Q > 1 a query attends only to
-// the tokens at or before its own position.
-palu_status decode_steps(const palu_config* cfg, int batch, int Q, const void* q, const int32_t* q_pos,
-                         const void* zk_pool, const void* zv_pool, const void* zk_scales,
-                         const void* zv_scales, const int32_t* pos_pool, const int32_t* page_table,
-                         int max_pages, const int32_t* seq_lens, int num_pages, const void* B_k,
-                         const void* B_v, void* out, float* lse, void* workspace, size_t workspace_bytes,
-                         int num_splits, palu_stream_t stream) {
-  palu_status s = check_config(cfg);
+palu_status palu_decode_ranked_workspace_size(const palu_config* cfg, const int32_t* ranks_k,
+                                              const int32_t* ranks_v, int batch, int num_queries, int max_pages,
+                                              int num_splits, size_t* bytes) {
+  Layer L;
+  palu_status s = make_layer(cfg, ranks_k, ranks_v, &L);
   if (s != PALU_OK) return s;
-  if (batch < 0 || max_pages <= 0 || num_pages < 0 || num_splits < 0 || Q < 1 || Q > kMaxQueries)
+  if (bytes == nullptr || batch < 0 || max_pages <= 0 || num_splits < 0 || num_queries < 1 ||
+      num_queries > kMaxQueries)
     return PALU_ERR_INVALID_ARG;
-  const int kind = kernel_kind(cfg);
-  const int S = run_S(cfg, kind, batch, max_pages, num_splits);
-  if (S > max_pages) return PALU_ERR_INVALID_ARG;
-  size_t fused_off = 0;
-  const size_t need = workspace_layout(cfg, kind, batch * pass_queries(kind, Q), S, &fused_off);
-  if (workspace == nullptr || workspace_bytes < need) return PALU_ERR_WORKSPACE;
-  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return PALU_ERR_ALIGNMENT;
-  if (batch == 0) return PALU_OK;
-  if (!q || !q_pos || !zk_pool || !zv_pool || !page_table || !seq_lens || !B_k || !B_v || !out)
-    return PALU_ERR_INVALID_ARG;
-  const bool int4 = cfg->latent_dtype == PALU_INT4;
-  if (int4 && (!zk_scales || !zv_scales)) return PALU_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(zk_pool) || !aligned16(zv_pool) || !aligned16(B_k) ||
-      !aligned16(B_v) || (int4 && (!aligned16(zk_scales) || !aligned16(zv_scales))))
-    return PALU_ERR_ALIGNMENT;
-
-  palu::DecodeArgs a{};
-  a.H = cfg->num_heads;
-  a.d_h = cfg->head_dim;
-  a.gs = cfg->group_size;
-  a.G = cfg->num_heads / cfg->group_size;
-  a.W = cfg->group_size * cfg->head_dim;
-  a.r_k = cfg->rank_k;
-  a.r_v = cfg->rank_v;
-  a.P = cfg->page_size;
-  a.batch = batch;
-  a.max_pages = max_pages;
-  a.num_pages = num_pages;
-  a.S = S;
-  a.act = cfg->act_dtype;
-  a.lat = cfg->latent_dtype;
-  a.rope = cfg->rope_base != 0.f;
-  a.sm_scale = (float)(1.0 / sqrt((double)cfg->head_dim));
-  a.q = q;
-  a.q_pos = q_pos;
-  a.zk = zk_pool;
-  a.zv = zv_pool;
-  a.zks = zk_scales;
-  a.zvs = zv_scales;
-  a.pos_pool = pos_pool;
-  a.page_table = page_table;
-  a.seq_lens = seq_lens;
-  a.Bk = B_k;
-  a.Bv = B_v;
-  a.out = out;
-  a.lse = lse;
-  a.status = workspace;
-  a.part = reinterpret_cast<float*>(static_cast<char*>(workspace) + kStatusBytes);
-  a.fused_q = static_cast<char*>(workspace) + fused_off;
-  a.k_row = palu::latent_row_bytes(a.lat, a.r_k);
-  a.v_row = palu::latent_row_bytes(a.lat, a.r_v);
-  a.ks_row = palu::scale_row_bytes(a.lat, a.r_k);
-  a.vs_row = palu::scale_row_bytes(a.lat, a.r_v);
-  fill_omega(cfg, a.omega);
-
-  const long long qrow = (long long)a.H * a.d_h;       // one query's elements per sequence
-  const size_t elt = cfg->act_dtype == PALU_F32 ? 4 : 2;
-  if (Q > 1 && (qrow * (long long)elt) % 16 != 0) return PALU_ERR_ALIGNMENT;
-  a.q_bstride = Q * qrow;
-  a.o_bstride = Q * qrow;
-  a.qpos_bstride = Q;
-  a.lse_bstride = Q * a.H;
-  a.causal = Q > 1;
-
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  for (int j = 0; j < Q; j += a.qn) {
-    a.qn = pass_queries(kind, Q - j);   // queries j .. j + qn - 1 of every sequence
-    a.q = static_cast<const char*>(q) + (size_t)j * qrow * elt;
-    a.q_pos = q_pos + j;
-    a.out = static_cast<char*>(out) + (size_t)j * qrow * elt;
-    a.lse = lse != nullptr ? lse + (size_t)j * a.H : nullptr;
-    cudaError_t e = kind == 3   ? palu::launch_decode_fused(a, st)
-                    : kind == 2 ? palu::launch_decode_tc(a, st)
-                                : palu::launch_decode_simt(a, st);
-    if (e != cudaSuccess) return cuda_status(e);
-    e = palu::launch_combine(a, st);
-    if (e != cudaSuccess) return cuda_status(e);
-  }
+  *bytes = decode_workspace(L, batch, num_queries, max_pages, num_splits, nullptr);
   return PALU_OK;
 }
-
-}  // namespace
-
-extern "C" {
 
 palu_status palu_decode_attn(const palu_config* cfg, int batch, const void* q, const int32_t* q_pos,
                              const void* zk_pool, const void* zv_pool, const void* zk_scales,
@@ -355,22 +531,9 @@ palu_status palu_decode_attn(const palu_config* cfg, int batch, const void* q, c
                              int num_pages, const void* B_k, const void* B_v, void* out, float* lse,
                              void* workspace, size_t workspace_bytes, int num_splits,
                              palu_stream_t stream) {
-  return decode_steps(cfg, batch, 1, q, q_pos, zk_pool, zv_pool, zk_scales, zv_scales, pos_pool, page_table,
-                      max_pages, seq_lens, num_pages, B_k, B_v, out, lse, workspace, workspace_bytes, num_splits,
-                      stream);
-}
-
-palu_status palu_decode_multi_workspace_size(const palu_config* cfg, int batch, int num_queries, int max_pages,
-                                             int num_splits, size_t* bytes) {
-  palu_status s = check_config(cfg);
-  if (s != PALU_OK) return s;
-  if (bytes == nullptr || batch < 0 || max_pages <= 0 || num_splits < 0 || num_queries < 1 ||
-      num_queries > kMaxQueries)
-    return PALU_ERR_INVALID_ARG;
-  const int kind = kernel_kind(cfg);
-  const int S = run_S(cfg, kind, batch, max_pages, num_splits);
-  *bytes = workspace_layout(cfg, kind, batch * pass_queries(kind, num_queries), S, nullptr);
-  return PALU_OK;
+  return palu_decode_attn_ranked(cfg, nullptr, nullptr, batch, 1, q, q_pos, zk_pool, zv_pool, zk_scales, zv_scales,
+                                 pos_pool, page_table, max_pages, seq_lens, num_pages, B_k, B_v, out, lse, workspace,
+                                 workspace_bytes, num_splits, stream);
 }
 
 palu_status palu_decode_attn_multi(const palu_config* cfg, int batch, int num_queries, const void* q,
@@ -380,7 +543,22 @@ palu_status palu_decode_attn_multi(const palu_config* cfg, int batch, int num_qu
                                    int num_pages, const void* B_k, const void* B_v, void* out, float* lse,
                                    void* workspace, size_t workspace_bytes, int num_splits,
                                    palu_stream_t stream) {
-  return decode_steps(cfg, batch, num_queries, q, q_pos, zk_pool, zv_pool, zk_scales, zv_scales, pos_pool,
+  return palu_decode_attn_ranked(cfg, nullptr, nullptr, batch, num_queries, q, q_pos, zk_pool, zv_pool, zk_scales,
+                                 zv_scales, pos_pool, page_table, max_pages, seq_lens, num_pages, B_k, B_v, out, lse,
+                                 workspace, workspace_bytes, num_splits, stream);
+}
+
+palu_status palu_decode_attn_ranked(const palu_config* cfg, const int32_t* ranks_k, const int32_t* ranks_v,
+                                    int batch, int num_queries, const void* q, const int32_t* q_pos,
+                                    const void* zk_pool, const void* zv_pool, const void* zk_scales,
+                                    const void* zv_scales, const int32_t* pos_pool, const int32_t* page_table,
+                                    int max_pages, const int32_t* seq_lens, int num_pages, const void* B_k,
+                                    const void* B_v, void* out, float* lse, void* workspace,
+                                    size_t workspace_bytes, int num_splits, palu_stream_t stream) {
+  Layer L;
+  palu_status s = make_layer(cfg, ranks_k, ranks_v, &L);
+  if (s != PALU_OK) return s;
+  return decode_layer(L, batch, num_queries, q, q_pos, zk_pool, zv_pool, zk_scales, zv_scales, pos_pool,
                       page_table, max_pages, seq_lens, num_pages, B_k, B_v, out, lse, workspace, workspace_bytes,
                       num_splits, stream);
 }

@@ -11,6 +11,24 @@
 namespace palu {
 
 constexpr int kMaxHalfDim = 64;  // head_dim <= 128
+constexpr int kMaxGroups = 64;   // head groups per layer
+
+// Where the head groups a launch covers keep their latents.  All groups of a
+// launch share one rank pair (r_k, r_v); a layer whose groups have different
+// ranks runs one launch per rank pair.  With one pool for all groups (equal
+// ranks), group g's block of page pg starts at pool + (pg·G + g)·P·row; with a
+// pool per group, at pool_g + pg·P·row_g.  Either way: base[g] + pg·page.
+struct GroupMap {
+  int n;                                // groups this launch covers
+  int g[kMaxGroups];                    // model group of entry i (heads g·gs .. g·gs + gs − 1)
+  const uint8_t* zk[kMaxGroups];        // per model group: block of page 0
+  const uint8_t* zv[kMaxGroups];
+  const uint8_t* zks[kMaxGroups];       // int4 scale rows (NULL otherwise)
+  const uint8_t* zvs[kMaxGroups];
+  long long k_page, v_page, ks_page, vs_page;   // bytes from one page's block to the next
+  int k_row0[kMaxGroups];               // first row of the group in B_k (= first column in A_k)
+  int v_row0[kMaxGroups];               // same for B_v / A_v
+};
 
 // Everything a decode launch needs, already validated.
 struct DecodeArgs {
@@ -29,19 +47,17 @@ struct DecodeArgs {
   int causal;          // 1: a token counts only if its position <= the query's position
   int qn;              // queries of each sequence this launch serves (the fused kernel takes
                        // several per pass; their partials sit at virtual sequence b·qn + j)
-  const void* zk;
-  const void* zv;
-  const void* zks;
-  const void* zvs;
+  GroupMap gm;
   const int32_t* pos_pool;
   const int32_t* page_table;
   const int32_t* seq_lens;
-  const void* Bk;
-  const void* Bv;
+  const void* Bk;      // [bk_rows][W]: group entry i's rows start at gm.k_row0[i]
+  const void* Bv;      // [bv_rows][W]
+  int bk_rows, bv_rows;
   void* out;
   float* lse;
-  float* part;         // [batch][H][S][r_v + 2] float32
-  void* fused_q;       // fused (no-RoPE) path: folded queries [batch][G][2·gs][r_k], act dtype
+  float* part;         // [batch·qn][gm.n·gs][S][r_v + 2] float32, heads in group-map order
+  void* fused_q;       // fused (no-RoPE) path: folded queries [batch·qn][gm.n][8][r_k], act dtype
   void* status;        // DevStatus*
   long long k_row, v_row, ks_row, vs_row;  // bytes per latent / scale row
   uint64_t omega[kMaxHalfDim];             // RoPE frequencies as 64-bit fixed-point turns
@@ -65,10 +81,8 @@ struct CompressArgs {
   const void* Av;
   const int32_t* slots;
   const int32_t* positions;
-  void* zk;
-  void* zv;
-  void* zks;
-  void* zvs;
+  GroupMap gm;         // the groups of this launch; A column offsets in k_row0 / v_row0
+  long long a_kcols, a_vcols;   // columns of A_k / A_v (row strides in elements)
   int32_t* pos_pool;
   void* status;
   float* scratch;  // workspace past the status header

@@ -171,3 +171,69 @@ def test_multi_query_workspace():
     assert P.palu_decode_multi_workspace_size(r, 16, 8, 128, 4) == P.palu_decode_workspace_size(r, 16, 128, 4)
     with pytest.raises(P.PaluError):
         P.palu_decode_multi_workspace_size(c, 16, P.MAX_QUERIES + 1, 128, 4)
+
+
+def test_ranked_layout_equal_ranks_is_uniform():
+    # one rank pair for every group: the ranked layout is the uniform one, byte for byte
+    c = cfg()
+    kb, vb, ksb, vsb, ko, vo = P.palu_cache_strides_ranked(c, [256] * 8, [128] * 8)
+    assert (kb, vb, ksb, vsb) == P.palu_cache_strides(c)
+    assert ko == [g * 128 * 512 for g in range(8)] and vo == [g * 128 * 256 for g in range(8)]
+    assert P.palu_cache_strides_ranked(c, None, None)[:4] == P.palu_cache_strides(c)
+    for Q in (1, 3):
+        assert P.palu_decode_ranked_workspace_size(c, [256] * 8, [128] * 8, 16, Q, 128, 0) == \
+            P.palu_decode_multi_workspace_size(c, 16, Q, 128, 0)
+    assert P.palu_compress_ranked_workspace_size(c, [256] * 8, [128] * 8, 64, 4096) == \
+        P.palu_compress_workspace_size(c, 64, 4096)
+
+
+def test_ranked_layout_offsets_are_prefix_sums():
+    c = cfg(num_heads=16)
+    rk, rv = [64, 384, 128, 256], [128, 64, 256, 128]
+    kb, vb, ksb, vsb, ko, vo = P.palu_cache_strides_ranked(c, rk, rv)
+    assert kb == 128 * 2 * sum(rk) and vb == 128 * 2 * sum(rv) and ksb == vsb == 0
+    assert ko == [128 * 2 * sum(rk[:g]) for g in range(4)]
+    assert vo == [128 * 2 * sum(rv[:g]) for g in range(4)]
+    ci = cfg(num_heads=16, act_dtype="f16", latent_dtype="int4")
+    kb, vb, ksb, vsb, ko, vo = P.palu_cache_strides_ranked(ci, [256, 512, 256, 512], [256] * 4)
+    assert ko == [0, 128 * 128, 128 * 384, 128 * 512] and kb == 128 * 768
+    srow = lambda r: (2 * (r // 32) + 15) // 16 * 16
+    assert ksb == 128 * sum(srow(r) for r in [256, 512, 256, 512])
+
+
+def test_ranked_argument_checks():
+    lib = load()
+    c = cfg(num_heads=16)
+    arr = lambda v: (ctypes.c_int32 * 4)(*v)
+    k = ctypes.c_size_t()
+    # a rank that breaks the row rule, one rank array without the other
+    assert lib.palu_cache_strides_ranked(ctypes.byref(c), arr([256, 100, 256, 256]), arr([128] * 4),
+                                         ctypes.byref(k), None, None, None, None, None) == 3
+    assert lib.palu_cache_strides_ranked(ctypes.byref(c), arr([256] * 4), None, ctypes.byref(k), None, None,
+                                         None, None, None) == 1
+    assert lib.palu_cache_strides_ranked(ctypes.byref(c), arr([256, 1024, 256, 256]), arr([128] * 4),
+                                         ctypes.byref(k), None, None, None, None, None) == 2
+    # decode: too small a workspace, unaligned workspace
+    ws = P.palu_decode_ranked_workspace_size(c, [256, 128, 384, 128], [128, 256, 128, 128], 2, 1, 8, 0)
+    p = ctypes.c_void_p(4096)
+    call = lambda wsp, nbytes: lib.palu_decode_attn_ranked(
+        ctypes.byref(c), arr([256, 128, 384, 128]), arr([128, 256, 128, 128]), 2, 1, p, p, p, p, None, None,
+        None, p, 8, p, 8, p, p, p, None, wsp, nbytes, 0, None)
+    assert call(p, ws - 1) == 4                                  # PALU_ERR_WORKSPACE
+    assert call(ctypes.c_void_p(4096 + 16), ws) == 3             # PALU_ERR_ALIGNMENT
+    # compress: d_model not a multiple of 64
+    assert lib.palu_compress_append_ranked(ctypes.byref(c), arr([256] * 4), arr([128] * 4), 4, 100, None,
+                                           None, None, None, None, None, None, None, None, None, 8, p, 1 << 20,
+                                           None) == 2
+
+
+def test_ranked_workspace_covers_every_class():
+    # the classes run one after another and share the workspace: it is as large
+    # as the largest class's, which is at least the largest single group's need
+    c = cfg(num_heads=16)
+    rk, rv = [256, 128, 384, 128], [128, 256, 128, 128]
+    ws = P.palu_decode_ranked_workspace_size(c, rk, rv, 16, 1, 128, 4)
+    for r_k, r_v in zip(rk, rv):
+        one = cfg(num_heads=4, rank_k=r_k, rank_v=r_v)        # one group of this class
+        assert ws >= P.palu_decode_workspace_size(one, 16, 128, 4)
+    assert ws == 256 + 16 * 4 * 4 * 258 * 4                  # partials of class (128, 256): 4 heads

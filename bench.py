@@ -166,24 +166,27 @@ class ClockSampler:
 
 # ----------------------------------------------------------------- work accounting
 def step_work(w, seq_lens):
-    """Algorithmic bytes and flops of one decode call (latents + B + q/out), per the layout."""
-    from rank_kv_cache_palu_b200.api import DTYPE_CODE  # noqa: F401
+    """Algorithmic bytes and flops of one decode call (latents + B + q/out), per the layout.
+
+    Sums over the head groups, each with its own (r_k, r_v) (all equal unless the
+    workload carries a rank-search output)."""
     elt = {"f32": 4, "f16": 2, "bf16": 2}[w.act_dtype]
-    G, W, gs = w.groups, w.width, w.group_size
-    if w.latent_dtype == "int4":
-        row = w.rank_k // 2 + w.rank_v // 2 + 2 * (w.rank_k // 32 + w.rank_v // 32)
-    else:
-        row = (w.rank_k + w.rank_v) * {"f32": 4, "f16": 2, "bf16": 2}[w.latent_dtype]
+    W, gs, d_h = w.width, w.group_size, w.head_dim
     tok = sum(seq_lens)
-    bytes_ = tok * G * row + G * (w.rank_k + w.rank_v) * W * elt \
-        + len(seq_lens) * w.num_heads * w.head_dim * elt * 2
-    if w.rope_base == 0:
-        # fused path: scores in latent space (q̃ = B_k q per head, r_k long)
-        flops = tok * G * (2 * gs * w.rank_k + 2 * gs * w.rank_v) \
-            + len(seq_lens) * w.num_heads * 2 * (w.rank_k + w.rank_v) * w.head_dim
-    else:
-        flops = tok * G * (2 * w.rank_k * W + 2 * gs * w.rank_v) \
-            + len(seq_lens) * w.num_heads * 2 * w.rank_v * w.head_dim
+    nb = len(seq_lens)
+    bytes_ = nb * w.num_heads * d_h * elt * 2
+    flops = 0
+    for rk, rv in zip(*w.group_ranks):
+        if w.latent_dtype == "int4":
+            row = rk // 2 + rv // 2 + 2 * (rk // 32 + rv // 32)
+        else:
+            row = (rk + rv) * {"f32": 4, "f16": 2, "bf16": 2}[w.latent_dtype]
+        bytes_ += tok * row + (rk + rv) * W * elt
+        if w.rope_base == 0:
+            # fused path: scores in latent space (q̃ = B_k q per head, r_k long)
+            flops += tok * (2 * gs * rk + 2 * gs * rv) + nb * gs * 2 * (rk + rv) * d_h
+        else:
+            flops += tok * (2 * rk * W + 2 * gs * rv) + nb * gs * 2 * rv * d_h
     return bytes_, flops
 
 
@@ -203,24 +206,44 @@ def oracle_sample(w, seconds: float, seed: int = 99):
     except Exception:
         threads = os.cpu_count() or 1
     T, G, W = w.context, w.groups, w.width
-    rk, rv = w.rank_k, w.rank_v
-    zk = normal(seed, "cpu_zk", (G, T, rk)).astype(np.float64)
-    zv = normal(seed, "cpu_zv", (G, T, rv)).astype(np.float64)
-    Bk = normal(seed, "cpu_Bk", (G, rk, W), 1 / math.sqrt(rk)).astype(np.float64)
-    Bv = normal(seed, "cpu_Bv", (G, rv, W), 1 / math.sqrt(rv)).astype(np.float64)
     q = normal(seed, "cpu_q", (w.num_heads, w.head_dim)).astype(np.float64)
     pos = np.arange(T)
     heads = 0
     t0 = time.perf_counter()
-    while True:
-        h = heads % w.num_heads
-        O.decode_attention_head(h, q, T - 1, zk, zv, pos, Bk, Bv, w.group_size, w.rope_base)
-        heads += 1
-        el = time.perf_counter() - t0
-        if el >= seconds:
-            break
-    desc = (f"oracle decode_attention_head on {heads} (sequence, head) units of one sequence "
-            f"at context {T} ({el:.1f} s of CPU work)")
+    if not w.ranked:
+        rk, rv = w.rank_k, w.rank_v
+        zk = normal(seed, "cpu_zk", (G, T, rk)).astype(np.float64)
+        zv = normal(seed, "cpu_zv", (G, T, rv)).astype(np.float64)
+        Bk = normal(seed, "cpu_Bk", (G, rk, W), 1 / math.sqrt(rk)).astype(np.float64)
+        Bv = normal(seed, "cpu_Bv", (G, rv, W), 1 / math.sqrt(rv)).astype(np.float64)
+        t0 = time.perf_counter()
+        while True:
+            h = heads % w.num_heads
+            O.decode_attention_head(h, q, T - 1, zk, zv, pos, Bk, Bv, w.group_size, w.rope_base)
+            heads += 1
+            el = time.perf_counter() - t0
+            if el >= seconds:
+                break
+        what = "decode_attention_head on %d (sequence, head) units" % heads
+    else:
+        # one group (its group_size heads) per call, each with its own ranks
+        rks, rvs = w.group_ranks
+        gs = w.group_size
+        zk = [normal(seed, f"cpu_zk{g}", (T, r)).astype(np.float64) for g, r in enumerate(rks)]
+        zv = [normal(seed, f"cpu_zv{g}", (T, r)).astype(np.float64) for g, r in enumerate(rvs)]
+        Bk = [normal(seed, f"cpu_Bk{g}", (r, W), 1 / math.sqrt(r)).astype(np.float64) for g, r in enumerate(rks)]
+        Bv = [normal(seed, f"cpu_Bv{g}", (r, W), 1 / math.sqrt(r)).astype(np.float64) for g, r in enumerate(rvs)]
+        t0 = time.perf_counter()
+        while True:
+            g = (heads // gs) % G
+            O.decode_attention_ranked(q[g * gs:(g + 1) * gs][None], [T - 1], [zk[g]], [zv[g]], pos, [Bk[g]],
+                                      [Bv[g]], gs, w.rope_base)
+            heads += gs
+            el = time.perf_counter() - t0
+            if el >= seconds:
+                break
+        what = "decode_attention_ranked, one group per call, on %d (sequence, head) units" % heads
+    desc = f"oracle {what} of one sequence at context {T} ({el:.1f} s of CPU work)"
     return heads * T / el, desc, threads, heads * T
 
 
@@ -287,8 +310,10 @@ def run_ours(args):
     act = TORCH_DTYPE[w.act_dtype]
 
     # ---- the latent cache, filled with N(0,1) latents (the distribution of x·A)
-    cache = P.LatentCache.allocate(cfg, num_pages, device=dev)
-    for pool, lat_bytes in ((cache.zk, w.rank_k), (cache.zv, w.rank_v)):
+    rks, rvs = w.group_ranks
+    rk_arg, rv_arg = (rks, rvs) if w.ranked else (None, None)
+    cache = P.LatentCache.allocate(cfg, num_pages, device=dev, ranks_k=rk_arg, ranks_v=rv_arg)
+    for pool in (cache.zk, cache.zv):
         if w.latent_dtype == "int4":
             pool.copy_(torch.randint(0, 256, pool.shape, dtype=torch.uint8, device=dev, generator=gen))
         else:
@@ -305,13 +330,14 @@ def run_ours(args):
     pt_host = page_table.cpu().numpy()
 
     d_model = w.d_model
-    A_k = (torch.randn((d_model, G * w.rank_k), device=dev, generator=gen) / math.sqrt(d_model)).to(act)
-    A_v = (torch.randn((d_model, G * w.rank_v), device=dev, generator=gen) / math.sqrt(d_model)).to(act)
-    B_k = (torch.randn((G, w.rank_k, W), device=dev, generator=gen) / math.sqrt(w.rank_k)).to(act)
-    B_v = (torch.randn((G, w.rank_v, W), device=dev, generator=gen) / math.sqrt(w.rank_v)).to(act)
+    # A_k [d_model][Σ r_k], B_k [Σ r_k][W]: group g's columns / rows follow the groups before it
+    A_k = (torch.randn((d_model, sum(rks)), device=dev, generator=gen) / math.sqrt(d_model)).to(act)
+    A_v = (torch.randn((d_model, sum(rvs)), device=dev, generator=gen) / math.sqrt(d_model)).to(act)
+    B_k = torch.cat([torch.randn((r, W), device=dev, generator=gen) / math.sqrt(r) for r in rks]).to(act)
+    B_v = torch.cat([torch.randn((r, W), device=dev, generator=gen) / math.sqrt(r) for r in rvs]).to(act)
     ring = 4
     xs = [torch.randn((b * Q, d_model), device=dev, generator=gen).to(act) for _ in range(ring)]
-    qshape = (b, w.num_heads, w.head_dim) if Q == 1 else (b, Q, w.num_heads, w.head_dim)
+    qshape = (b, w.num_heads, w.head_dim) if Q == 1 and not w.ranked else (b, Q, w.num_heads, w.head_dim)
     qs = [torch.randn(qshape, device=dev, generator=gen).to(act) for _ in range(ring)]
 
     # per-step metadata, all on the device before timing: the step appends Q
@@ -329,22 +355,41 @@ def run_ours(args):
         base = T0 + s * Q
         return b * w.num_heads * sum(base + j + 1 for j in range(Q))
 
-    S = args.num_splits or P.palu_decode_num_splits(cfg, b, max_pages)
-    ws_d = torch.zeros(P.palu_decode_multi_workspace_size(cfg, b, Q, max_pages, S), dtype=torch.uint8,
-                       device=dev)
-    ws_c = torch.zeros(P.palu_compress_workspace_size(cfg, b * Q, d_model), dtype=torch.uint8, device=dev)
+    if w.ranked:
+        # one split count per rank class, chosen by the library (0 = automatic)
+        S = args.num_splits
+        ws_d = torch.zeros(P.palu_decode_ranked_workspace_size(cfg, rks, rvs, b, Q, max_pages, S),
+                           dtype=torch.uint8, device=dev)
+        ws_c = torch.zeros(P.palu_compress_ranked_workspace_size(cfg, rks, rvs, b * Q, d_model),
+                           dtype=torch.uint8, device=dev)
+    else:
+        S = args.num_splits or P.palu_decode_num_splits(cfg, b, max_pages)
+        ws_d = torch.zeros(P.palu_decode_multi_workspace_size(cfg, b, Q, max_pages, S), dtype=torch.uint8,
+                           device=dev)
+        ws_c = torch.zeros(P.palu_compress_workspace_size(cfg, b * Q, d_model), dtype=torch.uint8, device=dev)
     out = torch.empty(qshape, dtype=act, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     def decode(q, qpos, lens):
+        if w.ranked:
+            P.palu_decode_attn_ranked(cfg, rks, rvs, q, qpos, cache.zk, cache.zv, cache.zks, cache.zvs, None,
+                                      page_table, lens, num_pages, B_k, B_v, out, None, ws_d, S, stream)
+            return
         fn = P.palu_decode_attn if Q == 1 else P.palu_decode_attn_multi
         fn(cfg, q, qpos, cache.zk, cache.zv, cache.zks, cache.zvs, None, page_table, lens, num_pages, B_k, B_v,
            out, None, ws_d, S, stream)
 
+    def compress(x, slots):
+        if w.ranked:
+            P.palu_compress_append_ranked(cfg, rks, rvs, x, A_k, A_v, slots, None, cache.zk, cache.zv, cache.zks,
+                                          cache.zvs, None, num_pages, ws_c, stream)
+        else:
+            P.palu_compress_append(cfg, x, A_k, A_v, slots, None, cache.zk, cache.zv, cache.zks, cache.zvs, None,
+                                   num_pages, ws_c, stream)
+
     def step(s, x=None, q=None):
         slots, qpos, lens = metas[s]
-        P.palu_compress_append(cfg, xs[s % ring] if x is None else x, A_k, A_v, slots, None,
-                               cache.zk, cache.zv, cache.zks, cache.zvs, None, num_pages, ws_c, stream)
+        compress(xs[s % ring] if x is None else x, slots)
         decode(qs[s % ring] if q is None else q, qpos, lens)
 
     # ---- device-resident timing
@@ -365,8 +410,7 @@ def run_ours(args):
         for k in range(args.steps):
             slots, qpos, lens = metas[s_idx]
             ev[k][0].record(stream)
-            P.palu_compress_append(cfg, xs[s_idx % ring], A_k, A_v, slots, None, cache.zk, cache.zv,
-                                   cache.zks, cache.zvs, None, num_pages, ws_c, stream)
+            compress(xs[s_idx % ring], slots)
             ev[k][1].record(stream)
             decode(qs[s_idx % ring], qpos, lens)
             ev[k][2].record(stream)
@@ -401,8 +445,7 @@ def run_ours(args):
         q_d.copy_(qh[s % ring], non_blocking=True)
         for dst, src in zip(m_d, meta_h[s]):
             dst.copy_(src, non_blocking=True)
-        P.palu_compress_append(cfg, x_d, A_k, A_v, m_d[0], None, cache.zk, cache.zv, cache.zks,
-                               cache.zvs, None, num_pages, ws_c, stream)
+        compress(x_d, m_d[0])
         decode(q_d, m_d[1], m_d[2])
         outh.copy_(out, non_blocking=True)
 
@@ -426,7 +469,7 @@ def run_ours(args):
     # ---- prefill: palu_compress_append of a prompt (x·A for n tokens into fresh pages)
     prefill = None
     n_pre = args.prefill if args.prefill is not None else (8192 if w.name == "7b_bf16_r256_b32_t16k" else 0)
-    if n_pre > 0 and world >= 1:
+    if n_pre > 0 and world >= 1 and not w.ranked:
         pre_pages = (n_pre + Pz - 1) // Pz
         pcache = P.LatentCache.allocate(cfg, pre_pages, device=dev)
         xp = torch.randn((n_pre, d_model), device=dev, generator=gen).to(act)
@@ -468,7 +511,10 @@ def run_ours(args):
     tfs = dflops / dec_avg_s / 1e12
     t_hbm = dbytes / (peaks["hbm_gbs"] * 1e9)
     t_tc = dflops / (peaks["bf16_tflops_sustained"] * 1e12)
-    kind = P.palu_decode_kernel_kind(cfg)
+    kinds = sorted({P.palu_decode_kernel_kind(P.make_config(w.num_heads, w.head_dim, w.group_size, rk, rv, Pz,
+                                                             w.rope_base, w.act_dtype, w.latent_dtype))
+                    for rk, rv in zip(rks, rvs)})
+    kind = kinds[0] if len(kinds) == 1 else kinds
     if t_tc > t_hbm:
         roof = {"bound": "tensor", "achieved": tfs, "peak": peaks["bf16_tflops_sustained"],
                 "unit": "TFLOP/s", "frac": tfs / peaks["bf16_tflops_sustained"]}
@@ -482,8 +528,9 @@ def run_ours(args):
     roof["tensor_achieved_tflops"] = tfs
     roof["algorithmic_bytes_per_launch"] = dbytes
     roof["algorithmic_flops_per_launch"] = dflops
-    roof["kernel"] = "palu_decode_attn (%s), kernel kind %d" % (
-        "fold-query + fused split + combine" if kind == 3 else "split + combine", kind)
+    roof["kernel"] = "palu_decode_attn (%s), kernel kind %s%s" % (
+        "fold-query + fused split + combine" if kind == 3 else "split + combine", kind,
+        ", one launch set per rank class (%d classes)" % len(set(zip(rks, rvs))) if w.ranked else "")
     roof["avg_launch_ms"] = dec_avg_s * 1e3
 
     line = {
@@ -495,7 +542,9 @@ def run_ours(args):
                    "context_at_first_timed_step": T0 + first_step + 1, "heads": w.num_heads,
                    "head_dim": w.head_dim, "group_size": w.group_size, "rank_k": w.rank_k,
                    "rank_v": w.rank_v, "latent_dtype": w.latent_dtype, "page_size": Pz,
-                   "num_splits": S, "decode_kernel_kind": kind, "queries_per_step": Q,
+                   "num_splits": S if S else "automatic per rank class", "decode_kernel_kind": kind,
+                   "queries_per_step": Q,
+                   **({"ranks_k": list(rks), "ranks_v": list(rvs)} if w.ranked else {}),
                    "l2": "inputs larger than L2 (latent cache %.2f GB vs 126 MB L2)" %
                          ((cache.zk.numel() + cache.zv.numel()) / 1e9),
                    "parallelism": f"dp{world} replicas (independent sequences per GPU)"},

@@ -263,15 +263,23 @@ class LatentCache:
     zks: torch.Tensor | None
     zvs: torch.Tensor | None
     pos: torch.Tensor | None
+    ranks_k: tuple | None = None     # per-group ranks (None: the config's for every group)
+    ranks_v: tuple | None = None
 
     @classmethod
     def allocate(cls, cfg: PaluConfig, num_pages: int, device="cuda", with_positions=False,
-                 fill=None) -> "LatentCache":
-        kb, vb, ksb, vsb = palu_cache_strides(cfg)
+                 fill=None, ranks_k=None, ranks_v=None) -> "LatentCache":
+        """Pools for num_pages pages; with ranks_k / ranks_v, the layout of a layer whose
+        groups carry their own ranks (each page holds every group's block back to back)."""
+        if ranks_k is None:
+            kb, vb, ksb, vsb = palu_cache_strides(cfg)
+        else:
+            kb, vb, ksb, vsb, _, _ = palu_cache_strides_ranked(cfg, ranks_k, ranks_v)
         mk = (lambda n: torch.empty(n, dtype=torch.uint8, device=device)) if fill is None else \
             (lambda n: torch.full((n,), fill, dtype=torch.uint8, device=device))
         zks = mk(num_pages * ksb) if ksb else None
         zvs = mk(num_pages * vsb) if vsb else None
         pos = torch.zeros(num_pages * cfg.page_size, dtype=torch.int32, device=device) \
             if with_positions else None
-        return cls(cfg, num_pages, mk(num_pages * kb), mk(num_pages * vb), zks, zvs, pos)
+        return cls(cfg, num_pages, mk(num_pages * kb), mk(num_pages * vb), zks, zvs, pos,
+                   None if ranks_k is None else tuple(ranks_k), None if ranks_v is None else tuple(ranks_v))

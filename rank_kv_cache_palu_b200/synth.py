@@ -91,11 +91,25 @@ class Workload:
     page_size: int = 128
     d_model: int = 4096
     seed: int = 0
+    # per-group ranks (a rank-search output); empty = rank_k / rank_v for every group
+    ranks_k: tuple = ()
+    ranks_v: tuple = ()
     notes: str = field(default="", compare=False)
 
     @property
     def groups(self) -> int:
         return self.num_heads // self.group_size
+
+    @property
+    def ranked(self) -> bool:
+        return bool(self.ranks_k)
+
+    @property
+    def group_ranks(self) -> tuple[tuple, tuple]:
+        """(key ranks, value ranks) of every group."""
+        if self.ranks_k:
+            return tuple(self.ranks_k), tuple(self.ranks_v)
+        return (self.rank_k,) * self.groups, (self.rank_v,) * self.groups
 
     @property
     def width(self) -> int:
@@ -133,5 +147,16 @@ WORKLOADS = {
         _w("7b_bf16_r256v128_b16_t16k_norope", num_heads=32, head_dim=128, group_size=4,
            rank_k=256, rank_v=128, batch=16, context=16384, act_dtype="bf16",
            latent_dtype="bf16", rope_base=0.0, seed=6),
+        # a rank-search output: the 8 groups keep different key / value ranks
+        # (mean key rank 208, value ranks 128 and 256), all on the tcgen05 path;
+        # rank_k / rank_v name the largest
+        _w("7b_bf16_ranked_b16_t16k", num_heads=32, head_dim=128, group_size=4, rank_k=256,
+           rank_v=256, batch=16, context=16384, act_dtype="bf16", latent_dtype="bf16", seed=7,
+           ranks_k=(128, 192, 256, 256, 128, 192, 256, 256),
+           ranks_v=(128, 128, 128, 256, 128, 128, 128, 256)),
+        _w("7b_bf16_ranked_b16_t16k_norope", num_heads=32, head_dim=128, group_size=4, rank_k=320,
+           rank_v=256, batch=16, context=16384, act_dtype="bf16", latent_dtype="bf16", rope_base=0.0,
+           seed=8, ranks_k=(128, 192, 256, 320, 128, 192, 256, 192),
+           ranks_v=(128, 128, 128, 256, 128, 128, 128, 256)),
     ]
 }

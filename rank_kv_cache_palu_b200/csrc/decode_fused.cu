@@ -96,6 +96,7 @@ __global__ void __launch_bounds__(256) fold_query_kernel(const __grid_constant__
   // blockIdx.x: entry gi of the group map (model group g)
   const int gi = blockIdx.x, jb = blockIdx.y, v0 = blockIdx.z * kFoldSeqs;
   const int g = a.gm.g[gi];
+  const int r_k = a.gm.rk[gi];          // this entry's key rank; rows are a.r_k apart
   const int gs = a.gs, d_h = a.d_h;
   const int nvb = a.batch * qslots;
   auto live = [&](int vb) { return vb < nvb && vb % qslots < a.qn; };
@@ -112,7 +113,7 @@ __global__ void __launch_bounds__(256) fold_query_kernel(const __grid_constant__
   __syncthreads();
   const int jl = threadIdx.x >> 2, h = threadIdx.x & 3;
   const int j = jb * 64 + jl;
-  if (j >= a.r_k) return;
+  if (j >= r_k) return;
   // the row segment as 8-element vectors (d_h is a multiple of 8 here)
   uint4 bseg[16];
   const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const TA*>(a.Bk) +
@@ -158,7 +159,7 @@ __host__ __device__ inline Smem smem_layout(int r_k) {
   using PS = Pass<QN>;
   Smem s{};
   uint32_t o = 0;
-  s.qt = o;   o += (uint32_t)(r_k / kChunk) * PS::kN * 128;   // [K chunk][kN rows][128 B], 128-byte swizzle
+  // fixed offsets first; the folded queries (their size follows the key rank) last
   s.zk = o;   o += kNZK * kStageBytes;
   s.zv = o;   o += kNZV * kStageBytes;
   s.p = o;    o += 2 * PS::kPBytes;
@@ -167,6 +168,8 @@ __host__ __device__ inline Smem smem_layout(int r_k) {
   s.bars = o; o += 32 * 8;
   s.tmem_slot = o; o += 16;
   s.abort = o;     o += 16;
+  o = (o + 1023u) & ~1023u;                             // 128-byte-swizzle atoms: 1024-byte aligned
+  s.qt = o;   o += (uint32_t)(r_k / kChunk) * PS::kN * 128;   // [K chunk][kN rows][128 B], 128-byte swizzle
   s.total = o;
   return s;
 }
@@ -188,18 +191,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* sbase = smem_raw + (base - raw);
-  const Smem L = smem_layout<QN>(a.r_k);
+  // blockIdx.y: entry gi of the group map (model group gm.g[gi]); its key rank sets the layout
+  const int s = blockIdx.x, gi = blockIdx.y, b = blockIdx.z;
+  const GroupMap& gm = a.gm;
+  const int r_k = gm.rk[gi];
+  const Smem L = smem_layout<QN>(r_k);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   DevStatus* st = reinterpret_cast<DevStatus*>(a.status);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sbase + L.abort);
   auto bar = [&](int i) { return base + L.bars + 8u * i; };
 
-  // blockIdx.y: entry gi of the group map (model group gm.g[gi])
-  const int s = blockIdx.x, gi = blockIdx.y, b = blockIdx.z;
-  const GroupMap& gm = a.gm;
   const int gs = a.gs;
   const int nq = a.qn;                  // queries of this pass (<= QN)
-  const int nkc = a.r_k / kChunk;
+  const int nkc = r_k / kChunk;
   int T = a.seq_lens[b];
   const int cap = a.max_pages * a.P;
   if (T < 0 || T > cap) {
@@ -245,11 +249,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   for (int i = threadIdx.x; i < nkc * kN * 32; i += kThreads) reinterpret_cast<uint32_t*>(sbase + L.qt)[i] = 0u;
   __syncthreads();
   // q̃ into the K-major swizzled B operand: row n = 8·jj + r of query jj, entry j
-  for (int i = threadIdx.x; i < nq * 2 * kMaxG * a.r_k; i += kThreads) {
-    const int n = i / a.r_k, j = i % a.r_k;
+  for (int i = threadIdx.x; i < nq * 2 * kMaxG * r_k; i += kThreads) {
+    const int n = i / r_k, j = i % r_k;
     const int jj = n >> 3, r = n & 7;
     const uint16_t* src = reinterpret_cast<const uint16_t*>(qt) +
-                          ((((size_t)b * QN + jj) * gm.n + gi) * 2 * kMaxG + r) * a.r_k;
+                          ((((size_t)b * QN + jj) * gm.n + gi) * 2 * kMaxG + r) * a.r_k;   // rows a.r_k apart
     const int c = j / kChunk, kin = j % kChunk;
     *reinterpret_cast<uint16_t*>(sbase + L.qt + c * (kN * 128) + n * 128 + (((kin >> 3) ^ (n & 7)) << 4) +
                                  (kin & 7) * 2) = src[j];

@@ -53,12 +53,14 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const __grid_constant__
   const int tid = threadIdx.x;
   const int gi = hl / a.gs, jh = hl % a.gs;
   const int h = a.gm.g[gi] * a.gs + jh;   // model head
+  const int r_k = a.gm.rk[gi];            // this group's key rank (<= a.r_k)
+  const long long ks_row = (2 * (r_k / 32) + 15) / 16 * 16;   // int4 scale row bytes of this group
   const int d_h = a.d_h, half = d_h / 2;
   DevStatus* st = reinterpret_cast<DevStatus*>(a.status);
 
   float* qr = smem;                       // [d_h] rotated, scaled query
   float* zk_t = qr + d_h;                 // [kTT][r_k]
-  float* zv_t = zk_t + kTT * a.r_k;       // [kTT][r_v]
+  float* zv_t = zk_t + kTT * r_k;         // [kTT][r_v]
   float* kt = zv_t + kTT * a.r_v;         // [kTT][d_h]
   float* sc = kt + kTT * d_h;             // [kTT] scores
   int* tpos = reinterpret_cast<int*>(sc + kTT);  // [kTT] positions
@@ -104,8 +106,8 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const __grid_constant__
       }
       tpos[tid] = pv;
     }
-    for (int e = tid; e < kTT * a.r_k; e += kThreads) {
-      const int tt = e / a.r_k, j = e % a.r_k;
+    for (int e = tid; e < kTT * r_k; e += kThreads) {
+      const int tt = e / r_k, j = e % r_k;
       float v = 0.f;
       if (tt < nt) {
         const int t = t0 + tt;
@@ -115,7 +117,7 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const __grid_constant__
         } else {
           v = load_latent<LAT, ACT>(zk_base + (size_t)page * a.gm.k_page, t % a.P, a.P,
                                     LAT == PALU_INT4 ? zks_base + (size_t)page * a.gm.ks_page +
-                                                           (size_t)(t % a.P) * a.ks_row
+                                                           (size_t)(t % a.P) * ks_row
                                                      : nullptr,
                                     j);
         }
@@ -144,10 +146,10 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const __grid_constant__
       float acc[kTT];
 #pragma unroll
       for (int tt = 0; tt < kTT; ++tt) acc[tt] = 0.f;
-      for (int r = 0; r < a.r_k; ++r) {
+      for (int r = 0; r < r_k; ++r) {
         const float bv = Dt<ACT>::to_f(Bk[(size_t)r * a.W + d]);
 #pragma unroll
-        for (int tt = 0; tt < kTT; ++tt) acc[tt] = fmaf(zk_t[tt * a.r_k + r], bv, acc[tt]);
+        for (int tt = 0; tt < kTT; ++tt) acc[tt] = fmaf(zk_t[tt * r_k + r], bv, acc[tt]);
       }
 #pragma unroll
       for (int tt = 0; tt < kTT; ++tt) kt[tt * d_h + d] = acc[tt];

@@ -60,10 +60,11 @@ struct Smem {
 
 constexpr int kVRawBytes = 128 * 128 + 128 * 16;   // int4: one page of value codes + its scale rows
 
+// Every region but B_k (whose size follows the key rank) sits at a fixed offset,
+// so the kernel's offsets are compile-time constants; B_k comes last.
 __host__ __device__ inline Smem smem_layout(int r_k, bool int4) {
   Smem s{};
   uint32_t o = 0;
-  s.b = o;      o += (uint32_t)r_k * 256 * 2;          // B_k for 2 heads
   s.zk = o;     o += zk_stages(int4) * kZkBytes;
   s.zv = o;     o += kNVS * kZvBytes;
   s.vraw = o;   o += int4 ? kVRawBytes : 0;
@@ -77,6 +78,8 @@ __host__ __device__ inline Smem smem_layout(int r_k, bool int4) {
   s.bars = o;   o += 32 * 8;
   s.tmem_slot = o; o += 16;
   s.abort = o;  o += 16;
+  o = (o + 1023u) & ~1023u;                              // 128-byte-swizzle atoms: 1024-byte aligned
+  s.b = o;      o += (uint32_t)r_k * 256 * 2;            // B_k for 2 heads
   s.total = o;
   return s;
 }
@@ -243,7 +246,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* sbase = smem_raw + (base - raw);
-  const Smem L = smem_layout(a.r_k, LAT == PALU_INT4);
+  // blockIdx.y: entry gi of the group map and head pair hp; the entry's key rank sets the layout
+  const int gi = blockIdx.y / (a.gs / 2), hp = blockIdx.y % (a.gs / 2);
+  const int r_k = a.gm.rk[gi];
+  const Smem L = smem_layout(r_k, LAT == PALU_INT4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr bool kInt4 = LAT == PALU_INT4;
   constexpr int kNZK = zk_stages(kInt4);
@@ -253,10 +259,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar = [&](int i) { return base + L.bars + 8u * i; };
 
   const int b = blockIdx.z;
-  const int nhp = a.gs / 2;                         // head pairs per group
-  const int gi = blockIdx.y / nhp, hp = blockIdx.y % nhp;   // entry gi of the group map
   const GroupMap& gm = a.gm;
-  const int nkc = a.r_k / kChunk;
+  const int nkc = r_k / kChunk;
+  const uint32_t k_blk_bytes = (uint32_t)a.P * (kInt4 ? r_k / 2 : 2 * r_k);   // this entry's block of a page
   const TileRange tr = tile_range(a, b, st, threadIdx.x == 0);
   const long long t_start = clock64();
   auto trace = [&](int ev, int k) {
@@ -307,9 +312,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sbase + L.tmem_slot);
 
   if (warp == 0 && lane == 0) {
-    mbar_expect_tx(bar(BAR_B), (uint32_t)a.r_k * 256 * 2);
+    mbar_expect_tx(bar(BAR_B), (uint32_t)r_k * 256 * 2);
+    // 64-column blocks of B_k (MN-major, 128-byte swizzle), each in boxes of bk_box rows
     for (int nb = 0; nb < 4; ++nb)
-      tma_load_2d(base + L.b + (uint32_t)nb * a.r_k * 128, &tm_bk, hp * 256 + nb * 64, gm.k_row0[gi], bar(BAR_B));
+      for (int rb = 0; rb < r_k; rb += a.bk_box)
+        tma_load_2d(base + L.b + (uint32_t)nb * r_k * 128 + rb * 128, &tm_bk, hp * 256 + nb * 64,
+                    gm.k_row0[gi] + rb, bar(BAR_B));
   }
   if (kInt4 && (warp == 0 || warp == 3)) {
     // ============================================================ int4 key codes (warps 0, 3)
@@ -335,7 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = (k == 0 ? 1 : k + kPrefetch); kk <= k + kPrefetch && kk < tr.ntiles; ++kk) {
           const int ppg = page_of(a, b, tr.t_begin / kTile + kk);
           if (ppg < 0) continue;
-          prefetch_l2(gm.zk[gi] + (size_t)ppg * gm.k_page, (uint32_t)(a.P * a.k_row));
+          prefetch_l2(gm.zk[gi] + (size_t)ppg * gm.k_page, k_blk_bytes);
           prefetch_l2(gm.zks[gi] + (size_t)ppg * gm.ks_page, (uint32_t)(a.P * a.ks_row));
           prefetch_l2(gm.zv[gi] + (size_t)ppg * gm.v_page, (uint32_t)(a.P * a.v_row));
           prefetch_l2(gm.zvs[gi] + (size_t)ppg * gm.vs_page, (uint32_t)(a.P * a.vs_row));
@@ -447,7 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (kk >= tr.ntiles) return;
         const int ppg = page_of(a, b, tr.t_begin / kTile + kk);
         if (ppg < 0) return;
-        prefetch_l2(gm.zk[gi] + (size_t)ppg * gm.k_page, (uint32_t)(a.P * a.k_row));
+        prefetch_l2(gm.zk[gi] + (size_t)ppg * gm.k_page, k_blk_bytes);
         if (!(tr.ragged_last && kk == tr.ntiles - 1))
           prefetch_l2(gm.zv[gi] + (size_t)ppg * gm.v_page, (uint32_t)(a.P * a.v_row));
       };
@@ -501,7 +509,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr int kBf = ACT == PALU_BF16 ? 1 : 0;
       const uint32_t idesc_d = idesc_f16(kBf, 0, 1, 256, 128);    // z_k K-major, B_k MN-major
       const uint32_t idesc_pv = idesc_f16(kBf, 1, 0, 16, 128);    // z_vᵀ MN-major, Pᵀ K-major
-      const uint32_t b_lbo = (uint32_t)a.r_k * 128;                // bytes between 64-column blocks of B
+      const uint32_t b_lbo = (uint32_t)r_k * 128;                  // bytes between 64-column blocks of B
       int zs = 0;
       uint32_t zph = 0, vph = 0;
       bool ok = mbar_wait(bar(BAR_B), 0, abort_flag, st, 20);
@@ -908,7 +916,8 @@ template <int ACT, int NRV, int LAT>
 cudaError_t launch_t(const DecodeArgs& a, cudaStream_t st) {
   const CUtensorMapDataType dt = ACT == PALU_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   CUtensorMap tm_bk;
-  if (!make_map_2d(&tm_bk, a.Bk, dt, 2, a.W, (uint64_t)a.bk_rows, (uint64_t)a.W * 2, 64, a.r_k,
+  if (a.bk_box <= 0 || a.bk_box > 256 || a.bk_box % 64 != 0) return cudaErrorInvalidValue;
+  if (!make_map_2d(&tm_bk, a.Bk, dt, 2, a.W, (uint64_t)a.bk_rows, (uint64_t)a.W * 2, 64, a.bk_box,
                    CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   const Smem L = smem_layout(a.r_k, LAT == PALU_INT4);

@@ -119,7 +119,9 @@ int run_S(const palu_config* c, int kind, int batch, int max_pages, int num_spli
 // B_k stacks the groups' [r_k,g × W] blocks, so group g's rows start at
 // Σ_{g'<g} r_k,g', and A_k's columns follow the same order.  With one rank pair
 // this is the layout pool[page][g][P rows].  Groups with equal rank pairs form
-// a class, which one launch of each kernel serves.
+// a class, which one launch of the compress kernel serves.  The decode kernels
+// take a key rank per group: one launch serves every group with the same value
+// rank and kernel family (a decode set).
 struct Layer {
   palu_config cfg;   // model shape and dtypes (rank fields: see rk / rv)
   int G;
@@ -132,6 +134,9 @@ struct Layer {
   int nclass;
   int cls[palu::kMaxGroups];                    // class of each group
   int crk[palu::kMaxGroups], crv[palu::kMaxGroups], cn[palu::kMaxGroups];
+  int nset;
+  int dset[palu::kMaxGroups];                   // decode set of each group
+  int srk[palu::kMaxGroups], srv[palu::kMaxGroups], sn[palu::kMaxGroups];   // max key rank, value rank, groups
 };
 
 palu_status make_layer(const palu_config* cfg, const int32_t* ranks_k, const int32_t* ranks_v, Layer* L) {
@@ -189,10 +194,36 @@ palu_status make_layer(const palu_config* cfg, const int32_t* ranks_k, const int
   L->vs_page = vso;
   L->bk_rows = kr;
   L->bv_rows = vr;
+  // decode sets: one value rank and one kernel family (the family's limits grow
+  // with the key rank, so the set's largest key rank is supported as well)
+  L->nset = 0;
+  for (int g = 0; g < G; ++g) {
+    palu_config c = *cfg;
+    c.rank_k = L->rk[g];
+    c.rank_v = L->rv[g];
+    const int kind = kernel_kind(&c);
+    int k = 0;
+    while (k < L->nset) {
+      palu_config d = *cfg;
+      d.rank_k = L->srk[k];
+      d.rank_v = L->srv[k];
+      if (L->srv[k] == c.rank_v && kernel_kind(&d) == kind) break;
+      ++k;
+    }
+    if (k == L->nset) {
+      L->srk[k] = c.rank_k;
+      L->srv[k] = c.rank_v;
+      L->sn[k] = 0;
+      ++L->nset;
+    }
+    if (c.rank_k > L->srk[k]) L->srk[k] = c.rank_k;
+    L->dset[g] = k;
+    ++L->sn[k];
+  }
   return PALU_OK;
 }
 
-// The config one class's launches see: its groups and its ranks.
+// The config one compress class's launch sees: its groups and its ranks.
 palu_config class_cfg(const Layer& L, int c) {
   palu_config x = L.cfg;
   x.num_heads = L.cn[c] * L.cfg.group_size;
@@ -201,8 +232,18 @@ palu_config class_cfg(const Layer& L, int c) {
   return x;
 }
 
-void class_map(const Layer& L, int c, const void* zk, const void* zv, const void* zks, const void* zvs,
-               palu::GroupMap& m) {
+// The config one decode set's launches see: its groups, its largest key rank, its value rank.
+palu_config set_cfg(const Layer& L, int k) {
+  palu_config x = L.cfg;
+  x.num_heads = L.sn[k] * L.cfg.group_size;
+  x.rank_k = L.srk[k];
+  x.rank_v = L.srv[k];
+  return x;
+}
+
+// Group map of the groups g with part[g] == c (compress class or decode set).
+void build_map(const Layer& L, const int* part, int c, const void* zk, const void* zv, const void* zks,
+               const void* zvs, palu::GroupMap& m) {
   auto at = [](const void* pool, long long off) {
     return pool == nullptr ? nullptr : static_cast<const uint8_t*>(pool) + off;
   };
@@ -212,7 +253,7 @@ void class_map(const Layer& L, int c, const void* zk, const void* zv, const void
   m.ks_page = L.ks_page;
   m.vs_page = L.vs_page;
   for (int g = 0; g < L.G; ++g) {
-    if (L.cls[g] != c) continue;
+    if (part[g] != c) continue;
     const int i = m.n++;
     m.g[i] = g;
     m.zk[i] = at(zk, L.k_off[g]);
@@ -221,17 +262,18 @@ void class_map(const Layer& L, int c, const void* zk, const void* zv, const void
     m.zvs[i] = at(zvs, L.vs_off[g]);
     m.k_row0[i] = L.k_row0[g];
     m.v_row0[i] = L.v_row0[g];
+    m.rk[i] = L.rk[g];
   }
 }
 
-// Decode workspace: the status word, then the partials of the largest class
-// ([vb][heads][S][r_v + 2] float32, vb = sequence × query slot of a pass),
-// then the folded queries of the largest fused-kernel class.  Classes run one
-// after another on the stream, so they share both regions.
+// Decode workspace: the status word, then the partials of the largest decode
+// set ([vb][heads][S][r_v + 2] float32, vb = sequence × query slot of a pass),
+// then the folded queries of the largest fused-kernel set.  Sets run one after
+// another on the stream, so they share both regions.
 size_t decode_workspace(const Layer& L, int batch, int Q, int max_pages, int num_splits, size_t* fused_off) {
   size_t part = 0, fq = 0;
-  for (int c = 0; c < L.nclass; ++c) {
-    const palu_config cc = class_cfg(L, c);
+  for (int c = 0; c < L.nset; ++c) {
+    const palu_config cc = set_cfg(L, c);
     const int kind = kernel_kind(&cc);
     const int S = run_S(&cc, kind, batch, max_pages, num_splits);
     const int vb = batch * pass_queries(kind, Q);
@@ -300,7 +342,7 @@ palu_status compress_layer(const Layer& L, int n_tokens, int d_model, const void
     a.v_row = palu::latent_row_bytes(a.lat, a.r_v);
     a.ks_row = palu::scale_row_bytes(a.lat, a.r_k);
     a.vs_row = palu::scale_row_bytes(a.lat, a.r_v);
-    class_map(L, c, zk_pool, zv_pool, zk_scales, zv_scales, a.gm);
+    build_map(L, L.cls, c, zk_pool, zv_pool, zk_scales, zv_scales, a.gm);
     a.positions = c == 0 ? positions : nullptr;   // once per token
     const cudaError_t e = palu::tc_compress_supported(&cc, n_tokens, d_model) ? palu::launch_compress_tc(a, st)
                                                                              : palu::launch_compress_simt(a, st);
@@ -310,8 +352,8 @@ palu_status compress_layer(const Layer& L, int n_tokens, int d_model, const void
 }
 
 // One decode step for Q queries per sequence (Q = 1: palu_decode_attn).  Each
-// rank class runs its split kernel and combine over its own groups; within a
-// class, passes of queries run one after another on the stream, sharing the
+// decode set runs its split kernel and combine over its own groups; within a
+// set, passes of queries run one after another on the stream, sharing the
 // workspace.  With Q > 1 a query attends only to the tokens at or before its
 // own position.
 palu_status decode_layer(const Layer& L, int batch, int Q, const void* q, const int32_t* q_pos,
@@ -372,8 +414,8 @@ palu_status decode_layer(const Layer& L, int batch, int Q, const void* q, const 
   a.causal = Q > 1;
 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  for (int c = 0; c < L.nclass; ++c) {
-    const palu_config cc = class_cfg(L, c);
+  for (int c = 0; c < L.nset; ++c) {
+    const palu_config cc = set_cfg(L, c);
     const int kind = kernel_kind(&cc);
     a.S = run_S(&cc, kind, batch, max_pages, num_splits);
     a.r_k = cc.rank_k;
@@ -382,7 +424,10 @@ palu_status decode_layer(const Layer& L, int batch, int Q, const void* q, const 
     a.v_row = palu::latent_row_bytes(a.lat, a.r_v);
     a.ks_row = palu::scale_row_bytes(a.lat, a.r_k);
     a.vs_row = palu::scale_row_bytes(a.lat, a.r_v);
-    class_map(L, c, zk_pool, zv_pool, zk_scales, zv_scales, a.gm);
+    build_map(L, L.dset, c, zk_pool, zv_pool, zk_scales, zv_scales, a.gm);
+    a.bk_box = a.r_k;
+    for (int i = 0; i < a.gm.n; ++i)
+      if (a.gm.rk[i] != a.r_k) a.bk_box = 64;   // mixed key ranks: boxes of 64 rows
     for (int j = 0; j < Q; j += a.qn) {
       a.qn = pass_queries(kind, Q - j);   // queries j .. j + qn - 1 of every sequence
       a.q = static_cast<const char*>(q) + (size_t)j * qrow * elt;

@@ -28,6 +28,8 @@ struct GroupMap {
   long long k_page, v_page, ks_page, vs_page;   // bytes from one page's block to the next
   int k_row0[kMaxGroups];               // first row of the group in B_k (= first column in A_k)
   int v_row0[kMaxGroups];               // same for B_v / A_v
+  int rk[kMaxGroups];                   // key rank of the entry (decode launches may mix key ranks;
+                                        // the launch's r_k is their maximum, r_v is shared)
 };
 
 // Everything a decode launch needs, already validated.
@@ -54,6 +56,7 @@ struct DecodeArgs {
   const void* Bk;      // [bk_rows][W]: group entry i's rows start at gm.k_row0[i]
   const void* Bv;      // [bv_rows][W]
   int bk_rows, bv_rows;
+  int bk_box;          // rows per tensor-map box of B_k: the key rank when every entry has it, else 64
   void* out;
   float* lse;
   float* part;         // [batch·qn][gm.n·gs][S][r_v + 2] float32, heads in group-map order

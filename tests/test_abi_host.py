@@ -227,13 +227,16 @@ def test_ranked_argument_checks():
                                            None) == 2
 
 
-def test_ranked_workspace_covers_every_class():
-    # the classes run one after another and share the workspace: it is as large
-    # as the largest class's, which is at least the largest single group's need
+def test_ranked_workspace_covers_every_decode_set():
+    # decode launches group the heads by value rank and kernel family (key ranks
+    # may differ within one); the sets run one after another and share the
+    # workspace, which is as large as the largest set's
     c = cfg(num_heads=16)
     rk, rv = [256, 128, 384, 128], [128, 256, 128, 128]
     ws = P.palu_decode_ranked_workspace_size(c, rk, rv, 16, 1, 128, 4)
     for r_k, r_v in zip(rk, rv):
-        one = cfg(num_heads=4, rank_k=r_k, rank_v=r_v)        # one group of this class
+        one = cfg(num_heads=4, rank_k=r_k, rank_v=r_v)        # one group
         assert ws >= P.palu_decode_workspace_size(one, 16, 128, 4)
-    assert ws == 256 + 16 * 4 * 4 * 258 * 4                  # partials of class (128, 256): 4 heads
+    # set (r_v 128, tensor cores) = groups 0 and 3 (key ranks 256 and 128): 8 heads;
+    # group 2 (key rank 384) runs on the CUDA-core kernel, group 1 (r_v 256) alone
+    assert ws == 256 + 16 * 8 * 4 * 130 * 4

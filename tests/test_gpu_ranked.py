@@ -104,6 +104,9 @@ def test_ranked_int4():
     case = make_ranked_case(w, [256, 512, 256, 256], [256, 256, 512, 256], [520, 129])
     assert class_kinds(case) == {1, 2}
     check_ranked(case)
+    # groups 0 and 1 share a value rank on the CUDA-core kernel with key ranks 256 and 512
+    # (one launch; per-group scale rows)
+    check_ranked(make_ranked_case(w, [256, 512, 512, 256], [512, 512, 256, 256], [300, 77]))
 
 
 def test_ranked_equal_ranks_is_the_uniform_call():

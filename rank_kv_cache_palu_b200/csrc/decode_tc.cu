@@ -48,6 +48,8 @@ constexpr uint32_t kZkSwz = 2u;    // 128-byte swizzle
 constexpr uint32_t kZkSbo = 1024;  // bytes per 8-row swizzle atom
 constexpr int kNVS = 2;            // z_v ring stages
 constexpr int kPrefetch = 3;       // pages pulled into L2 ahead of the TMA loads
+constexpr int kBatch = 8;          // frequency pairs per TMEM round trip of the score pass
+constexpr int kNB = 32 / kBatch;   // score batches per warpgroup and tile
 constexpr int kThreads = 384;      // 12 warps: producers + MMA (warps 0-3), two epilogue warpgroups
 constexpr int kZkBytes = kTile * kChunk * 2;   // bytes per z_k stage
 constexpr int kZvBytes = 128 * 64 * 2;         // 16 KB: one 64-entry column block of a page (128 tokens)
@@ -676,24 +678,31 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) acc[hh][0] = acc[hh][1] = 0ull;
 #pragma unroll
-      for (int jj = 0; jj < 2; ++jj) {
-        if (jj == 1) mid();
-        const int i0 = wg * 32 + jj * 16;
+      for (int jj = 0; jj < kNB; ++jj) {
+        mid(jj);   // the previous tile's latent sums, folded as soon as they are in
+        const int i0 = wg * 32 + jj * kBatch;
         const uint32_t col = tmem + lane_addr + (uint32_t)slot * 256 + i0;
-        // both heads' keys of these 16 frequency pairs in one TMEM round trip
-        float lo[2][16], hi[2][16];
-        tmem_ld16(col, lo[0]);
-        tmem_ld16(col + 64, hi[0]);
-        tmem_ld16(col + 128, lo[1]);
-        tmem_ld16(col + 192, hi[1]);
+        // both heads' keys of these kBatch frequency pairs in one TMEM round trip
+        float lo[2][kBatch], hi[2][kBatch];
+        if constexpr (kBatch == 16) {
+          tmem_ld16(col, lo[0]);
+          tmem_ld16(col + 64, hi[0]);
+          tmem_ld16(col + 128, lo[1]);
+          tmem_ld16(col + 192, hi[1]);
+        } else {
+          tmem_ld8(col, lo[0]);
+          tmem_ld8(col + 64, hi[0]);
+          tmem_ld8(col + 128, lo[1]);
+          tmem_ld8(col + 192, hi[1]);
+        }
         tmem_wait_ld();
 #pragma unroll
-        for (int v4 = 0; v4 < 4; ++v4) {
+        for (int v4 = 0; v4 < kBatch / 4; ++v4) {
           float4 cb4 = make_float4(0.f, 0.f, 0.f, 0.f), sb4 = cb4, nb4 = cb4;
           if (contig) {
-            cb4 = reinterpret_cast<const float4*>(tbw + jj * 16)[v4];
-            sb4 = reinterpret_cast<const float4*>(tbw + 32 + jj * 16)[v4];
-            nb4 = reinterpret_cast<const float4*>(tbw + 64 + jj * 16)[v4];
+            cb4 = reinterpret_cast<const float4*>(tbw + jj * kBatch)[v4];
+            sb4 = reinterpret_cast<const float4*>(tbw + 32 + jj * kBatch)[v4];
+            nb4 = reinterpret_cast<const float4*>(tbw + 64 + jj * kBatch)[v4];
           }
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
@@ -704,8 +713,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               const f2 s0 = e ? f2_pack(sb4.z, sb4.w) : f2_pack(sb4.x, sb4.y);
               const f2 n0 = e ? f2_pack(nb4.z, nb4.w) : f2_pack(nb4.x, nb4.y);
               // cos(t0+row) = c0 cr - s0 sr ; sin(t0+row) = s0 cr + c0 sr
-              cs = f2_fma(c0, crow[jj * 8 + v], f2_mul(n0, srow[jj * 8 + v]));
-              sn = f2_fma(s0, crow[jj * 8 + v], f2_mul(c0, srow[jj * 8 + v]));
+              const int vr = jj * (kBatch / 2) + v;
+              cs = f2_fma(c0, crow[vr], f2_mul(n0, srow[vr]));
+              sn = f2_fma(s0, crow[vr], f2_mul(c0, srow[vr]));
             } else {
               // explicit positions: a sincos per token
               float c0, s0, c1, s1;
@@ -786,11 +796,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         // scores: its value MMA has had that long to finish, and its TMEM slot
         // (where the next key MMA goes) is released early enough for that MMA
         // to finish before the next tile's scores start.
-        bool folded = true;
-        half_scores(slot, t0, pos, part, [&] {
-          if (k >= 1) folded = fold_at(k - 1, prev_scale);
+        // Fold the previous tile's latent sums before the first score batch that
+        // finds them complete (lane 0 tests, the warp follows), and at the latest
+        // halfway through: that releases its TMEM slot for the next key MMA.
+        bool folded = k == 0, fold_ok = true;
+        half_scores(slot, t0, pos, part, [&](int jj) {
+          if (folded) return;
+          int ready = 1;
+          if (jj < kNB / 2) {
+            if (lane == 0) ready = mbar_test_wait(bar(BAR_AT_FULL), (k - 1) & 1) ? 1 : 0;
+            ready = __shfl_sync(0xffffffffu, ready, 0);
+          }
+          if (ready) {
+            fold_ok = fold_at(k - 1, prev_scale);
+            folded = true;
+          }
         });
-        if (!folded) { ok = false; break; }
+        if (!fold_ok) { ok = false; break; }
         tc_fence_before();
         psc[(slot * 2 + (1 - hw)) * 128 + row] = part[1 - hw];
         __syncwarp();

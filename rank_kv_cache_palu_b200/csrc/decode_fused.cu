@@ -92,7 +92,8 @@ constexpr int kFoldSeqs = 4;
 template <int ACT>
 __global__ void __launch_bounds__(256) fold_query_kernel(const __grid_constant__ DecodeArgs a, int qslots, void* qt) {
   using TA = typename Dt<ACT>::T;
-  __shared__ float qs[kFoldSeqs][kMaxG][128];
+  // rows padded by 4 floats: the four heads' 16-byte reads of one warp land in distinct banks
+  __shared__ __align__(16) float qs[kFoldSeqs][kMaxG][128 + 4];
   // blockIdx.x: entry gi of the group map (model group g)
   const int gi = blockIdx.x, jb = blockIdx.y, v0 = blockIdx.z * kFoldSeqs;
   const int g = a.gm.g[gi];
@@ -124,14 +125,22 @@ __global__ void __launch_bounds__(256) fold_query_kernel(const __grid_constant__
   const float sc = a.sm_scale * kLog2e;
   for (int bb = 0; bb < kFoldSeqs; ++bb) {
     if (!live(v0 + bb)) continue;
-    float acc = 0.f;
+    float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
     for (int v = 0; v < 16; ++v) {
       const TA* e = reinterpret_cast<const TA*>(&bseg[v]);
-#pragma unroll
-      for (int u = 0; u < 8; ++u) acc = fmaf(Dt<ACT>::to_f(e[u]), qs[bb][h][v * 8 + u], acc);
+      const float4 qa = *reinterpret_cast<const float4*>(&qs[bb][h][v * 8]);
+      const float4 qb = *reinterpret_cast<const float4*>(&qs[bb][h][v * 8 + 4]);
+      acc0 = fmaf(Dt<ACT>::to_f(e[0]), qa.x, acc0);
+      acc1 = fmaf(Dt<ACT>::to_f(e[1]), qa.y, acc1);
+      acc0 = fmaf(Dt<ACT>::to_f(e[2]), qa.z, acc0);
+      acc1 = fmaf(Dt<ACT>::to_f(e[3]), qa.w, acc1);
+      acc0 = fmaf(Dt<ACT>::to_f(e[4]), qb.x, acc0);
+      acc1 = fmaf(Dt<ACT>::to_f(e[5]), qb.y, acc1);
+      acc0 = fmaf(Dt<ACT>::to_f(e[6]), qb.z, acc0);
+      acc1 = fmaf(Dt<ACT>::to_f(e[7]), qb.w, acc1);
     }
-    acc *= sc;
+    float acc = (acc0 + acc1) * sc;
     const TA hi = Dt<ACT>::from_f(acc);
     const TA lo = Dt<ACT>::from_f(acc - Dt<ACT>::to_f(hi));
     TA* out = reinterpret_cast<TA*>(qt) + ((size_t)(v0 + bb) * a.gm.n + gi) * 2 * kMaxG * a.r_k;

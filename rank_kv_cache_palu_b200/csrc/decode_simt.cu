@@ -213,14 +213,35 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const __grid_constant__
 }
 
 // Log-sum-exp merge of the split partials, then the value up-projection
-// out_h = a_h · B_v[g][:, cols_h] (a GEMV per (sequence, head)).
+// out_h = a_h · B_v[g][:, cols_h] (a GEMV per (sequence, head)): 256 threads =
+// 64 output pairs × 4 interleaved quarters of the latent rows, two accumulator
+// chains each, summed across the quarters in shared memory.
+template <typename TA>
+struct Pair;
+template <> struct Pair<float> {
+  __device__ __forceinline__ static float2 load(const float* p) { return *reinterpret_cast<const float2*>(p); }
+};
+template <> struct Pair<__half> {
+  __device__ __forceinline__ static float2 load(const __half* p) {
+    return __half22float2(*reinterpret_cast<const __half2*>(p));
+  }
+};
+template <> struct Pair<__nv_bfloat16> {
+  __device__ __forceinline__ static float2 load(const __nv_bfloat16* p) {
+    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
+  }
+};
+
+constexpr int kCombineThreads = 256;   // 64 output pairs x 4 row quarters
+
 template <int ACT>
-__global__ void __launch_bounds__(kThreads) combine_kernel(const __grid_constant__ DecodeArgs a) {
+__global__ void __launch_bounds__(kCombineThreads) combine_kernel(const __grid_constant__ DecodeArgs a) {
   using TA = typename Dt<ACT>::T;
+  constexpr int kThreads = kCombineThreads;
   extern __shared__ float smem[];
   float* av = smem;             // [r_v]
   float* wgt = av + a.r_v;      // [S]
-  // virtual sequence vb = b·qn + j: query j of sequence b (qn = 1: one query per sequence)
+  float* red = wgt + a.S;       // [4][d_h] per-quarter outputs
   // blockIdx.x: head hl of this launch (entry hl / gs of the group map)
   const int hl = blockIdx.x, vb = blockIdx.y;
   const int b = vb / a.qn, jq = vb % a.qn;
@@ -256,9 +277,30 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const __grid_constant
   }
   __syncthreads();
   const TA* Bv = reinterpret_cast<const TA*>(a.Bv) + (size_t)a.gm.v_row0[gi] * a.W + jh * a.d_h;
+  const int dp = tid & 63, rq = tid >> 6;
+  const int d0 = 2 * dp;
+  if (d0 < a.d_h) {
+    float2 acc0 = make_float2(0.f, 0.f), acc1 = acc0;
+    int r = rq;
+    for (; r + 4 < a.r_v; r += 8) {
+      const float2 b0 = Pair<TA>::load(Bv + (size_t)r * a.W + d0);
+      const float2 b1 = Pair<TA>::load(Bv + (size_t)(r + 4) * a.W + d0);
+      acc0.x = fmaf(av[r], b0.x, acc0.x);
+      acc0.y = fmaf(av[r], b0.y, acc0.y);
+      acc1.x = fmaf(av[r + 4], b1.x, acc1.x);
+      acc1.y = fmaf(av[r + 4], b1.y, acc1.y);
+    }
+    if (r < a.r_v) {
+      const float2 b0 = Pair<TA>::load(Bv + (size_t)r * a.W + d0);
+      acc0.x = fmaf(av[r], b0.x, acc0.x);
+      acc0.y = fmaf(av[r], b0.y, acc0.y);
+    }
+    red[rq * a.d_h + d0] = acc0.x + acc1.x;
+    red[rq * a.d_h + d0 + 1] = acc0.y + acc1.y;
+  }
+  __syncthreads();
   for (int d = tid; d < a.d_h; d += kThreads) {
-    float o = 0.f;
-    for (int r = 0; r < a.r_v; ++r) o = fmaf(av[r], Dt<ACT>::to_f(Bv[(size_t)r * a.W + d]), o);
+    const float o = (red[d] + red[a.d_h + d]) + (red[2 * a.d_h + d] + red[3 * a.d_h + d]);
     out[d] = Dt<ACT>::from_f(o);
   }
   if (tid == 0 && a.lse != nullptr) a.lse[(size_t)b * a.lse_bstride + (size_t)jq * a.H + h] = M + logf(L);
@@ -290,11 +332,11 @@ cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t st) {
 }
 
 cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t st) {
-  const size_t smem = sizeof(float) * (a.r_v + a.S);
+  const size_t smem = sizeof(float) * (a.r_v + a.S + 4 * a.d_h);
   dim3 grid(a.gm.n * a.gs, a.batch * a.qn);
-  if (a.act == PALU_F32) combine_kernel<PALU_F32><<<grid, kThreads, smem, st>>>(a);
-  else if (a.act == PALU_F16) combine_kernel<PALU_F16><<<grid, kThreads, smem, st>>>(a);
-  else if (a.act == PALU_BF16) combine_kernel<PALU_BF16><<<grid, kThreads, smem, st>>>(a);
+  if (a.act == PALU_F32) combine_kernel<PALU_F32><<<grid, kCombineThreads, smem, st>>>(a);
+  else if (a.act == PALU_F16) combine_kernel<PALU_F16><<<grid, kCombineThreads, smem, st>>>(a);
+  else if (a.act == PALU_BF16) combine_kernel<PALU_BF16><<<grid, kCombineThreads, smem, st>>>(a);
   else return cudaErrorInvalidValue;
   count_launch();
   return cudaGetLastError();

@@ -88,16 +88,31 @@ int auto_splits(const palu_config* c, int batch, int max_pages, int kind) {
   const long long units = kind == 3   ? groups
                           : kind == 2 ? groups * palu::tc_head_blocks(c)
                                       : (long long)batch * c->num_heads;
-  // enough CTAs for ~4 waves of one CTA per SM, but never more splits than pages
-  long long S = (4LL * sms + units - 1) / units;
-  if (kind == 2) {
-    // whole waves: round the CTA count up to a multiple of the SM count when cheap
-    S = (S < 1) ? 1 : S;
+  if (units <= 0) return 1;
+  if (kind == 1) {
+    // CUDA-core kernel: enough CTAs for ~4 waves of one CTA per SM
+    long long S = (4LL * sms + units - 1) / units;
+    if (S > max_pages) S = max_pages;
+    return (int)(S < 1 ? 1 : S > 256 ? 256 : S);
   }
-  if (S > max_pages) S = max_pages;
-  if (S < 1) S = 1;
-  if (S > 256) S = 256;
-  return (int)S;
+  // Tensor-core kernels hold one CTA per SM and every CTA of a launch walks about
+  // the same number of pages, so the launch takes ceil(CTAs / SMs) rounds of
+  // (pages per split + a start-up of ~2 pages).  Take the split count that
+  // minimises that (the smallest on ties), sized for the longest possible
+  // sequence (max_pages).  At least one full round of CTAs when the pages allow.
+  long long S0 = (sms + units - 1) / units;
+  if (S0 > max_pages) S0 = max_pages;
+  if (S0 < 1) S0 = 1;
+  long long best_S = S0, best_t = -1;
+  for (long long S = S0; S <= max_pages && S <= 64; ++S) {
+    const long long rounds = (units * S + sms - 1) / sms;
+    const long long t = rounds * ((max_pages + S - 1) / S + 2);
+    if (best_t < 0 || t < best_t) {
+      best_t = t;
+      best_S = S;
+    }
+  }
+  return (int)best_S;
 }
 
 int kernel_kind(const palu_config* c) {

@@ -53,7 +53,9 @@ Plan make_plan(int n, int d_model, int G, int r_k, int r_v) {
   const int kst = d_model / kKStage;
   int ks = 1;
   if (p.ntt == 1) {
-    ks = (2 * 148 + tiles - 1) / tiles;
+    // an append (one token tile): split K so that every column tile streams A from
+    // its own SMs, all CTAs in one round (one CTA per SM)
+    ks = 148 / tiles;
     if (ks > kst / 2) ks = kst / 2;   // at least two stages per split
     if (ks > 16) ks = 16;
     if (ks < 1) ks = 1;

@@ -196,3 +196,79 @@ def test_ranked_compress_append(lat):
                 err = np.abs(val - ref)
                 # within one rounding step of bf16 (float32 accumulation may cross a tie)
                 assert np.all(err <= 2 ** -7 * np.abs(ref) + 1e-6 * np.abs(ref).max()), (side, g, float(err.max()))
+
+
+def ranked_full_size(w, context, units, seed=321):
+    """The ranked bench workload at full size on the GPU, in the bench's launch configuration
+    (automatic split counts per decode set); the sampled (sequence, group) units come from the
+    host generator and are checked against the oracle, the rest of the cache is N(0,1) noise."""
+    from palu_testlib import swizzle_block
+    from rank_kv_cache_palu_b200.synth import normal, page_permutation
+    b, G, W, Pz = w.batch, w.groups, w.width, w.page_size
+    rks, rvs = w.group_ranks
+    cfg = P.make_config(w.num_heads, w.head_dim, w.group_size, w.rank_k, w.rank_v, Pz, w.rope_base,
+                        w.act_dtype, w.latent_dtype)
+    max_pages = (context + Pz - 1) // Pz
+    num_pages = b * max_pages
+    pt = page_permutation(seed, num_pages).reshape(b, max_pages)
+    dev = torch.device("cuda")
+    cache = P.LatentCache.allocate(cfg, num_pages, device=dev, ranks_k=rks, ranks_v=rvs)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(seed)
+    for pool in (cache.zk, cache.zv):
+        view = pool.view(TORCH_DTYPE[w.latent_dtype])
+        for i in range(0, view.numel(), 1 << 28):
+            seg = view[i:i + (1 << 28)]
+            seg.copy_(torch.randn(seg.shape, device=dev, generator=gen))
+    layout = ranked_offsets(w, rks, rvs)
+    host = {}
+    for (bi, g) in units:
+        for name, ranks, pool in (("zk", rks, cache.zk), ("zv", rvs, cache.zv)):
+            r = ranks[g]
+            rows_g, offs, page_bytes = layout[name]
+            z = torch.from_numpy(normal(seed, name, (context, r), unit=(bi, g))).to(TORCH_DTYPE[w.latent_dtype])
+            host[(name, bi, g)] = z.to(torch.float64).numpy()
+            zb = z.view(torch.uint8).numpy()
+            pages = pool.view(num_pages, page_bytes)
+            for p in range(max_pages):
+                t0, t1 = p * Pz, min(context, (p + 1) * Pz)
+                rows = np.zeros((Pz, rows_g[g]), np.uint8)
+                rows[: t1 - t0] = zb[t0:t1]
+                pages[pt[bi, p], offs[g]: offs[g] + Pz * rows_g[g]].copy_(torch.from_numpy(swizzle_block(rows)).to(dev))
+    q = normal_tensor(seed, "q", (b, 1, w.num_heads, w.head_dim), w.act_dtype)
+    B_k = torch.cat([normal_tensor(seed, f"B_k{g}", (r, W), w.act_dtype, 1 / math.sqrt(r)) for g, r in enumerate(rks)])
+    B_v = torch.cat([normal_tensor(seed, f"B_v{g}", (r, W), w.act_dtype, 1 / math.sqrt(r)) for g, r in enumerate(rvs)])
+    ws = torch.zeros(P.palu_decode_ranked_workspace_size(cfg, rks, rvs, b, 1, max_pages, 0), dtype=torch.uint8,
+                     device=dev)
+    out = torch.empty((b, 1, w.num_heads, w.head_dim), dtype=TORCH_DTYPE[w.act_dtype], device=dev)
+    lse = torch.empty((b, 1, w.num_heads), dtype=torch.float32, device=dev)
+    q_pos = torch.full((b, 1), context - 1, dtype=torch.int32, device=dev)
+    lens = torch.full((b,), context, dtype=torch.int32, device=dev)
+    P.palu_decode_attn_ranked(cfg, rks, rvs, q.to(dev), q_pos, cache.zk, cache.zv, None, None, None,
+                              torch.from_numpy(pt).to(dev), lens, num_pages, B_k.to(dev), B_v.to(dev), out, lse, ws, 0)
+    torch.cuda.synchronize()
+    assert P.palu_get_device_status(ws)[0] == 0
+    got = out.to(torch.float64).cpu().numpy()
+    qn = q.to(torch.float64).numpy()
+    Bk_l = [t.to(torch.float64).numpy() for t in torch.split(B_k, list(rks))]
+    Bv_l = [t.to(torch.float64).numpy() for t in torch.split(B_v, list(rvs))]
+    worst = 0.0
+    gs = w.group_size
+    for (bi, g) in units:
+        heads = slice(g * gs, (g + 1) * gs)
+        ref, _ = O.decode_attention_ranked(qn[bi][:, heads], np.array([context - 1]), [host[("zk", bi, g)]],
+                                           [host[("zv", bi, g)]], np.arange(context), [Bk_l[g]], [Bv_l[g]], gs,
+                                           w.rope_base)
+        err = rel_err(got[bi, 0, heads], ref[0])
+        worst = max(worst, err)
+        assert err <= TOL[w.act_dtype], f"unit ({bi},{g}): {err:.3e}"
+    return worst
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", ["7b_bf16_ranked_b16_t16k", "7b_bf16_ranked_b16_t16k_norope"])
+def test_ranked_full_size_sampled(name):
+    # the ranked bench workloads (16 x 16k + a ragged page), one sampled unit per key / value rank
+    w = WORKLOADS[name]
+    worst = ranked_full_size(w, w.context + 9, [(0, 0), (5, 1), (9, 3), (15, 6)])
+    print(f"{name}: worst rel err {worst:.2e}")

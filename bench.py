@@ -19,7 +19,6 @@ Rank 0 prints one JSON line.
 from __future__ import annotations
 
 import argparse
-import glob
 import hashlib
 import json
 import math
@@ -69,9 +68,17 @@ def measured_peaks() -> dict:
             "source": "fallback"}
 
 
+# The sources the decode kernels are built from (their own files and every header
+# they include); a committed traffic figure is used only while these are unchanged.
+DECODE_SOURCES = ["decode_tc.cu", "decode_fused.cu", "decode_simt.cu", "palu_common.cuh", "palu_internal.h",
+                  "palu_tc.h", "tc_ptx.cuh"]
+
+
 def csrc_hash() -> str:
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "rank_kv_cache_palu_b200", "csrc", "*"))):
+    paths = [os.path.join(ROOT, "rank_kv_cache_palu_b200", "csrc", n) for n in DECODE_SOURCES]
+    paths.append(os.path.join(ROOT, "include", "palu.h"))
+    for p in paths:
         with open(p, "rb") as f:
             h.update(os.path.basename(p).encode() + f.read())
     return h.hexdigest()[:16]

@@ -22,10 +22,11 @@ __global__ void __launch_bounds__(kThreads) compress_kernel(const __grid_constan
   DevStatus* st = reinterpret_cast<DevStatus*>(a.status);
 
   const bool is_v = blockIdx.z == 1;
-  const int r = is_v ? a.r_v : a.r_k;
-  const int N = a.gm.n * r;                 // output columns: entry gc / r, latent entry gc % r
+  // output column gc belongs to entry col_entry(cols, n, gc), latent entry gc - cols[entry]
+  const uint16_t* cols = is_v ? a.vcol : a.kcol;
+  const int N = is_v ? a.ncols_v : a.ncols_k;
   const long long acols = is_v ? a.a_vcols : a.a_kcols;
-  const int* col0s = is_v ? a.gm.v_row0 : a.gm.k_row0;
+  const uint16_t* col0s = is_v ? a.gm.v_row0 : a.gm.k_row0;
   const int row0 = blockIdx.x * kBM, col0 = blockIdx.y * kBN;
   if (col0 >= N) return;
   const TA* X = reinterpret_cast<const TA*>(a.x);
@@ -42,7 +43,12 @@ __global__ void __launch_bounds__(kThreads) compress_kernel(const __grid_constan
     for (int e = tid; e < kBK * kBN; e += kThreads) {
       const int k = e / kBN, c = e % kBN;
       const int gk = k0 + k, gc = col0 + c;
-      as_[k][c] = (gk < a.d_model && gc < N) ? Dt<ACT>::to_f(A[(size_t)gk * acols + col0s[gc / r] + gc % r]) : 0.f;
+      float v = 0.f;
+      if (gk < a.d_model && gc < N) {
+        const int e = col_entry(cols, a.gm.n, gc);
+        v = Dt<ACT>::to_f(A[(size_t)gk * acols + col0s[e] + (gc - cols[e])]);
+      }
+      as_[k][c] = v;
     }
     __syncthreads();
 #pragma unroll 8
@@ -71,7 +77,6 @@ __global__ void __launch_bounds__(kThreads) compress_kernel(const __grid_constan
 
   if constexpr (LAT == PALU_INT4) {
     // one thread per (token row, 32-entry block)
-    const long long srow = is_v ? a.vs_row : a.ks_row;
     const long long spage = is_v ? a.gm.vs_page : a.gm.ks_page;
     if (tid < kBM * 2) {
       const int i = tid / 2, blk = tid % 2;
@@ -82,7 +87,8 @@ __global__ void __launch_bounds__(kThreads) compress_kernel(const __grid_constan
           if (slot >= cap) {
             report(st, PALU_ERR_DEVICE_BOUNDS, 3000000 + gi);
           } else {
-            const int e = gc / r, j0 = gc % r;
+            const int e = col_entry(cols, a.gm.n, gc), j0 = gc - cols[e];
+            const long long srow = int4_scale_row(cols[e + 1] - cols[e]);
             const int tok = slot % a.P;
             uint8_t* pblk = const_cast<uint8_t*>(is_v ? a.gm.zv[e] : a.gm.zk[e]) + (long long)(slot / a.P) * page_bytes;
             uint8_t* sblk = const_cast<uint8_t*>(is_v ? a.gm.zvs[e] : a.gm.zks[e]) + (long long)(slot / a.P) * spage;
@@ -124,7 +130,7 @@ __global__ void __launch_bounds__(kThreads) compress_kernel(const __grid_constan
       for (int v = 0; v < 4; ++v) {
         const int gc = col0 + tx * 4 + v;
         if (gc >= N) continue;
-        const int e = gc / r, j = gc % r;
+        const int e = col_entry(cols, a.gm.n, gc), j = gc - cols[e];
         uint8_t* blk = const_cast<uint8_t*>(is_v ? a.gm.zv[e] : a.gm.zk[e]) + (long long)(slot / a.P) * page_bytes;
         *reinterpret_cast<TL*>(blk + swz_offset(slot % a.P, (long long)j * sizeof(TL), a.P)) =
             Dt<LAT>::from_f(ct[i][tx * 4 + v]);
@@ -144,7 +150,7 @@ __global__ void __launch_bounds__(kThreads) compress_kernel(const __grid_constan
 
 template <int ACT, int LAT>
 cudaError_t launch_t(const CompressArgs& a, cudaStream_t st) {
-  const int ncol = a.gm.n * (a.r_k > a.r_v ? a.r_k : a.r_v);
+  const int ncol = a.ncols_k > a.ncols_v ? a.ncols_k : a.ncols_v;
   dim3 grid((a.n + kBM - 1) / kBM, (ncol + kBN - 1) / kBN, 2);
   compress_kernel<ACT, LAT><<<grid, kThreads, 0, st>>>(a);
   count_launch();

@@ -43,12 +43,13 @@ struct Plan {
   size_t counter_bytes, partial_bytes;
 };
 
-Plan make_plan(int n, int d_model, int G, int r_k, int r_v) {
+// ncols_k / ncols_v: the launch's output columns on the key and value sides
+Plan make_plan(int n, int d_model, int ncols_k, int ncols_v) {
   Plan p{};
   p.NT = n <= 256 ? ((n + 15) / 16) * 16 : 256;
   p.ntt = (n + p.NT - 1) / p.NT;
-  p.tk = (G * r_k + kM - 1) / kM;
-  p.tv = (G * r_v + kM - 1) / kM;
+  p.tk = (ncols_k + kM - 1) / kM;
+  p.tv = (ncols_v + kM - 1) / kM;
   const int tiles = (p.tk + p.tv) * p.ntt;
   const int kst = d_model / kKStage;
   int ks = 1;
@@ -77,14 +78,14 @@ struct TcArgs {
   float* partials;
 };
 
-// Column of A holding column lc of this launch (group entry lc / r, latent
-// entry lc % r).  Past the last entry it continues from the last one, so a TMA
-// box that runs off the end still has a valid start (those columns are
-// computed and dropped).
-__device__ __forceinline__ int a_column(const GroupMap& gm, const int* row0, int r, int lc) {
-  int e = lc / r;
-  if (e >= gm.n) e = gm.n - 1;
-  return row0[e] + (lc - e * r);
+// Column of A holding output column lc of this launch (entry e = the column
+// table's entry of lc, latent entry lc - cols[e]).  Past the last entry it
+// continues from the last one, so a TMA box that runs off the end still has a
+// valid start (those columns are computed and dropped).  Entries are multiples
+// of 64 columns wide, so a 64-column box never straddles two.
+__device__ __forceinline__ int a_column(const GroupMap& gm, const uint16_t* cols, const uint16_t* row0, int lc) {
+  const int e = col_entry(cols, gm.n, lc);
+  return row0[e] + (lc - cols[e]);
 }
 
 // Write latent entry j of one token into its (page, group) block.
@@ -121,8 +122,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool is_v = blockIdx.x >= p.tk;
   const int ctile = is_v ? blockIdx.x - p.tk : blockIdx.x;
   const int c0 = ctile * kM;
-  const int r = is_v ? a.r_v : a.r_k;
-  const int ncols = a.gm.n * r;
+  const uint16_t* cols = is_v ? a.vcol : a.kcol;
+  const int ncols = is_v ? a.ncols_v : a.ncols_k;
   const int t0 = blockIdx.y * p.NT;
   const int kst = a.d_model / kKStage;
   const int split = blockIdx.z;
@@ -154,13 +155,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tm_x);
       int s = 0;
       uint32_t ph = 0;
+      // the tile's two 64-column boxes of A, fixed over the K loop
+      const uint16_t* row0 = is_v ? a.gm.v_row0 : a.gm.k_row0;
+      const int ax0 = a_column(a.gm, cols, row0, c0), ax1 = a_column(a.gm, cols, row0, c0 + 64);
       for (int kb = ks0; kb < ks1 && !*abort_flag; ++kb) {
         if (!mbar_wait(empty(s), ph ^ 1, abort_flag, st, 50)) break;
         mbar_expect_tx(full(s), (uint32_t)stage_bytes);
         const uint32_t dst = base + (uint32_t)s * stage_bytes;
-        const int* row0 = is_v ? a.gm.v_row0 : a.gm.k_row0;
-        tma_load_2d(dst, tm_a, a_column(a.gm, row0, r, c0), kb * kKStage, full(s));
-        tma_load_2d(dst + kABytes / 2, tm_a, a_column(a.gm, row0, r, c0 + 64), kb * kKStage, full(s));
+        tma_load_2d(dst, tm_a, ax0, kb * kKStage, full(s));
+        tma_load_2d(dst + kABytes / 2, tm_a, ax1, kb * kKStage, full(s));
         tma_load_2d(dst + kABytes, &tm_x, kb * kKStage, t0, full(s));
         if (++s == p.stages) { s = 0; ph ^= 1; }
       }
@@ -233,7 +236,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok && finalize) {
       const long long cap = (long long)a.num_pages * a.P;
       const bool col_ok = gc < ncols;
-      const int e = col_ok ? gc / r : 0, j = gc % r;   // group entry and latent entry of this column
+      const int e = col_ok ? col_entry(cols, a.gm.n, gc) : 0;   // group entry of this column
+      const int j = gc - cols[e];                                 // latent entry within it
       uint8_t* pool = const_cast<uint8_t*>(is_v ? a.gm.zv[e] : a.gm.zk[e]);
       const long long page_bytes = is_v ? a.gm.v_page : a.gm.k_page;
       const int ntok = min(p.NT, a.n - t0);
@@ -282,7 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   (uint8_t)((code & 0xF) | ((hi & 0xF) << 4));
             if (col_ok && lane == 0) {
               const uint8_t* spool = is_v ? a.gm.zvs[e] : a.gm.zks[e];
-              const long long srow = is_v ? a.vs_row : a.ks_row;
+              const long long srow = int4_scale_row(cols[e + 1] - cols[e]);
               const long long spage = is_v ? a.gm.vs_page : a.gm.ks_page;
               reinterpret_cast<__half*>(const_cast<uint8_t*>(spool) + (long long)(slot / a.P) * spage +
                                         (slot % a.P) * srow)[j >> 5] = s16;
@@ -340,7 +344,7 @@ bool map2d(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, uint64_t inn
 
 template <int ACT, int LAT>
 cudaError_t launch_t(const CompressArgs& a, cudaStream_t st) {
-  const Plan p = make_plan(a.n, a.d_model, a.gm.n, a.r_k, a.r_v);
+  const Plan p = make_plan(a.n, a.d_model, a.ncols_k, a.ncols_v);
   const CUtensorMapDataType dt = ACT == PALU_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   CUtensorMap tm_ak, tm_av, tm_x;
   if (!map2d(&tm_ak, a.Ak, dt, (uint64_t)a.a_kcols, a.d_model, (uint64_t)a.a_kcols * 2, 64, kKStage) ||
@@ -376,10 +380,9 @@ bool tc_compress_supported(const palu_config* c, int n_tokens, int d_model) {
   return true;
 }
 
-size_t tc_compress_scratch_bytes(const palu_config* c, int n_tokens, int d_model) {
+size_t tc_compress_scratch_bytes(const palu_config* c, int n_tokens, int d_model, int ncols_k, int ncols_v) {
   if (!tc_compress_supported(c, n_tokens, d_model)) return 0;
-  const int G = c->num_heads / c->group_size;
-  const Plan p = make_plan(n_tokens, d_model, G, c->rank_k, c->rank_v);
+  const Plan p = make_plan(n_tokens, d_model, ncols_k, ncols_v);
   return p.counter_bytes + p.partial_bytes;
 }
 

@@ -256,7 +256,7 @@ palu_config set_cfg(const Layer& L, int k) {
   return x;
 }
 
-// Group map of the groups g with part[g] == c (compress class or decode set).
+// Group map of the groups g with part[g] == c (a decode set), or of every group (part NULL).
 void build_map(const Layer& L, const int* part, int c, const void* zk, const void* zv, const void* zks,
                const void* zvs, palu::GroupMap& m) {
   auto at = [](const void* pool, long long off) {
@@ -268,16 +268,16 @@ void build_map(const Layer& L, const int* part, int c, const void* zk, const voi
   m.ks_page = L.ks_page;
   m.vs_page = L.vs_page;
   for (int g = 0; g < L.G; ++g) {
-    if (part[g] != c) continue;
+    if (part != nullptr && part[g] != c) continue;
     const int i = m.n++;
-    m.g[i] = g;
+    m.g[i] = (uint16_t)g;
     m.zk[i] = at(zk, L.k_off[g]);
     m.zv[i] = at(zv, L.v_off[g]);
     m.zks[i] = at(zks, L.ks_off[g]);
     m.zvs[i] = at(zvs, L.vs_off[g]);
-    m.k_row0[i] = L.k_row0[g];
-    m.v_row0[i] = L.v_row0[g];
-    m.rk[i] = L.rk[g];
+    m.k_row0[i] = (uint16_t)L.k_row0[g];
+    m.v_row0[i] = (uint16_t)L.v_row0[g];
+    m.rk[i] = (uint16_t)L.rk[g];
   }
 }
 
@@ -303,14 +303,21 @@ size_t decode_workspace(const Layer& L, int batch, int Q, int max_pages, int num
   return kStatusBytes + part + fq;
 }
 
-size_t compress_workspace(const Layer& L, int n_tokens, int d_model) {
-  size_t sc = 0;
+// The compress kernels take every group of the layer in one launch (output
+// columns follow the groups' ranks); the tensor-core kernel serves the layer
+// when it serves each group's rank pair.
+bool compress_tc_ok(const Layer& L, int n_tokens, int d_model) {
   for (int c = 0; c < L.nclass; ++c) {
     const palu_config cc = class_cfg(L, c);
-    const size_t b = palu::tc_compress_scratch_bytes(&cc, n_tokens, d_model);
-    if (b > sc) sc = b;
+    if (!palu::tc_compress_supported(&cc, n_tokens, d_model)) return false;
   }
-  return kStatusBytes + sc;
+  return true;
+}
+
+size_t compress_workspace(const Layer& L, int n_tokens, int d_model) {
+  if (!compress_tc_ok(L, n_tokens, d_model)) return kStatusBytes;
+  const palu_config c0 = class_cfg(L, 0);
+  return kStatusBytes + palu::tc_compress_scratch_bytes(&c0, n_tokens, d_model, L.bk_rows, L.bv_rows);
 }
 
 palu_status compress_layer(const Layer& L, int n_tokens, int d_model, const void* x, const void* A_k,
@@ -348,21 +355,21 @@ palu_status compress_layer(const Layer& L, int n_tokens, int d_model, const void
   a.scratch_bytes = workspace_bytes - kStatusBytes;
   a.a_kcols = L.bk_rows;
   a.a_vcols = L.bv_rows;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  for (int c = 0; c < L.nclass; ++c) {
-    const palu_config cc = class_cfg(L, c);
-    a.r_k = cc.rank_k;
-    a.r_v = cc.rank_v;
-    a.k_row = palu::latent_row_bytes(a.lat, a.r_k);
-    a.v_row = palu::latent_row_bytes(a.lat, a.r_v);
-    a.ks_row = palu::scale_row_bytes(a.lat, a.r_k);
-    a.vs_row = palu::scale_row_bytes(a.lat, a.r_v);
-    build_map(L, L.cls, c, zk_pool, zv_pool, zk_scales, zv_scales, a.gm);
-    a.positions = c == 0 ? positions : nullptr;   // once per token
-    const cudaError_t e = palu::tc_compress_supported(&cc, n_tokens, d_model) ? palu::launch_compress_tc(a, st)
-                                                                             : palu::launch_compress_simt(a, st);
-    if (e != cudaSuccess) return cuda_status(e);
+  a.positions = positions;
+  // every group in one launch: output column c of the key side is column c of A_k
+  // (the groups' columns follow each other in order), owned by group col_entry(kcol, G, c)
+  build_map(L, nullptr, 0, zk_pool, zv_pool, zk_scales, zv_scales, a.gm);
+  a.ncols_k = L.bk_rows;
+  a.ncols_v = L.bv_rows;
+  for (int g = 0; g <= L.G; ++g) {
+    a.kcol[g] = (uint16_t)(g < L.G ? L.k_row0[g] : L.bk_rows);
+    a.vcol[g] = (uint16_t)(g < L.G ? L.v_row0[g] : L.bv_rows);
   }
+  a.r_k = a.r_v = 0;   // per group: see kcol / vcol
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const cudaError_t e = compress_tc_ok(L, n_tokens, d_model) ? palu::launch_compress_tc(a, st)
+                                                             : palu::launch_compress_simt(a, st);
+  if (e != cudaSuccess) return cuda_status(e);
   return PALU_OK;
 }
 

@@ -46,6 +46,17 @@ template <> struct Dt<PALU_BF16> {
   __device__ __forceinline__ static T from_f(float v) { return __float2bfloat16_rn(v); }
 };
 
+// Entry of a column table (entry i owns columns [col[i], col[i + 1]), n entries)
+// that holds column c; columns past the last entry map to the last one.
+__host__ __device__ inline int col_entry(const uint16_t* col, int n, int c) {
+  int e = 0;
+  while (e + 1 < n && col[e + 1] <= c) ++e;
+  return e;
+}
+
+// Bytes of one token's int4 scale row for rank r: r/32 fp16 scales, padded to 16.
+__host__ __device__ inline long long int4_scale_row(int r) { return (2LL * (r / 32) + 15) / 16 * 16; }
+
 // Decode latent entry j of token t from its (page, group) block `blk` of P
 // tokens (swizzled layout; int4: code × fp16 scale from the token-major scale
 // row `srow`, rounded to the compute dtype ACT exactly as the dequantised value

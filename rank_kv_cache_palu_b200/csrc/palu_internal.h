@@ -20,15 +20,15 @@ constexpr int kMaxGroups = 64;   // head groups per layer
 // pool per group, at pool_g + pg·P·row_g.  Either way: base[g] + pg·page.
 struct GroupMap {
   int n;                                // groups this launch covers
-  int g[kMaxGroups];                    // model group of entry i (heads g·gs .. g·gs + gs − 1)
+  uint16_t g[kMaxGroups];               // model group of entry i (heads g·gs .. g·gs + gs − 1)
   const uint8_t* zk[kMaxGroups];        // per model group: block of page 0
   const uint8_t* zv[kMaxGroups];
   const uint8_t* zks[kMaxGroups];       // int4 scale rows (NULL otherwise)
   const uint8_t* zvs[kMaxGroups];
   long long k_page, v_page, ks_page, vs_page;   // bytes from one page's block to the next
-  int k_row0[kMaxGroups];               // first row of the group in B_k (= first column in A_k)
-  int v_row0[kMaxGroups];               // same for B_v / A_v
-  int rk[kMaxGroups];                   // key rank of the entry (decode launches may mix key ranks;
+  uint16_t k_row0[kMaxGroups];          // first row of the group in B_k (= first column in A_k)
+  uint16_t v_row0[kMaxGroups];          // same for B_v / A_v
+  uint16_t rk[kMaxGroups];              // key rank of the entry (decode launches may mix key ranks;
                                         // the launch's r_k is their maximum, r_v is shared)
 };
 
@@ -86,6 +86,10 @@ struct CompressArgs {
   const int32_t* positions;
   GroupMap gm;         // the groups of this launch; A column offsets in k_row0 / v_row0
   long long a_kcols, a_vcols;   // columns of A_k / A_v (row strides in elements)
+  // Output columns of this launch, key side: entry i owns [kcol[i], kcol[i + 1]) (its rank
+  // wide; ranks may differ between entries), kcol[gm.n] = ncols_k; likewise the value side.
+  int ncols_k, ncols_v;
+  uint16_t kcol[kMaxGroups + 1], vcol[kMaxGroups + 1];
   int32_t* pos_pool;
   void* status;
   float* scratch;  // workspace past the status header

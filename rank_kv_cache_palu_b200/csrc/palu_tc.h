@@ -25,7 +25,8 @@ cudaError_t launch_decode_fused(const DecodeArgs& a, cudaStream_t st);
 
 // Compress: shapes the tensor-core GEMM takes, and the scratch it needs.
 bool tc_compress_supported(const palu_config* c, int n_tokens, int d_model);
-size_t tc_compress_scratch_bytes(const palu_config* c, int n_tokens, int d_model);
+// ncols_k / ncols_v: output columns of the launch (Σ of its groups' key / value ranks)
+size_t tc_compress_scratch_bytes(const palu_config* c, int n_tokens, int d_model, int ncols_k, int ncols_v);
 cudaError_t launch_compress_tc(const CompressArgs& a, cudaStream_t st);
 
 }  // namespace palu

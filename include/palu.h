@@ -218,10 +218,11 @@ palu_status palu_decode_attn_multi(const palu_config* cfg, int batch, int num_qu
  *           inside the block the swizzled layout above applies unchanged.
  *   A_k     [d_model][Σ_g r_k,g]: group g's columns start at Σ_{g'<g} r_k,g'
  *   B_k     [Σ_g r_k,g][W]: group g's rows start at Σ_{g'<g} r_k,g'
- * With equal ranks this is byte for byte the uniform layout.  Groups that share
- * a rank pair are served by one launch of each kernel; the calls run the rank
- * classes one after another on `stream`.  Every other argument, rule and
- * status is that of the uniform call named in each comment. */
+ * With equal ranks this is byte for byte the uniform layout.  Compress runs one
+ * launch for every group; decode runs one split launch and one combine per set
+ * of groups sharing a value rank and kernel family (key ranks may differ within
+ * a set), the sets one after another on `stream`.  Every other argument, rule
+ * and status is that of the uniform call named in each comment. */
 /* as palu_cache_strides; k_group_offsets / v_group_offsets [G] (optional)
  * receive the byte offset of each group's block within a K / V page.  In an
  * int4 scale page, group g's block starts at Σ_{g'<g} page_size·srow_g'. */

@@ -82,7 +82,7 @@ int pass_queries(int kind, int remaining) {
   return remaining >= m ? m : remaining >= 2 ? 2 : 1;
 }
 
-int auto_splits(const palu_config* c, int batch, int max_pages, int kind) {
+int auto_splits(const palu_config* c, int batch, int max_pages, int kind, int qn = 1) {
   const int sms = 148;
   const long long groups = (long long)batch * (c->num_heads / c->group_size);
   const long long units = kind == 3   ? groups
@@ -97,16 +97,18 @@ int auto_splits(const palu_config* c, int batch, int max_pages, int kind) {
   }
   // Tensor-core kernels hold one CTA per SM and every CTA of a launch walks about
   // the same number of pages, so the launch takes ceil(CTAs / SMs) rounds of
-  // (pages per split + a start-up of ~2 pages).  Take the split count that
-  // minimises that (the smallest on ties), sized for the longest possible
-  // sequence (max_pages).  At least one full round of CTAs when the pages allow.
+  // (pages per split + a start-up of ~2 pages); with several queries per pass the
+  // combine adds about a page per split and query (measured: 4 queries per pass at
+  // 16 x 16k ran best at 4 splits, one query at 8).  Take the split count that minimises that (the
+  // smallest on ties), sized for the longest possible sequence (max_pages).  At
+  // least one full round of CTAs when the pages allow.
   long long S0 = (sms + units - 1) / units;
   if (S0 > max_pages) S0 = max_pages;
   if (S0 < 1) S0 = 1;
   long long best_S = S0, best_t = -1;
   for (long long S = S0; S <= max_pages && S <= 64; ++S) {
     const long long rounds = (units * S + sms - 1) / sms;
-    const long long t = rounds * ((max_pages + S - 1) / S + 2);
+    const long long t = rounds * ((max_pages + S - 1) / S + 2) + (qn > 1 ? S * qn : 0);
     if (best_t < 0 || t < best_t) {
       best_t = t;
       best_S = S;
@@ -122,9 +124,9 @@ int kernel_kind(const palu_config* c) {
   return 1;
 }
 
-// The split count a call runs (num_splits = 0: automatic).
-int run_S(const palu_config* c, int kind, int batch, int max_pages, int num_splits) {
-  return num_splits == 0 ? auto_splits(c, batch, max_pages, kind) : num_splits;
+// The split count a call runs (num_splits = 0: automatic); qn = queries per pass.
+int run_S(const palu_config* c, int kind, int batch, int max_pages, int num_splits, int qn = 1) {
+  return num_splits == 0 ? auto_splits(c, batch, max_pages, kind, qn) : num_splits;
 }
 
 // One layer's head groups and where their latents live.  Group g has its own
@@ -290,7 +292,7 @@ size_t decode_workspace(const Layer& L, int batch, int Q, int max_pages, int num
   for (int c = 0; c < L.nset; ++c) {
     const palu_config cc = set_cfg(L, c);
     const int kind = kernel_kind(&cc);
-    const int S = run_S(&cc, kind, batch, max_pages, num_splits);
+    const int S = run_S(&cc, kind, batch, max_pages, num_splits, pass_queries(kind, Q));
     const int vb = batch * pass_queries(kind, Q);
     const size_t pc = align256((size_t)vb * cc.num_heads * S * (cc.rank_v + 2) * sizeof(float));
     if (pc > part) part = pc;
@@ -439,7 +441,7 @@ palu_status decode_layer(const Layer& L, int batch, int Q, const void* q, const 
   for (int c = 0; c < L.nset; ++c) {
     const palu_config cc = set_cfg(L, c);
     const int kind = kernel_kind(&cc);
-    a.S = run_S(&cc, kind, batch, max_pages, num_splits);
+    a.S = run_S(&cc, kind, batch, max_pages, num_splits, pass_queries(kind, Q));
     a.r_k = cc.rank_k;
     a.r_v = cc.rank_v;
     a.k_row = palu::latent_row_bytes(a.lat, a.r_k);

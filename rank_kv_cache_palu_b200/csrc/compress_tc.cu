@@ -95,6 +95,55 @@ __device__ __forceinline__ void store_latent(const CompressArgs& a, uint8_t* blk
   *reinterpret_cast<TL*>(blk + swz_offset(slot % a.P, (long long)j * sizeof(TL), a.P)) = Dt<LAT>::from_f(v);
 }
 
+// Write 16 tokens (t0 + j0 .. t0 + j0 + 15, fewer at the end) of latent column gc
+// (this thread's; its warp holds 32 consecutive columns) into the paged cache:
+// rounded to the latent dtype, or int4-quantised per 32-column block.
+template <int LAT>
+__device__ __forceinline__ void store_tokens(const CompressArgs& a, bool is_v, const uint16_t* cols, int ncols, int gc,
+                                             int t0, int j0, int ntok, const float* v, DevStatus* st) {
+  const int lane = threadIdx.x & 31;
+  const long long cap = (long long)a.num_pages * a.P;
+  const bool col_ok = gc < ncols;
+  const int e = col_ok ? col_entry(cols, a.gm.n, gc) : 0;   // group entry of this column
+  const int j = gc - cols[e];                                 // latent entry within it
+  uint8_t* pool = const_cast<uint8_t*>(is_v ? a.gm.zv[e] : a.gm.zk[e]);
+  const long long page_bytes = is_v ? a.gm.v_page : a.gm.k_page;
+#pragma unroll 1
+  for (int u = 0; u < 16; ++u) {
+    const int ti = t0 + j0 + u;
+    if (j0 + u >= ntok) break;
+    const int slot = a.slots[ti];
+    if (slot < 0) continue;
+    if (slot >= cap) {
+      if (col_ok && (gc & 127) == 0) report(st, PALU_ERR_DEVICE_BOUNDS, 3000000 + ti);
+      continue;
+    }
+    if constexpr (LAT == PALU_INT4) {
+      // the warp's 32 columns are one quantisation block of this token
+      float amax = col_ok ? fabsf(v[u]) : 0.f;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+      const __half s16 = __float2half_rn(__fdiv_rn(amax, 7.0f));
+      const float s = __half2float(s16);
+      int code = 0;
+      if (s != 0.f) code = (int)fminf(fmaxf(rintf(__fdiv_rn(v[u], s)), -7.f), 7.f);
+      const int hi = __shfl_down_sync(0xffffffffu, code, 1);
+      if (col_ok && (lane & 1) == 0)
+        pool[(long long)(slot / a.P) * page_bytes + swz_offset(slot % a.P, j >> 1, a.P)] =
+            (uint8_t)((code & 0xF) | ((hi & 0xF) << 4));
+      if (col_ok && lane == 0) {
+        const uint8_t* spool = is_v ? a.gm.zvs[e] : a.gm.zks[e];
+        const long long srow = int4_scale_row(cols[e + 1] - cols[e]);
+        const long long spage = is_v ? a.gm.vs_page : a.gm.ks_page;
+        reinterpret_cast<__half*>(const_cast<uint8_t*>(spool) + (long long)(slot / a.P) * spage +
+                                  (slot % a.P) * srow)[j >> 5] = s16;
+      }
+    } else {
+      if (col_ok) store_latent<LAT>(a, pool + (long long)(slot / a.P) * page_bytes, j, slot, v[u]);
+    }
+  }
+}
+
 template <int ACT, int LAT>
 __global__ void __launch_bounds__(kThreads, 1)
     compress_tc_kernel(const __grid_constant__ CUtensorMap tm_ak, const __grid_constant__ CUtensorMap tm_av,
@@ -235,11 +284,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok && finalize) {
       const long long cap = (long long)a.num_pages * a.P;
-      const bool col_ok = gc < ncols;
-      const int e = col_ok ? col_entry(cols, a.gm.n, gc) : 0;   // group entry of this column
-      const int j = gc - cols[e];                                 // latent entry within it
-      uint8_t* pool = const_cast<uint8_t*>(is_v ? a.gm.zv[e] : a.gm.zk[e]);
-      const long long page_bytes = is_v ? a.gm.v_page : a.gm.k_page;
       const int ntok = min(p.NT, a.n - t0);
       for (int j0 = 0; j0 < ntok; j0 += 16) {
         float v[16];
@@ -261,40 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-#pragma unroll 1
-        for (int u = 0; u < 16; ++u) {
-          const int ti = t0 + j0 + u;
-          if (j0 + u >= ntok) break;
-          const int slot = a.slots[ti];
-          if (slot < 0) continue;
-          if (slot >= cap) {
-            if (col_ok && c == 0) report(st, PALU_ERR_DEVICE_BOUNDS, 3000000 + ti);
-            continue;
-          }
-          if constexpr (LAT == PALU_INT4) {
-            // the warp's 32 columns are one quantisation block of this token
-            float amax = col_ok ? fabsf(v[u]) : 0.f;
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-            const __half s16 = __float2half_rn(__fdiv_rn(amax, 7.0f));
-            const float s = __half2float(s16);
-            int code = 0;
-            if (s != 0.f) code = (int)fminf(fmaxf(rintf(__fdiv_rn(v[u], s)), -7.f), 7.f);
-            const int hi = __shfl_down_sync(0xffffffffu, code, 1);
-            if (col_ok && (lane & 1) == 0)
-              pool[(long long)(slot / a.P) * page_bytes + swz_offset(slot % a.P, j >> 1, a.P)] =
-                  (uint8_t)((code & 0xF) | ((hi & 0xF) << 4));
-            if (col_ok && lane == 0) {
-              const uint8_t* spool = is_v ? a.gm.zvs[e] : a.gm.zks[e];
-              const long long srow = int4_scale_row(cols[e + 1] - cols[e]);
-              const long long spage = is_v ? a.gm.vs_page : a.gm.ks_page;
-              reinterpret_cast<__half*>(const_cast<uint8_t*>(spool) + (long long)(slot / a.P) * spage +
-                                        (slot % a.P) * srow)[j >> 5] = s16;
-            }
-          } else {
-            if (col_ok) store_latent<LAT>(a, pool + (long long)(slot / a.P) * page_bytes, j, slot, v[u]);
-          }
-        }
+        store_tokens<LAT>(a, is_v, cols, ncols, gc, t0, j0, ntok, v, st);
       }
       // positions, once per token
       if (!is_v && ctile == 0 && a.positions != nullptr && a.pos_pool != nullptr) {
@@ -313,6 +324,170 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, 256);
+  }
+}
+
+// Prefill (several token tiles, no K split): a persistent kernel, one CTA per SM,
+// walking the (column tile, token tile) tiles round-robin with two TMEM
+// accumulators, so that the epilogue of one tile overlaps the MMAs of the next.
+// Consecutive tiles share their token tile (x stays in L2 while the column tiles
+// pass over it).  Same roles as above: warp 0 TMA, warp 1 MMA, warps 2-5 epilogue.
+template <int ACT, int LAT>
+__global__ void __launch_bounds__(kThreads, 1)
+    compress_tc_persistent_kernel(const __grid_constant__ CUtensorMap tm_ak, const __grid_constant__ CUtensorMap tm_av,
+                                  const __grid_constant__ CUtensorMap tm_x, const TcArgs t) {
+  extern __shared__ uint8_t smem_raw[];
+  const CompressArgs& a = t.a;
+  const Plan& p = t.p;
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* sbase = smem_raw + (base - raw);
+  const int stage_bytes = kABytes + p.NT * 128;
+  const uint32_t bars = base + (uint32_t)p.stages * stage_bytes;      // 2·stages + 4 barriers
+  uint8_t* misc = sbase + (uint32_t)p.stages * stage_bytes + 256;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 16);
+  auto full = [&](int s) { return bars + 8u * s; };
+  auto empty = [&](int s) { return bars + 8u * (p.stages + s); };
+  auto acc_full = [&](int b) { return bars + 8u * (2 * p.stages + b); };
+  auto acc_empty = [&](int b) { return bars + 8u * (2 * p.stages + 2 + b); };
+  DevStatus* st = reinterpret_cast<DevStatus*>(a.status);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ctiles = p.tk + p.tv;
+  const int ntiles = ctiles * p.ntt;
+  const int kst = a.d_model / kKStage;
+  // tile i of this CTA: global tile blockIdx.x + i·gridDim.x = (column tile, token tile)
+  auto tile_of = [&](int i, int& ctile, bool& is_v, int& c0, int& t0) {
+    const int tg = blockIdx.x + i * gridDim.x;
+    const int ct = tg % ctiles;
+    is_v = ct >= p.tk;
+    ctile = is_v ? ct - p.tk : ct;
+    c0 = ctile * kM;
+    t0 = (tg / ctiles) * p.NT;
+  };
+  const int my_tiles = blockIdx.x < ntiles ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    for (int s = 0; s < p.stages; ++s) {
+      mbar_init(full(s), 1);
+      mbar_init(empty(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(acc_full(b), 1);
+      mbar_init(acc_empty(b), 4);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tmap(&tm_ak);
+      prefetch_tmap(&tm_av);
+      prefetch_tmap(&tm_x);
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int i = 0; i < my_tiles && ok; ++i) {
+        int ctile, c0, t0;
+        bool is_v;
+        tile_of(i, ctile, is_v, c0, t0);
+        const CUtensorMap* tm_a = is_v ? &tm_av : &tm_ak;
+        const uint16_t* cols = is_v ? a.vcol : a.kcol;
+        const uint16_t* row0 = is_v ? a.gm.v_row0 : a.gm.k_row0;
+        const int ax0 = a_column(a.gm, cols, row0, c0), ax1 = a_column(a.gm, cols, row0, c0 + 64);
+        for (int kb = 0; kb < kst; ++kb) {
+          if (*abort_flag || !mbar_wait(empty(s), ph ^ 1, abort_flag, st, 60)) { ok = false; break; }
+          mbar_expect_tx(full(s), (uint32_t)stage_bytes);
+          const uint32_t dst = base + (uint32_t)s * stage_bytes;
+          tma_load_2d(dst, tm_a, ax0, kb * kKStage, full(s));
+          tma_load_2d(dst + kABytes / 2, tm_a, ax1, kb * kKStage, full(s));
+          tma_load_2d(dst + kABytes, &tm_x, kb * kKStage, t0, full(s));
+          if (++s == p.stages) { s = 0; ph ^= 1; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr int kBf = ACT == PALU_BF16 ? 1 : 0;
+      const uint32_t idesc = idesc_f16(kBf, 1, 0, p.NT, kM);    // Aᵀ MN-major, xᵀ K-major
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int i = 0; i < my_tiles && ok; ++i) {
+        const int b = i & 1;
+        // the epilogue has read this accumulator's previous tile (i - 2)
+        if (!mbar_wait(acc_empty(b), ((i >> 1) & 1) ^ 1, abort_flag, st, 61)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + 256u * b;
+        for (int kb = 0; kb < kst; ++kb) {
+          if (!mbar_wait(full(s), ph, abort_flag, st, 62)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = base + (uint32_t)s * stage_bytes;
+          const uint32_t sx = sa + kABytes;
+#pragma unroll
+          for (int kk = 0; kk < kKStage / 16; ++kk) {
+            const uint64_t ad = sdesc(sa + kk * 16 * 128, kABytes / 2, 1024, kSw128);
+            const uint64_t bd = sdesc(sx + kk * 32, 16, 1024, kSw128);
+            umma_f16(d, ad, bd, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(empty(s));
+          if (++s == p.stages) { s = 0; ph ^= 1; }
+        }
+        umma_commit(acc_full(b));   // fires once every MMA of the tile has completed
+      }
+      // drain before TMEM is released
+      if (my_tiles > 0) mbar_wait(acc_full((my_tiles - 1) & 1), ((my_tiles - 1) >> 1) & 1, abort_flag, st, 63);
+    }
+  } else {
+    // ============================================================ epilogue (warps 2-5)
+    const int q4 = warp & 3;
+    const int c = q4 * 32 + lane;            // latent column of this thread within the tile
+    const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
+    for (int i = 0; i < my_tiles; ++i) {
+      const int b = i & 1;
+      int ctile, c0, t0;
+      bool is_v;
+      tile_of(i, ctile, is_v, c0, t0);
+      if (!mbar_wait(acc_full(b), (i >> 1) & 1, abort_flag, st, 64)) break;
+      tc_fence_after();
+      const uint16_t* cols = is_v ? a.vcol : a.kcol;
+      const int ncols = is_v ? a.ncols_v : a.ncols_k;
+      const int ntok = min(p.NT, a.n - t0);
+      for (int j0 = 0; j0 < ntok; j0 += 16) {
+        float v[16];
+        tmem_ld16(tmem + lane_addr + 256u * b + j0, v);
+        tmem_wait_ld();
+        store_tokens<LAT>(a, is_v, cols, ncols, c0 + c, t0, j0, ntok, v, st);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty(b));
+      // positions, once per token
+      if (!is_v && ctile == 0 && a.positions != nullptr && a.pos_pool != nullptr) {
+        const long long cap = (long long)a.num_pages * a.P;
+        for (int k = c; k < ntok; k += kM) {
+          const int slot = a.slots[t0 + k];
+          if (slot >= 0 && slot < cap) a.pos_pool[slot] = a.positions[t0 + k];
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -358,6 +533,16 @@ cudaError_t launch_t(const CompressArgs& a, cudaStream_t st) {
   t.counters = reinterpret_cast<int*>(scratch);
   t.partials = reinterpret_cast<float*>(scratch + p.counter_bytes);
   const size_t smem = (size_t)p.stages * (kABytes + p.NT * 128) + 256 + 64 + 1024;
+  if (p.ntt >= 2 && p.KS == 1) {
+    // prefill: persistent, one CTA per SM over every tile
+    auto kern = compress_tc_persistent_kernel<ACT, LAT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int tiles = (p.tk + p.tv) * p.ntt;
+    kern<<<tiles < 148 ? tiles : 148, kThreads, smem, st>>>(tm_ak, tm_av, tm_x, t);
+    count_launch();
+    return cudaGetLastError();
+  }
   auto kern = compress_tc_kernel<ACT, LAT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

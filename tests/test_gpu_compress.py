@@ -230,3 +230,29 @@ def test_compress_append_step_full_size():
     rows = np.flatnonzero(slots >= 0)
     _check_rows(w, x, A_k, cache.zk, slots, rows, w.rank_k, "bf16")
     _check_rows(w, x, A_v, cache.zv, slots, rows, w.rank_v, "bf16")
+
+
+@pytest.mark.parametrize("act", ["f16", "bf16"])
+def test_compress_int4_prefill_bit_exact(act):
+    # several 256-token tiles (the persistent prefill kernel) with int4 latents: exactly
+    # representable latents give bit-exact codes, bytes and scales; positions are written once
+    w = dataclasses.replace(WORKLOADS["tiny_f32"], act_dtype=act, latent_dtype="int4", rank_k=256,
+                            rank_v=512, d_model=256)
+    n = 700
+    x, A_k, A_v = exact_inputs(w, n, 13)
+    num_pages = 8
+    slots = make_slots(n, num_pages, w.page_size, seed=17)
+    positions = (np.arange(n) * 7 + 3).astype(np.int32)
+    cache, st, _ = run_compress(w, x, A_k, A_v, slots, positions, num_pages)
+    assert st == 0
+    keep = slots >= 0
+    for pool, spool, A, r in ((cache.zk, cache.zks, A_k, w.rank_k), (cache.zv, cache.zvs, A_v, w.rank_v)):
+        z = O.compress(x.to(torch.float64).numpy(), A.to(torch.float64).numpy(), "f32")
+        packed, sc = O.quantize_int4(z.reshape(n, w.groups, r).astype(np.float32))
+        srow = (2 * (r // 32) + 15) // 16 * 16
+        got = gather_rows(pool, w, slots, r, r // 2)
+        got_s = gather_rows(spool, w, slots, r, srow, swizzled=False)[..., : 2 * (r // 32)].copy().view(np.float16)
+        np.testing.assert_array_equal(got[keep], packed[keep])
+        np.testing.assert_array_equal(got_s[keep], sc[keep])
+    pos = cache.pos.cpu().numpy()
+    np.testing.assert_array_equal(pos[slots[keep]], positions[keep])

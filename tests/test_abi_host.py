@@ -240,3 +240,25 @@ def test_ranked_workspace_covers_every_decode_set():
     # set (r_v 128, tensor cores) = groups 0 and 3 (key ranks 256 and 128): 8 heads;
     # group 2 (key rank 384) runs on the CUDA-core kernel, group 1 (r_v 256) alone
     assert ws == 256 + 16 * 8 * 4 * 130 * 4
+
+
+def test_split_count_model():
+    # tensor-core launches: the split count minimises ceil(units·S / 148) · (pages/S + 2) over at
+    # least one full round of CTAs (smallest on ties); a pass of several fused queries adds S·Q
+    def model(units, pages, qn=1):
+        s0 = max(1, min(pages, -(-148 // units)))
+        best = None
+        for S in range(s0, min(pages, 64) + 1):
+            t = -(-units * S // 148) * (-(-pages // S) + 2) + (S * qn if qn > 1 else 0)
+            if best is None or t < best[0]:
+                best = (t, S)
+        return best[1]
+    rope = cfg()                                   # 32 heads / 4: 8 groups x 2 head pairs per sequence
+    norope = cfg(rope_base=0.0)                    # fused kernel: one CTA per (sequence, group)
+    for batch, pages in ((16, 130), (8, 130), (32, 130), (1, 34), (16, 514)):
+        assert P.palu_decode_num_splits(rope, batch, pages) == model(batch * 16, pages)
+        assert P.palu_decode_num_splits(norope, batch, pages) == model(batch * 8, pages)
+    assert P.palu_decode_num_splits(rope, 16, 130) == 4 and P.palu_decode_num_splits(norope, 16, 130) == 8
+    # the multi-query workspace is sized for the split count of its passes (4 queries: fewer splits)
+    one = P.palu_decode_multi_workspace_size(norope, 16, 4, 130, model(128, 130, 4))
+    assert P.palu_decode_multi_workspace_size(norope, 16, 4, 130, 0) == one

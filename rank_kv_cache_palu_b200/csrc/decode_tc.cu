@@ -18,7 +18,7 @@
 //   warp 1  MMA issuer: D[128 tok × 256] = z_k · B_k[:, 2 heads] into one of two
 //           TMEM slots (kind::f16, fp32 accumulate); then aᵀ[r_v × 16] =
 //           z_vᵀ · Pᵀ for the previous tile into the drained slot.
-//   warps 2-9 epilogue, two warpgroups of one thread per token: tcgen05.ld the rebuilt keys,
+//   warps 4-11 epilogue, two warpgroups of one thread per token: tcgen05.ld the rebuilt keys,
 //           rotate them (RoPE at the token's position), score against the
 //           rotated query, online softmax (exp2), write P (bf16/fp16) for the
 //           value MMA, and fold each tile's aᵀ into running latent sums.
@@ -136,6 +136,13 @@ __device__ __forceinline__ int page_of(const DecodeArgs& a, int b, int lp) {
   const int pg = a.page_table[(size_t)b * a.max_pages + lp];
   return (pg < 0 || pg >= a.num_pages) ? -1 : pg;
 }
+
+// The producers read the table entry of a tile one tile before they use it
+// (raw, checked at the use), so the dependent load never stalls the copies.
+__device__ __forceinline__ int page_ahead(const DecodeArgs& a, int b, const TileRange& tr, int k) {
+  return k < tr.ntiles ? a.page_table[(size_t)b * a.max_pages + tr.t_begin / kTile + k] : -1;
+}
+__device__ __forceinline__ bool page_valid(const DecodeArgs& a, int pg) { return pg >= 0 && pg < a.num_pages; }
 
 // P (softmax weights) tile, K-major with the 128-byte swizzle: row n (head),
 // token k.  Tokens 0-63 and 64-127 sit in two 2 KB atoms of 16 rows.
@@ -333,23 +340,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint4 raw[4];
       uint16_t sc[4];
     };
-    auto issue = [&](int n, Slot& sl) {
+    auto prefetch_page = [&](int ppg) {
+      if (zt != 0 || !page_valid(a, ppg)) return;
+      prefetch_l2(gm.zk[gi] + (size_t)ppg * gm.k_page, k_blk_bytes);
+      prefetch_l2(gm.zks[gi] + (size_t)ppg * gm.ks_page, (uint32_t)(a.P * a.ks_row));
+      prefetch_l2(gm.zv[gi] + (size_t)ppg * gm.v_page, (uint32_t)(a.P * a.v_row));
+      prefetch_l2(gm.zvs[gi] + (size_t)ppg * gm.vs_page, (uint32_t)(a.P * a.vs_row));
+    };
+    // pg = the raw table entry of chunk n's tile, read a tile earlier
+    auto issue = [&](int n, Slot& sl, int pg) {
       if (n >= N) return;
-      const int k = n >> 2;
-      int pg = page_of(a, b, tr.t_begin / kTile + k);
-      if (pg < 0) {
+      if (!page_valid(a, pg)) {
         if ((n & 3) == 0 && zt == 0) report(st, PALU_ERR_DEVICE_BOUNDS, 2000000 + b);
         pg = 0;   // keep the pipeline fed from a valid page; the status says the result is void
-      }
-      if ((n & 3) == 0 && zt == 0) {
-        for (int kk = (k == 0 ? 1 : k + kPrefetch); kk <= k + kPrefetch && kk < tr.ntiles; ++kk) {
-          const int ppg = page_of(a, b, tr.t_begin / kTile + kk);
-          if (ppg < 0) continue;
-          prefetch_l2(gm.zk[gi] + (size_t)ppg * gm.k_page, k_blk_bytes);
-          prefetch_l2(gm.zks[gi] + (size_t)ppg * gm.ks_page, (uint32_t)(a.P * a.ks_row));
-          prefetch_l2(gm.zv[gi] + (size_t)ppg * gm.v_page, (uint32_t)(a.P * a.v_row));
-          prefetch_l2(gm.zvs[gi] + (size_t)ppg * gm.vs_page, (uint32_t)(a.P * a.vs_row));
-        }
       }
       const uint8_t* blk = gm.zk[gi] + (size_t)pg * gm.k_page;
       const uint8_t* sblk = gm.zks[gi] + (size_t)pg * gm.ks_page;
@@ -383,18 +386,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       return true;
     };
     Slot s0, s1, s2, s3;
-    issue(0, s0);
-    issue(1, s1);
-    issue(2, s2);
+    for (int kk = 1; kk <= kPrefetch; ++kk) prefetch_page(page_ahead(a, b, tr, kk));
+    int pg_k = page_ahead(a, b, tr, 0);                // tile k (chunks n .. n+3)
+    int pg_k1 = page_ahead(a, b, tr, 1);               // tile k+1
+    int pf = page_ahead(a, b, tr, 1 + kPrefetch);      // tile k+1+kPrefetch, pulled into L2
+    issue(0, s0, pg_k);
+    issue(1, s1, pg_k);
+    issue(2, s2, pg_k);
     for (int n = 0; n < N && !*abort_flag; n += 4) {
-      issue(n + 3, s3);
+      const int k = n >> 2;
+      const int pg_k2 = page_ahead(a, b, tr, k + 2);                 // in flight during this tile
+      const int pf_next = page_ahead(a, b, tr, k + 2 + kPrefetch);
+      issue(n + 3, s3, pg_k);
       if (!consume(n, s0)) break;
-      issue(n + 4, s0);
+      prefetch_page(pf);
+      issue(n + 4, s0, pg_k1);
       if (!consume(n + 1, s1)) break;
-      issue(n + 5, s1);
+      issue(n + 5, s1, pg_k1);
       if (!consume(n + 2, s2)) break;
-      issue(n + 6, s2);
+      issue(n + 6, s2, pg_k1);
       if (!consume(n + 3, s3)) break;
+      pg_k = pg_k1;
+      pg_k1 = pg_k2;
+      pf = pf_next;
     }
   } else if (kInt4 && warp == 2) {
     // ============================================================ int4 value codes (warp 2)
@@ -405,19 +419,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     // are written PAIRED: row r of the value operand holds entry paired_row(r).
     const int nv_tiles = tr.ntiles - (tr.ragged_last ? 1 : 0);
     const uint32_t vraw = base + L.vraw;
-    auto load_raw = [&](int k) {
-      int pg = page_of(a, b, tr.t_begin / kTile + k);
-      if (pg < 0) pg = 0;   // reported by the key producer
+    auto load_raw = [&](int pg) {   // pg = raw table entry, read a tile earlier
+      if (!page_valid(a, pg)) pg = 0;   // reported by the key producer
       mbar_expect_tx(bar(BAR_VRAW), kVRawBytes);
       bulk_load(vraw, gm.zv[gi] + (size_t)pg * gm.v_page, 128 * 128, bar(BAR_VRAW));
       bulk_load(vraw + 128 * 128, gm.zvs[gi] + (size_t)pg * gm.vs_page, 128 * 16,
                 bar(BAR_VRAW));
     };
-    if (lane == 0 && nv_tiles > 0) load_raw(0);
+    if (lane == 0 && nv_tiles > 0) load_raw(page_ahead(a, b, tr, 0));
+    int pg_next = page_ahead(a, b, tr, 1);
     int stage = 0;
     uint32_t phase = 0;
     const int x = lane & 7, ub = (lane >> 3) & 1, tg = lane >> 4;
     for (int k = 0; k < nv_tiles && !*abort_flag; ++k) {
+      const int pg_after = page_ahead(a, b, tr, k + 2);   // in flight during this tile
       if (!mbar_wait(bar(BAR_VRAW), k & 1, abort_flag, st, 14)) break;
       bool ok = true;
       for (int sidx = 0; sidx < 2 * NRV; ++sidx) {   // column block 2mb + cb of the page
@@ -443,7 +458,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // every lane has read this page's codes: refill the buffer with the next page
       fence_proxy_async();
       __syncwarp();
-      if (lane == 0 && k + 1 < nv_tiles) load_raw(k + 1);
+      if (lane == 0 && k + 1 < nv_tiles) load_raw(pg_next);
+      pg_next = pg_after;
     }
   } else if (warp == 0) {
     // ============================================================ z_k producer (bulk copies)
@@ -453,20 +469,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Pull the next pages of this split into L2 ahead of the TMA loads: the
       // shared-memory ring is only a few chunks deep, so HBM latency is hidden
       // in L2 instead.
-      auto prefetch_page = [&](int kk) {
-        if (kk >= tr.ntiles) return;
-        const int ppg = page_of(a, b, tr.t_begin / kTile + kk);
-        if (ppg < 0) return;
+      auto prefetch_page = [&](int ppg, int kk) {   // ppg = raw table entry of tile kk
+        if (!page_valid(a, ppg)) return;
         prefetch_l2(gm.zk[gi] + (size_t)ppg * gm.k_page, k_blk_bytes);
         if (!(tr.ragged_last && kk == tr.ntiles - 1))
           prefetch_l2(gm.zv[gi] + (size_t)ppg * gm.v_page, (uint32_t)(a.P * a.v_row));
       };
-      for (int kk = 0; kk < kPrefetch; ++kk) prefetch_page(kk);
+      for (int kk = 0; kk < kPrefetch; ++kk) prefetch_page(page_ahead(a, b, tr, kk), kk);
+      int pg_next = page_ahead(a, b, tr, 0), pf_next = page_ahead(a, b, tr, kPrefetch);
       for (int k = 0; k < tr.ntiles && !*abort_flag; ++k) {
-        prefetch_page(k + kPrefetch);
-        const int lp = tr.t_begin / kTile + k;
-        int pg = page_of(a, b, lp);
-        if (pg < 0) {
+        int pg = pg_next;
+        const int pf = pf_next;
+        pg_next = page_ahead(a, b, tr, k + 1);   // in flight during this tile's copies
+        pf_next = page_ahead(a, b, tr, k + 1 + kPrefetch);
+        prefetch_page(pf, k + kPrefetch);
+        if (!page_valid(a, pg)) {
           report(st, PALU_ERR_DEVICE_BOUNDS, 2000000 + b);
           pg = 0;   // keep the pipeline fed from a valid page; the status says the result is void
         }
@@ -487,11 +504,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
+      int pg_next = page_ahead(a, b, tr, 0);
       for (int k = 0; k < tr.ntiles && !*abort_flag; ++k) {
         if (tr.ragged_last && k == tr.ntiles - 1) break;    // CUDA-core value sum for a partial page
-        const int lp = tr.t_begin / kTile + k;
-        int pg = page_of(a, b, lp);
-        if (pg < 0) pg = 0;   // reported by the z_k producer
+        int pg = pg_next;
+        pg_next = page_ahead(a, b, tr, k + 1);   // in flight during this tile's copies
+        if (!page_valid(a, pg)) pg = 0;   // reported by the z_k producer
         const uint8_t* src = gm.zv[gi] + (size_t)pg * gm.v_page;
         // one copy per 128-byte column block of the page (64 latent entries of
         // all 128 tokens); two consecutive blocks are the two MN-blocks of one
@@ -515,44 +533,48 @@ __global__ void __launch_bounds__(kThreads, 1)
       int zs = 0;
       uint32_t zph = 0, vph = 0;
       bool ok = mbar_wait(bar(BAR_B), 0, abort_flag, st, 20);
-      int pv_pending = -1;   // tile whose value MMA waits for its P
+      int pv_pending = -1;   // tile whose value MMA (aᵀ[r_v × 16] = z_vᵀ · Pᵀ) is not yet issued
+      int pv_mb = 0;         // next 128-entry block of that value MMA
 
-      // aᵀ[r_v × 16] = z_vᵀ · Pᵀ for tile j into its (drained) D slot
-      auto issue_pv = [&](int j) -> bool {
+      // aᵀ[128 entries × 16] of block pv_mb for tile pv_pending = z_vᵀ · Pᵀ into
+      // the tile's (drained) D slot; its P and both ring stages are in
+      auto issue_pv_block = [&]() {
+        const int j = pv_pending;
         tc_fence_after();
         const uint32_t a_tmem = tmem + (uint32_t)(j & 1) * 256;
         const uint32_t p_base = base + L.p + (uint32_t)(j & 1) * kPBytes;
         static_assert(kNVS == 2, "one value MMA operand = the two ring stages");
-        for (int mb = 0; mb < NRV; ++mb) {
-          for (int cb = 0; cb < 2; ++cb)
-            if (!mbar_wait(bar(BAR_ZV_FULL + cb), vph, abort_flag, st, 22)) return false;
-          tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < kTile / 16; ++kk) {
-            // rows = latent entries (two 64-entry blocks, one per stage), K = tokens
-            const uint64_t ad = sdesc(base + L.zv + kk * 16 * 128, kZvBytes, 1024, kSw128);
-            const uint64_t bd = sdesc(p_base + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024, kSw128);
-            umma_f16(a_tmem + mb * 16, ad, bd, idesc_pv, kk != 0);
-          }
-          umma_commit(bar(BAR_ZV_EMPTY + 0));
-          umma_commit(bar(BAR_ZV_EMPTY + 1));
-          vph ^= 1;
+        for (int kk = 0; kk < kTile / 16; ++kk) {
+          // rows = latent entries (two 64-entry blocks, one per stage), K = tokens
+          const uint64_t ad = sdesc(base + L.zv + kk * 16 * 128, kZvBytes, 1024, kSw128);
+          const uint64_t bd = sdesc(p_base + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024, kSw128);
+          umma_f16(a_tmem + pv_mb * 16, ad, bd, idesc_pv, kk != 0);
         }
-        umma_commit(bar(BAR_AT_FULL));
-        trace(2, j);
-        pv_pending = -1;
-        return true;
+        umma_commit(bar(BAR_ZV_EMPTY + 0));
+        umma_commit(bar(BAR_ZV_EMPTY + 1));
+        vph ^= 1;
+        if (++pv_mb == NRV) {
+          umma_commit(bar(BAR_AT_FULL));
+          trace(2, j);
+          pv_pending = -1;
+          pv_mb = 0;
+        }
       };
-      // Wait for z_k data; meanwhile issue the pending value MMA as soon as its
-      // P is ready, so the epilogue gets its latent sums early.  Bounded.
+      // The next block of the pending value MMA can go (its P and z_v are in)?
+      auto pv_ready = [&]() -> bool {
+        return pv_pending >= 0 &&
+               (pv_mb > 0 || mbar_test_wait(bar(BAR_P_FULL + (pv_pending & 1)), (pv_pending >> 1) & 1)) &&
+               mbar_test_wait(bar(BAR_ZV_FULL + 0), vph) && mbar_test_wait(bar(BAR_ZV_FULL + 1), vph);
+      };
+      // Wait for z_k data; meanwhile issue each block of the pending value MMA
+      // as soon as its P and z_v are in (never blocking on them, so key chunks
+      // keep flowing while the value operand is still being filled).  Bounded.
       auto wait_zk = [&]() -> bool {
         const long long t0 = clock64();
         while (true) {
           if (mbar_test_wait(bar(BAR_ZK_FULL + zs), zph)) return true;
-          if (pv_pending >= 0 &&
-              mbar_test_wait(bar(BAR_P_FULL + (pv_pending & 1)), (pv_pending >> 1) & 1)) {
-            if (!issue_pv(pv_pending)) return false;
-          }
+          if (pv_ready()) issue_pv_block();
           if (*abort_flag) return false;
           __nanosleep(64);   // leave the issue slots of this SM partition to the epilogue warps
           if (clock64() - t0 > kWaitCycles) {
@@ -562,11 +584,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       };
+      // Issue what is left of the pending value MMA, waiting for its operands.  Bounded.
       auto flush_pv = [&]() -> bool {
-        if (pv_pending < 0) return true;
-        if (!mbar_wait(bar(BAR_P_FULL + (pv_pending & 1)), (pv_pending >> 1) & 1, abort_flag, st, 21))
-          return false;
-        return issue_pv(pv_pending);
+        while (pv_pending >= 0) {
+          if (pv_mb == 0 &&
+              !mbar_wait(bar(BAR_P_FULL + (pv_pending & 1)), (pv_pending >> 1) & 1, abort_flag, st, 21))
+            return false;
+          for (int cb = 0; cb < 2; ++cb)
+            if (!mbar_wait(bar(BAR_ZV_FULL + cb), vph, abort_flag, st, 22)) return false;
+          issue_pv_block();
+        }
+        return true;
       };
 
       for (int k = 0; k < tr.ntiles && ok; ++k) {

@@ -385,30 +385,36 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (++stage == kNZK) { stage = 0; phase ^= 1; }
       return true;
     };
-    Slot s0, s1, s2, s3;
+    Slot s0, s1, s2, s3;                               // chunks n, n+1, n+2; s3 takes n+3
     for (int kk = 1; kk <= kPrefetch; ++kk) prefetch_page(page_ahead(a, b, tr, kk));
-    int pg_k = page_ahead(a, b, tr, 0);                // tile k (chunks n .. n+3)
+    int pg_k = page_ahead(a, b, tr, 0);                // tile k of chunk n
     int pg_k1 = page_ahead(a, b, tr, 1);               // tile k+1
+    int pg_k2 = page_ahead(a, b, tr, 2);               // tile k+2, in flight
     int pf = page_ahead(a, b, tr, 1 + kPrefetch);      // tile k+1+kPrefetch, pulled into L2
     issue(0, s0, pg_k);
     issue(1, s1, pg_k);
     issue(2, s2, pg_k);
-    for (int n = 0; n < N && !*abort_flag; n += 4) {
-      const int k = n >> 2;
-      const int pg_k2 = page_ahead(a, b, tr, k + 2);                 // in flight during this tile
-      const int pf_next = page_ahead(a, b, tr, k + 2 + kPrefetch);
-      issue(n + 3, s3, pg_k);
+    // One load batch and one conversion per chunk, the register slots shifted
+    // down after each: a single copy of the conversion code keeps the kernel's
+    // instruction footprint small (the warps of a sub-partition run different
+    // roles, so an unrolled copy per slot thrashed the instruction cache).
+#pragma unroll 1
+    for (int n = 0; n < N && !*abort_flag; ++n) {
+      const int c = n & 3;
+      if (c == 0 && n > 0) {
+        pg_k = pg_k1;
+        pg_k1 = pg_k2;
+        pg_k2 = page_ahead(a, b, tr, (n >> 2) + 2);
+      }
+      issue(n + 3, s3, c == 0 ? pg_k : pg_k1);
       if (!consume(n, s0)) break;
-      prefetch_page(pf);
-      issue(n + 4, s0, pg_k1);
-      if (!consume(n + 1, s1)) break;
-      issue(n + 5, s1, pg_k1);
-      if (!consume(n + 2, s2)) break;
-      issue(n + 6, s2, pg_k1);
-      if (!consume(n + 3, s3)) break;
-      pg_k = pg_k1;
-      pg_k1 = pg_k2;
-      pf = pf_next;
+      if (c == 0) {
+        prefetch_page(pf);
+        pf = page_ahead(a, b, tr, (n >> 2) + 2 + kPrefetch);
+      }
+      s0 = s1;
+      s1 = s2;
+      s2 = s3;
     }
   } else if (kInt4 && warp == 2) {
     // ============================================================ int4 value codes (warp 2)
@@ -439,7 +445,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(bar(BAR_ZV_EMPTY + stage), phase ^ 1, abort_flag, st, 13)) { ok = false; break; }
         const uint32_t dst = base + L.zv + stage * kZvBytes;
         const int u = 2 * sidx + ub;
-#pragma unroll 4
+#pragma unroll 2
         for (int i = 0; i < 8; ++i) {
           const int t = x + 8 * (2 * i + tg);
           const uint4 raw = ld_shared_v4(vraw + t * 128 + ((u ^ x) << 4));

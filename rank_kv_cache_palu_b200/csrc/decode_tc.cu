@@ -248,7 +248,10 @@ __device__ __forceinline__ void trace_record(const DecodeArgs& a, int ev, int k,
   a.trace[(cta * 8 + ev) * a.trace_tiles + k] = clock64() - t_start;
 }
 
-template <int ACT, int NRV, int LAT>
+// CONTIG: token positions are the cache slots (no position pool).  A separate
+// instantiation keeps the per-token sincos path of explicit positions out of
+// the score loop's instruction footprint.
+template <int ACT, int NRV, int LAT, bool CONTIG>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tm_bk, const __grid_constant__ DecodeArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -685,7 +688,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // tile base at t0 (one sincos per warp lane per tile) and this thread's
     // fixed offset `row`, by angle addition; explicit positions take a sincos
     // per token.  Math runs on packed fp32 pairs (two frequencies at a time).
-    const bool contig = a.pos_pool == nullptr;
+    constexpr bool contig = CONTIG;
     float* tbw = reinterpret_cast<float*>(sbase + L.tb) + (warp - 4) * 96;   // [cos|sin|-sin][32]
     f2 crow[16], srow[16];
     if (contig) {
@@ -978,7 +981,7 @@ cudaError_t launch_t(const DecodeArgs& a, cudaStream_t st) {
     return cudaErrorInvalidValue;
   const Smem L = smem_layout(a.r_k, LAT == PALU_INT4);
   const size_t smem = L.total + 1024;
-  auto kern = decode_tc_kernel<ACT, NRV, LAT>;
+  auto kern = a.pos_pool == nullptr ? decode_tc_kernel<ACT, NRV, LAT, true> : decode_tc_kernel<ACT, NRV, LAT, false>;
   DecodeArgs args = a;
   const TraceSetting ts = trace_setting();
   const size_t ctas = (size_t)a.S * a.gm.n * (a.gs / 2) * a.batch;

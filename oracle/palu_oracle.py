@@ -20,7 +20,7 @@ Sources (cited by page title and section):
   v2 abstract): medium-grained (group-head) decomposition, RoPE-based
   attention, quantisation compatibility.
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent (the oracle and the kernels take the same ones):
 
 * heads are grouped consecutively, group_size heads per group; head h uses
   columns [(h mod g)·d_h, +d_h) of its group's B;

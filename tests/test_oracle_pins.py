@@ -429,9 +429,32 @@ def test_int4_error_bound_and_roundtrip():
     sb = np.repeat(s.astype(np.float64), 32, axis=-1)
     # |z - code*s| <= s/2 (+ the tiny overshoot of fp16 scale rounding, + fp16 rounding of the product)
     assert np.all(np.abs(z - deq) <= 0.5 * sb * (1 + 2 ** -9) + np.abs(deq) * 2 ** -11 + 1e-12)
-    # re-quantising the dequantised codes (fp32 product) reproduces them
     codes = O.unpack_int4(packed)
     assert codes.min() >= -7 and codes.max() <= 7
+    # Re-quantising code*s (exact in float32: an 11-bit scale times a 3-bit code) gives the same
+    # bytes and scales back.  With a normal fp16 scale, max|z|/s rounds to 7, so the largest code
+    # of every block is +-7 and the block's new maximum 7*s divides back to s exactly.
+    assert np.all(np.abs(s.astype(np.float32)) >= np.float32(2.0 ** -14))
+    z2 = (codes.reshape(5, 9, 8, 32).astype(np.float32) * s.astype(np.float32)[..., None]).reshape(5, 9, 256)
+    packed2, s2 = O.quantize_int4(z2)
+    np.testing.assert_array_equal(packed2, packed)
+    np.testing.assert_array_equal(s2.view(np.uint16), s.view(np.uint16))
+    assert np.all(np.max(np.abs(codes.reshape(5, 9, 8, 32)), axis=-1) == 7)
+
+
+def test_int4_cache_bytes_hand_count():
+    # r_k = r_v = 256 per group, int4: 128 bytes of codes per side (two entries a byte) and
+    # 256/32 = 8 fp16 scales per side -> 2*128 + 2*8*2 = 288 bytes per (token, group); 8 groups.
+    latent, full = O.cache_bytes_per_token(32, 128, 4, 256, 256, "int4")
+    assert latent == 8 * 288
+    assert full == 2 * 32 * 128 * 2                       # fp16 K and V of 32 heads x 128
+    # the same count from what the quantiser actually emits for one token of one group
+    z = rng(21).standard_normal((2, 1, 256)).astype(np.float32)
+    packed, s = O.quantize_int4(z)
+    assert packed.nbytes + s.nbytes == 288
+    # unequal ranks and another group count: 8 groups x ((128 + 384)/2 + (4 + 12)*2) bytes
+    latent, _ = O.cache_bytes_per_token(32, 128, 4, 128, 384, "int4")
+    assert latent == 8 * (256 + 32)
 
 
 # ----------------------------------------------------------------- compression ratio (printed value)

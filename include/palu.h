@@ -98,7 +98,8 @@ palu_status palu_cache_strides(const palu_config* cfg, size_t* k_page_bytes, siz
 /* Workspace bytes palu_compress_append needs for n_tokens rows (status word +
  * per-split partial sums and counters when the K range is split across CTAs).
  * Always >= 256.  Zero-fill a workspace once before its first use; every call
- * leaves its counters back at zero. */
+ * leaves its counters back at zero (after a call whose kernels reported
+ * PALU_ERR_DEVICE_TIMEOUT, zero-fill it again). */
 palu_status palu_compress_workspace_size(const palu_config* cfg, int n_tokens, int d_model,
                                          size_t* bytes);
 
@@ -266,7 +267,9 @@ palu_status palu_decode_attn_ranked(const palu_config* cfg, const int32_t* ranks
  *     return PALU_ERR_WORKSPACE before launching anything.
  *   - The first call on a device looks up the array's device address for that
  *     device (cudaGetSymbolAddress, with that device current); make that first
- *     call before any stream capture.
+ *     call before any stream capture.  Only a successful lookup is kept: a
+ *     call whose lookup failed returns PALU_ERR_CUDA and the next call on that
+ *     device tries again.
  *   - Every call on a device shares the one array and leaves its contents
  *     behind; each call clears the status word (an asynchronous memset on
  *     `stream`) and rewrites all partials.  Calls that overlap on the GPU (on
@@ -319,6 +322,22 @@ int palu_decode_kernel_kind(const palu_config* cfg);
  * setting, not thread-safe with concurrent decode calls. */
 #define PALU_TRACE_EVENTS 8
 palu_status palu_debug_trace(void* buffer, size_t bytes, int tiles_per_cta);
+
+/* Test hook for the kernels' timeout path: every wait inside the tensor-core
+ * kernels (compress and decode) is bounded, and on expiry the kernel records
+ * PALU_ERR_DEVICE_TIMEOUT in the workspace status word, waits (with a bound of
+ * its own) for the copies and MMAs it has already issued, frees its tensor
+ * memory and returns, leaving the context usable.  The call's outputs are then
+ * void; a compress workspace must be zero-filled again before its next use.
+ *   wait_cycles  bound of each wait in SM clock cycles for launches after this
+ *                call; 0 = the default (2^31 cycles, about a second at 2 GHz)
+ *   stall        non-zero: the MMA thread of every tensor-core launch first
+ *                waits on a barrier phase that nothing completes before its
+ *                own teardown, so every such launch runs out that bound
+ * palu_debug_timeout_test(0, 0) restores normal operation.  Process-wide, not
+ * thread-safe with concurrent calls; meant for tests only.  Returns
+ * PALU_ERR_INVALID_ARG for a negative wait_cycles. */
+palu_status palu_debug_timeout_test(int64_t wait_cycles, int stall);
 
 /* Number of CUDA kernels this library has launched in this process (all
  * entry points, all devices).  A monotone counter for instrumentation. */

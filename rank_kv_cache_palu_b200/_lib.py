@@ -74,6 +74,7 @@ SIGNATURES = {
     "palu_decode_kernel_kind": (c_int, [_CFG]),
     "palu_kernel_launches": (ctypes.c_uint64, []),
     "palu_debug_trace": (c_int, [c_void_p, c_size_t, c_int]),
+    "palu_debug_timeout_test": (c_int, [ctypes.c_int64, c_int]),
 }
 
 _lock = threading.Lock()

@@ -109,6 +109,13 @@ def palu_debug_trace(buffer, tiles_per_cta: int = 0) -> None:
                                        tiles_per_cta), "palu_debug_trace")
 
 
+def palu_debug_timeout_test(wait_cycles: int = 0, stall: bool = False) -> None:
+    """Test hook of the kernels' timeout path: bound every wait of later tensor-core
+    launches to wait_cycles SM cycles (0 = the default) and, with stall, make each
+    such launch run that bound out.  palu_debug_timeout_test() restores normal operation."""
+    _check(load().palu_debug_timeout_test(int(wait_cycles), 1 if stall else 0), "palu_debug_timeout_test")
+
+
 def palu_compress_append(cfg: PaluConfig, x, A_k, A_v, slot_mapping, positions, zk_pool, zv_pool,
                          zk_scales, zv_scales, pos_pool, num_pages: int, workspace, stream=None):
     n, d_model = x.shape

@@ -164,6 +164,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto empty = [&](int s) { return bars + 8u * (p.stages + s); };
   const uint32_t d_full = bars + 8u * (2 * p.stages);
   const uint32_t epi_bar = d_full + 8;
+  const uint32_t td_bar = d_full + 16;   // teardown: every MMA of the CTA has completed
   DevStatus* st = reinterpret_cast<DevStatus*>(a.status);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -180,13 +181,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const CUtensorMap* tm_a = is_v ? &tm_av : &tm_ak;
 
   if (threadIdx.x == 0) {
-    *abort_flag = 0;
+    abort_init(abort_flag, a.wait_cycles);
     for (int s = 0; s < p.stages; ++s) {
       mbar_init(full(s), 1);
       mbar_init(empty(s), 1);
     }
     mbar_init(d_full, 1);
     mbar_init(epi_bar, 4);
+    mbar_init(td_bar, 1);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -207,6 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the tile's two 64-column boxes of A, fixed over the K loop
       const uint16_t* row0 = is_v ? a.gm.v_row0 : a.gm.k_row0;
       const int ax0 = a_column(a.gm, cols, row0, c0), ax1 = a_column(a.gm, cols, row0, c0 + 64);
+      long long issued = 0;
       for (int kb = ks0; kb < ks1 && !*abort_flag; ++kb) {
         if (!mbar_wait(empty(s), ph ^ 1, abort_flag, st, 50)) break;
         mbar_expect_tx(full(s), (uint32_t)stage_bytes);
@@ -214,8 +217,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_2d(dst, tm_a, ax0, kb * kKStage, full(s));
         tma_load_2d(dst + kABytes / 2, tm_a, ax1, kb * kKStage, full(s));
         tma_load_2d(dst + kABytes, &tm_x, kb * kKStage, t0, full(s));
+        ++issued;
         if (++s == p.stages) { s = 0; ph ^= 1; }
       }
+      // after an abort, loads already issued still land in shared memory: wait for them
+      drain_ring(full(0), p.stages, issued, st, 50);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -223,8 +229,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc = idesc_f16(kBf, 1, 0, p.NT, kM);    // Aᵀ MN-major, xᵀ K-major
       int s = 0;
       uint32_t ph = 0;
-      bool ok = true;
-      for (int kb = ks0; kb < ks1; ++kb) {
+      // timeout-path test hook: first wait on a phase nothing completes before the teardown commit
+      bool ok = a.stall_test == 0 || mbar_wait(td_bar, 0, abort_flag, st, 55);
+      for (int kb = ks0; kb < ks1 && ok; ++kb) {
         if (!mbar_wait(full(s), ph, abort_flag, st, 51)) { ok = false; break; }
         tc_fence_after();
         const uint32_t sa = base + (uint32_t)s * stage_bytes;
@@ -238,8 +245,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_commit(empty(s));
         if (++s == p.stages) { s = 0; ph ^= 1; }
       }
-      (void)ok;
-      umma_commit(d_full);   // also drains: fires once every MMA above has completed
+      if (ok) umma_commit(d_full);   // fires once every MMA above has completed
+      // drain, also after an abort: every MMA issued completes before TMEM is released
+      umma_commit(td_bar);
+      mbar_drain(td_bar, 0, st, 56);
     }
   } else {
     // ============================================================ epilogue (warps 2-5)
@@ -275,7 +284,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       __threadfence();
       ok = ep_sync(53) && ok;
       if (threadIdx.x == 64) {
-        const int prev = atomicAdd(t.counters + tile_id, 1);
+        // a CTA that gave up neither counts itself nor closes the tile
+        const int prev = ok ? atomicAdd(t.counters + tile_id, 1) : -1;
         *last_flag = (prev == p.KS - 1);
       }
       ok = ep_sync(54) && ok;
@@ -351,6 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto empty = [&](int s) { return bars + 8u * (p.stages + s); };
   auto acc_full = [&](int b) { return bars + 8u * (2 * p.stages + b); };
   auto acc_empty = [&](int b) { return bars + 8u * (2 * p.stages + 2 + b); };
+  const uint32_t td_bar = bars + 8u * (2 * p.stages + 4);   // teardown: every MMA has completed
   DevStatus* st = reinterpret_cast<DevStatus*>(a.status);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ctiles = p.tk + p.tv;
@@ -368,7 +379,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int my_tiles = blockIdx.x < ntiles ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
 
   if (threadIdx.x == 0) {
-    *abort_flag = 0;
+    abort_init(abort_flag, a.wait_cycles);
     for (int s = 0; s < p.stages; ++s) {
       mbar_init(full(s), 1);
       mbar_init(empty(s), 1);
@@ -377,6 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(acc_full(b), 1);
       mbar_init(acc_empty(b), 4);
     }
+    mbar_init(td_bar, 1);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -396,6 +408,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int s = 0;
       uint32_t ph = 0;
       bool ok = true;
+      long long issued = 0;
       for (int i = 0; i < my_tiles && ok; ++i) {
         int ctile, c0, t0;
         bool is_v;
@@ -411,9 +424,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d(dst, tm_a, ax0, kb * kKStage, full(s));
           tma_load_2d(dst + kABytes / 2, tm_a, ax1, kb * kKStage, full(s));
           tma_load_2d(dst + kABytes, &tm_x, kb * kKStage, t0, full(s));
+          ++issued;
           if (++s == p.stages) { s = 0; ph ^= 1; }
         }
       }
+      // after an abort, loads already issued still land in shared memory: wait for them
+      drain_ring(full(0), p.stages, issued, st, 60);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -421,11 +437,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc = idesc_f16(kBf, 1, 0, p.NT, kM);    // Aᵀ MN-major, xᵀ K-major
       int s = 0;
       uint32_t ph = 0;
-      bool ok = true;
+      // timeout-path test hook: first wait on a phase nothing completes before the teardown commit
+      bool ok = a.stall_test == 0 || mbar_wait(td_bar, 0, abort_flag, st, 65);
       for (int i = 0; i < my_tiles && ok; ++i) {
         const int b = i & 1;
         // the epilogue has read this accumulator's previous tile (i - 2)
-        if (!mbar_wait(acc_empty(b), ((i >> 1) & 1) ^ 1, abort_flag, st, 61)) break;
+        if (!mbar_wait(acc_empty(b), ((i >> 1) & 1) ^ 1, abort_flag, st, 61)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d = tmem + 256u * b;
         for (int kb = 0; kb < kst; ++kb) {
@@ -442,10 +459,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           umma_commit(empty(s));
           if (++s == p.stages) { s = 0; ph ^= 1; }
         }
+        if (!ok) break;
         umma_commit(acc_full(b));   // fires once every MMA of the tile has completed
       }
-      // drain before TMEM is released
-      if (my_tiles > 0) mbar_wait(acc_full((my_tiles - 1) & 1), ((my_tiles - 1) >> 1) & 1, abort_flag, st, 63);
+      // drain, also after an abort: every MMA issued completes before TMEM is released
+      umma_commit(td_bar);
+      mbar_drain(td_bar, 0, st, 63);
     }
   } else {
     // ============================================================ epilogue (warps 2-5)

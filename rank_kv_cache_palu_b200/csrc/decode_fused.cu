@@ -229,7 +229,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nvt = ntiles - (ragged_last ? 1 : 0);   // tiles whose value sum runs on the tensor cores
 
   if (threadIdx.x == 0) {
-    *abort_flag = 0;
+    abort_init(abort_flag, a.wait_cycles);
     for (int i = 0; i < kNZK; ++i) {
       mbar_init(bar(BAR_ZK_FULL + i), 1);
       mbar_init(bar(BAR_ZK_EMPTY + i), 1);
@@ -281,6 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       int zs = 0, vs = 0;
       uint32_t zph = 0, vph = 0;
+      long long zk_issued = 0, zv_issued = 0;
       // z_v of a tile is needed only after its scores: stream it one tile behind
       // z_k, so the two rings fill in the order the MMAs consume them
       auto push_zv = [&](int k) -> bool {
@@ -291,6 +292,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mbar_wait(bar(BAR_ZV_EMPTY + vs), vph ^ 1, abort_flag, st, 11)) return false;
           mbar_expect_tx(bar(BAR_ZV_FULL + vs), kStageBytes);
           bulk_load(base + L.zv + vs * kStageBytes, src + (size_t)cb * a.P * 128, kStageBytes, bar(BAR_ZV_FULL + vs));
+          ++zv_issued;
           if (++vs == kNZV) { vs = 0; vph ^= 1; }
         }
         return true;
@@ -307,11 +309,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mbar_wait(bar(BAR_ZK_EMPTY + zs), zph ^ 1, abort_flag, st, 10)) { ok = false; break; }
           mbar_expect_tx(bar(BAR_ZK_FULL + zs), kStageBytes);
           bulk_load(base + L.zk + zs * kStageBytes, src + (size_t)c * kStageBytes, kStageBytes, bar(BAR_ZK_FULL + zs));
+          ++zk_issued;
           if (++zs == kNZK) { zs = 0; zph ^= 1; }
         }
         if (ok && k >= 1 && k - 1 < nvt) ok = push_zv(k - 1);
       }
       if (ok && ntiles >= 1 && ntiles - 1 < nvt) push_zv(ntiles - 1);
+      // after an abort, copies already issued still land in shared memory: wait for them
+      drain_ring(bar(BAR_ZK_FULL), kNZK, zk_issued, st, 10);
+      drain_ring(bar(BAR_ZV_FULL), kNZV, zv_issued, st, 11);
     }
   } else if (warp == 1) {
     // ============================================================ MMA issuer
@@ -321,7 +327,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc_pv = idesc_f16(kBf, 1, 0, kNP, 128);  // z_vᵀ MN-major, Pᵀ K-major
       int zs = 0, vs = 0;
       uint32_t zph = 0, vph = 0;
-      bool ok = true;
+      // timeout-path test hook: first wait on a phase nothing completes before the teardown commit
+      bool ok = a.stall_test == 0 || mbar_wait(bar(BAR_TEARDOWN), 0, abort_flag, st, 27);
       auto issue_pv = [&](int j) -> bool {
         const uint32_t a_tmem = tmem + PS::kAt + (uint32_t)(j & 1) * NRV * kNP;
         const uint32_t p_base = base + L.p + (uint32_t)(j & 1) * kPB;
@@ -369,8 +376,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (k >= 1 && k - 1 < nvt && !issue_pv(k - 1)) { ok = false; break; }
       }
       if (ok && ntiles >= 1 && ntiles - 1 < nvt) issue_pv(ntiles - 1);
+      // drain, also after an abort: every MMA issued above completes before TMEM is released
       umma_commit(bar(BAR_TEARDOWN));
-      mbar_wait(bar(BAR_TEARDOWN), 0, abort_flag, st, 26);
+      mbar_drain(bar(BAR_TEARDOWN), 0, st, 26);
     }
   } else {
     // ============================================================ epilogue (warps 2-5)

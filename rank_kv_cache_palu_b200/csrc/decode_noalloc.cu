@@ -20,22 +20,25 @@ constexpr size_t kNoAllocScratchBytes = PALU_NOALLOC_SCRATCH_BYTES;
 static __device__ __align__(256) unsigned char g_decode_scratch[kNoAllocScratchBytes];
 
 constexpr int kMaxDevices = 64;
-std::once_flag g_once[kMaxDevices];
+std::mutex g_mutex[kMaxDevices];
 void* g_scratch_ptr[kMaxDevices] = {};
-cudaError_t g_setup_err[kMaxDevices] = {};
 
 // The array's name is only a host-side stand-in in host code: the device
-// address comes from cudaGetSymbolAddress, once per device, with that device
-// current.
+// address comes from cudaGetSymbolAddress, with that device current.  Only a
+// successful lookup is kept; after a failed one (for instance a first call
+// made while the stream was being captured) the next call looks again.
 palu_status scratch_address(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PALU_ERR_CUDA;
-  std::call_once(g_once[dev], [dev] {
+  std::lock_guard<std::mutex> lock(g_mutex[dev]);
+  if (g_scratch_ptr[dev] == nullptr) {
     void* p = nullptr;
-    g_setup_err[dev] = cudaGetSymbolAddress(&p, g_decode_scratch);
-    g_scratch_ptr[dev] = (g_setup_err[dev] == cudaSuccess) ? p : nullptr;
-  });
-  if (g_setup_err[dev] != cudaSuccess || g_scratch_ptr[dev] == nullptr) return PALU_ERR_CUDA;
+    if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr) {
+      (void)cudaGetLastError();   // do not leave the failed lookup as this thread's sticky error
+      return PALU_ERR_CUDA;
+    }
+    g_scratch_ptr[dev] = p;
+  }
   *out = g_scratch_ptr[dev];
   return PALU_OK;
 }

@@ -282,7 +282,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ---------------------------------------------------------------- setup
   if (threadIdx.x == 0) {
-    *abort_flag = 0;
+    abort_init(abort_flag, a.wait_cycles);
     mbar_init(bar(BAR_B), 1);
     for (int i = 0; i < kNZK; ++i) {
       mbar_init(bar(BAR_ZK_FULL + i), kInt4 ? 2 : 1);   // int4: one arrival per dequantising warp
@@ -428,8 +428,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // are written PAIRED: row r of the value operand holds entry paired_row(r).
     const int nv_tiles = tr.ntiles - (tr.ragged_last ? 1 : 0);
     const uint32_t vraw = base + L.vraw;
+    int raw_loads = 0;                // staged pages issued (lane 0); BAR_VRAW phase n completes load n
     auto load_raw = [&](int pg) {   // pg = raw table entry, read a tile earlier
       if (!page_valid(a, pg)) pg = 0;   // reported by the key producer
+      ++raw_loads;
       mbar_expect_tx(bar(BAR_VRAW), kVRawBytes);
       bulk_load(vraw, gm.zv[gi] + (size_t)pg * gm.v_page, 128 * 128, bar(BAR_VRAW));
       bulk_load(vraw + 128 * 128, gm.zvs[gi] + (size_t)pg * gm.vs_page, 128 * 16,
@@ -470,6 +472,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0 && k + 1 < nv_tiles) load_raw(pg_next);
       pg_next = pg_after;
     }
+    // the staging buffer may still be filling after an abort: wait for the last page issued
+    if (lane == 0 && raw_loads > 0) mbar_drain(bar(BAR_VRAW), (uint32_t)((raw_loads - 1) & 1), st, 14);
   } else if (warp == 0) {
     // ============================================================ z_k producer (bulk copies)
     if (lane == 0) {
@@ -486,6 +490,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       for (int kk = 0; kk < kPrefetch; ++kk) prefetch_page(page_ahead(a, b, tr, kk), kk);
       int pg_next = page_ahead(a, b, tr, 0), pf_next = page_ahead(a, b, tr, kPrefetch);
+      long long issued = 0;
       for (int k = 0; k < tr.ntiles && !*abort_flag; ++k) {
         int pg = pg_next;
         const int pf = pf_next;
@@ -503,10 +508,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mbar_wait(bar(BAR_ZK_EMPTY + stage), phase ^ 1, abort_flag, st, 10)) break;
           mbar_expect_tx(bar(BAR_ZK_FULL + stage), kZkBytes);
           bulk_load(base + L.zk + stage * kZkBytes, src + (size_t)c * kZkBytes, kZkBytes, bar(BAR_ZK_FULL + stage));
+          ++issued;
           if (c == 0) trace(6, k);
           if (++stage == kNZK) { stage = 0; phase ^= 1; }
         }
       }
+      drain_ring(bar(BAR_ZK_FULL), kNZK, issued, st, 10);
     }
   } else if (warp == 2) {
     // ============================================================ z_v producer (bulk copies)
@@ -514,6 +521,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       int pg_next = page_ahead(a, b, tr, 0);
+      long long issued = 0;
       for (int k = 0; k < tr.ntiles && !*abort_flag; ++k) {
         if (tr.ragged_last && k == tr.ntiles - 1) break;    // CUDA-core value sum for a partial page
         int pg = pg_next;
@@ -528,9 +536,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_expect_tx(bar(BAR_ZV_FULL + stage), kZvBytes);
           bulk_load(base + L.zv + stage * kZvBytes, src + (size_t)cb * a.P * 128, kZvBytes,
                     bar(BAR_ZV_FULL + stage));
+          ++issued;
           if (++stage == kNVS) { stage = 0; phase ^= 1; }
         }
       }
+      drain_ring(bar(BAR_ZV_FULL), kNVS, issued, st, 11);
     }
   } else if (warp == 1) {
     // ============================================================ MMA issuer
@@ -541,7 +551,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t b_lbo = (uint32_t)r_k * 128;                  // bytes between 64-column blocks of B
       int zs = 0;
       uint32_t zph = 0, vph = 0;
-      bool ok = mbar_wait(bar(BAR_B), 0, abort_flag, st, 20);
+      // timeout-path test hook: first wait on a phase nothing completes before the teardown commit
+      bool ok = a.stall_test == 0 || mbar_wait(bar(BAR_TEARDOWN), 0, abort_flag, st, 26);
+      ok = ok && mbar_wait(bar(BAR_B), 0, abort_flag, st, 20);
       int pv_pending = -1;   // tile whose value MMA (aᵀ[r_v × 16] = z_vᵀ · Pᵀ) is not yet issued
       int pv_mb = 0;         // next 128-entry block of that value MMA
 
@@ -586,7 +598,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (pv_ready()) issue_pv_block();
           if (*abort_flag) return false;
           __nanosleep(64);   // leave the issue slots of this SM partition to the epilogue warps
-          if (clock64() - t0 > kWaitCycles) {
+          if (clock64() - t0 > wait_limit(abort_flag)) {
             report(st, PALU_ERR_DEVICE_TIMEOUT, 24);
             *abort_flag = 1;
             return false;
@@ -635,9 +647,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(tr.ragged_last && k == tr.ntiles - 1)) pv_pending = k;
       }
       if (ok) ok = flush_pv();
-      // drain: every MMA issued above has completed before TMEM is released
+      // drain, also after an abort: every MMA issued above has completed before
+      // TMEM is released, and the B_k load has landed before the CTA exits
       umma_commit(bar(BAR_TEARDOWN));
-      mbar_wait(bar(BAR_TEARDOWN), 0, abort_flag, st, 25);
+      mbar_drain(bar(BAR_TEARDOWN), 0, st, 25);
+      mbar_drain(bar(BAR_B), 0, st, 20);
     }
   } else if (warp >= 4) {
     // ============================================================ epilogue (warps 4-11)

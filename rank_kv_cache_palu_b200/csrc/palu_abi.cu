@@ -15,6 +15,8 @@ namespace palu {
 static std::atomic<unsigned long long> g_launches{0};
 static TraceSetting g_trace{nullptr, 0, 0};
 TraceSetting trace_setting() { return g_trace; }
+static TimeoutTest g_timeout_test{0, 0};
+TimeoutTest timeout_test_setting() { return g_timeout_test; }
 void count_launch(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
 }  // namespace palu
 
@@ -355,6 +357,8 @@ palu_status compress_layer(const Layer& L, int n_tokens, int d_model, const void
   a.status = workspace;
   a.scratch = reinterpret_cast<float*>(static_cast<char*>(workspace) + kStatusBytes);
   a.scratch_bytes = workspace_bytes - kStatusBytes;
+  a.wait_cycles = palu::timeout_test_setting().wait_cycles;
+  a.stall_test = palu::timeout_test_setting().stall;
   a.a_kcols = L.bk_rows;
   a.a_vcols = L.bv_rows;
   a.positions = positions;
@@ -426,6 +430,8 @@ palu_status decode_layer(const Layer& L, int batch, int Q, const void* q, const 
   a.status = workspace;
   a.part = reinterpret_cast<float*>(static_cast<char*>(workspace) + kStatusBytes);
   a.fused_q = static_cast<char*>(workspace) + fused_off;
+  a.wait_cycles = palu::timeout_test_setting().wait_cycles;
+  a.stall_test = palu::timeout_test_setting().stall;
   fill_omega(cfg, a.omega);
 
   const long long qrow = (long long)a.H * a.d_h;       // one query's elements per sequence
@@ -498,6 +504,12 @@ palu_status palu_debug_trace(void* buffer, size_t bytes, int tiles_per_cta) {
 }
 
 uint64_t palu_kernel_launches(void) { return palu::g_launches.load(std::memory_order_relaxed); }
+
+palu_status palu_debug_timeout_test(int64_t wait_cycles, int stall) {
+  if (wait_cycles < 0) return PALU_ERR_INVALID_ARG;
+  palu::g_timeout_test = palu::TimeoutTest{(long long)wait_cycles, stall != 0 ? 1 : 0};
+  return PALU_OK;
+}
 
 palu_status palu_cache_strides(const palu_config* cfg, size_t* k_page_bytes, size_t* v_page_bytes,
                                size_t* k_scale_page_bytes, size_t* v_scale_page_bytes) {

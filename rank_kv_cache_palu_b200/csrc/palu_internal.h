@@ -66,6 +66,9 @@ struct DecodeArgs {
   uint64_t omega[kMaxHalfDim];             // RoPE frequencies as 64-bit fixed-point turns
   long long* trace;                        // phase trace (palu_debug_trace) or NULL
   int trace_tiles;
+  long long wait_cycles;                   // bound of every wait in the tensor-core kernels (SM cycles)
+  int stall_test;                          // timeout-path test: the MMA thread first waits on a phase
+                                           // that nothing completes, so the launch times out
 };
 
 // Phase-trace buffer set by palu_debug_trace (NULL: off).
@@ -95,7 +98,16 @@ struct CompressArgs {
   float* scratch;  // workspace past the status header
   size_t scratch_bytes;
   long long k_row, v_row, ks_row, vs_row;
+  long long wait_cycles;   // as in DecodeArgs
+  int stall_test;
 };
+
+// Wait bound and stall switch of the timeout-path test (palu_debug_timeout_test).
+struct TimeoutTest {
+  long long wait_cycles;   // <= 0: the default (about a second)
+  int stall;
+};
+TimeoutTest timeout_test_setting();
 
 // CUDA-core kernels (any supported dtype; the only path for float32).
 cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t st);

@@ -52,25 +52,69 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Every wait in the tensor-core kernels is bounded: after ~2^31 cycles (about a
-// second) it records PALU_ERR_DEVICE_TIMEOUT with `where`, raises the CTA's
-// abort flag and returns false, so every role can leave its loop and the CTA
-// can release its tensor memory instead of hanging the GPU.
+// Every wait in the tensor-core kernels is bounded: after a limit of SM cycles
+// (about a second by default; a test may set it lower, see DecodeArgs /
+// CompressArgs wait_cycles) it records PALU_ERR_DEVICE_TIMEOUT with `where`,
+// raises the CTA's abort flag and returns false, so every role can leave its
+// loop, wait for its own copies and MMAs in flight, and the CTA can release its
+// tensor memory instead of hanging the GPU.
+//
+// The abort flag and the limit share 16 bytes of shared memory: the flag (int)
+// at +0 and the limit (long long) at +8.
 constexpr long long kWaitCycles = 1LL << 31;
+// Bound of the drain waits at teardown (copies and MMAs already issued always
+// complete on their own; the bound only guards against a broken invariant).
+constexpr long long kDrainCycles = 1LL << 31;
+
+__device__ __forceinline__ void abort_init(volatile int* abort_flag, long long limit) {
+  abort_flag[0] = 0;
+  *reinterpret_cast<volatile long long*>(abort_flag + 2) = limit > 0 ? limit : kWaitCycles;
+}
+__device__ __forceinline__ long long wait_limit(volatile int* abort_flag) {
+  return *reinterpret_cast<volatile long long*>(abort_flag + 2);
+}
 
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                           DevStatus* st, int where) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
+  const long long limit = wait_limit(abort_flag);
   while (true) {
     for (int i = 0; i < 256; ++i)
       if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (clock64() - t0 > kWaitCycles) {
+    if (clock64() - t0 > limit) {
       report(st, PALU_ERR_DEVICE_TIMEOUT, where);
       *abort_flag = 1;
       return false;
     }
+  }
+}
+
+// Teardown wait for work this thread itself issued (a bulk copy, a TMA load, an
+// MMA commit): it ignores the abort flag, since that work completes and writes
+// shared or tensor memory whether or not the CTA gave up.  Detail 90000 + where
+// if even this bound runs out.
+__device__ __forceinline__ bool mbar_drain(uint32_t bar, uint32_t parity, DevStatus* st, int where) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > kDrainCycles) {
+      report(st, PALU_ERR_DEVICE_TIMEOUT, 90000 + where);
+      return false;
+    }
+  }
+  return true;
+}
+
+// Drain a ring of `stages` barriers (8 bytes apart from full0) into which
+// `issued` copies have gone, stage n % stages for copy n: wait for the last
+// copy into each stage to land.  Earlier copies into a stage had landed before
+// the next one could be issued (the producer waits for the stage to be empty).
+__device__ __forceinline__ void drain_ring(uint32_t full0, int stages, long long issued, DevStatus* st,
+                                           int where) {
+  for (int i = 1; i <= stages && i <= issued; ++i) {
+    const long long n = issued - i;
+    mbar_drain(full0 + 8u * (uint32_t)(n % stages), (uint32_t)((n / stages) & 1), st, where);
   }
 }
 

@@ -312,9 +312,10 @@ int palu_decode_kernel_kind(const palu_config* cfg);
  * records, per CTA and per tile (up to `tiles_per_cta`), the SM clock
  * (clock64, relative to the CTA's start) at kPaluTraceEvents points:
  *   0 MMA: slot free, key MMAs of the tile start   1 MMA: key MMAs issued
- *   2 MMA: value MMAs of the previous tile issued  3 epilogue: tile keys ready
+ *   2 MMA: the tile's value MMAs issued            3 epilogue: tile keys ready
  *   4 epilogue: scores done (both warpgroups)      5 epilogue: P written
- *   6 z_k producer: first chunk of the tile issued 7 MMA: first chunk landed
+ *   6 value latents of the tile: first copy issued (int4: codes staged)
+ *   7 MMA thread: the tile's first value-latent block seen in shared memory
  * into `buffer` (device memory, int64 [cta][event][tile], CTA = linear block
  * index); entries never reached stay as they were.  Pass NULL to stop.
  * `bytes` must cover grid CTAs × 8 × tiles_per_cta × 8 bytes of the launches

@@ -16,12 +16,14 @@
 //           rings instead (code × fp16 scale, rounded to the compute dtype),
 //           so the MMAs below are the same for every latent dtype.
 //   warp 1  MMA issuer: D[128 tok × 256] = z_k · B_k[:, 2 heads] into one of two
-//           TMEM slots (kind::f16, fp32 accumulate); then aᵀ[r_v × 16] =
-//           z_vᵀ · Pᵀ for the previous tile into the drained slot.
+//           TMEM slots (kind::f16, fp32 accumulate); aᵀ[r_v × 16] = z_vᵀ · Pᵀ of
+//           tile j into columns of tile j+1's slot that its epilogue has already
+//           read, so no slot waits for a value round trip.
 //   warps 4-11 epilogue, two warpgroups of one thread per token: tcgen05.ld the rebuilt keys,
 //           rotate them (RoPE at the token's position), score against the
 //           rotated query, online softmax (exp2), write P (bf16/fp16) for the
-//           value MMA, and fold each tile's aᵀ into running latent sums.
+//           value MMA, fold the previous tile's aᵀ into running latent sums and
+//           release the slot.
 // Output: per (b, head, split) the partial (m, l, a[r_v]) the combine merges.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -47,7 +49,7 @@ __host__ __device__ constexpr int zk_stages(bool int4) { return int4 ? 2 : kNKS;
 constexpr uint32_t kZkSwz = 2u;    // 128-byte swizzle
 constexpr uint32_t kZkSbo = 1024;  // bytes per 8-row swizzle atom
 constexpr int kNVS = 2;            // z_v ring stages
-constexpr int kPrefetch = 3;       // pages pulled into L2 ahead of the TMA loads
+constexpr int kPrefetch = 3;       // int4: pages of codes pulled into L2 ahead of the loads
 constexpr int kBatch = 8;          // frequency pairs per TMEM round trip of the score pass
 constexpr int kNB = 32 / kBatch;   // score batches per warpgroup and tile
 constexpr int kThreads = 384;      // 12 warps: producers + MMA (warps 0-3), two epilogue warpgroups
@@ -102,6 +104,7 @@ enum {
   BAR_QR = BAR_EPI + 2,              // rotated query staged
   BAR_XCH = BAR_QR + 1,              // 2: both warpgroups posted their cross-head partial scores
   BAR_VRAW = BAR_XCH + 2,            // int4: a page of value codes landed in the staging buffer
+  BAR_MID = BAR_VRAW + 1,            // the epilogue is halfway through a tile's score pass (one phase per tile)
   BAR_COUNT
 };
 static_assert(BAR_COUNT <= 32, "barrier space");
@@ -301,6 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(BAR_TEARDOWN), 1);
     mbar_init(bar(BAR_QR), 4);
     mbar_init(bar(BAR_VRAW), 1);
+    mbar_init(bar(BAR_MID), 8);
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(BAR_EPI + i), 4);
       mbar_init(bar(BAR_XCH + i), 8);
@@ -384,7 +388,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(BAR_ZK_FULL + stage));
-      if (zt == 0 && (n & 3) == 0) trace(6, n >> 2);
       if (++stage == kNZK) { stage = 0; phase ^= 1; }
       return true;
     };
@@ -445,6 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int k = 0; k < nv_tiles && !*abort_flag; ++k) {
       const int pg_after = page_ahead(a, b, tr, k + 2);   // in flight during this tile
       if (!mbar_wait(bar(BAR_VRAW), k & 1, abort_flag, st, 14)) break;
+      if (lane == 0) trace(6, k);
       bool ok = true;
       for (int sidx = 0; sidx < 2 * NRV; ++sidx) {   // column block 2mb + cb of the page
         if (!mbar_wait(bar(BAR_ZV_EMPTY + stage), phase ^ 1, abort_flag, st, 13)) { ok = false; break; }
@@ -479,24 +483,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      // Pull the next pages of this split into L2 ahead of the TMA loads: the
-      // shared-memory ring is only a few chunks deep, so HBM latency is hidden
-      // in L2 instead.
-      auto prefetch_page = [&](int ppg, int kk) {   // ppg = raw table entry of tile kk
-        if (!page_valid(a, ppg)) return;
-        prefetch_l2(gm.zk[gi] + (size_t)ppg * gm.k_page, k_blk_bytes);
-        if (!(tr.ragged_last && kk == tr.ntiles - 1))
-          prefetch_l2(gm.zv[gi] + (size_t)ppg * gm.v_page, (uint32_t)(a.P * a.v_row));
-      };
-      for (int kk = 0; kk < kPrefetch; ++kk) prefetch_page(page_ahead(a, b, tr, kk), kk);
-      int pg_next = page_ahead(a, b, tr, 0), pf_next = page_ahead(a, b, tr, kPrefetch);
+      // No bulk L2 prefetch of later pages here: with the bulk copies of the two
+      // head-pair CTAs of a group in flight, a prefetch 3 or 6 pages ahead left the
+      // copy latency unchanged and the call 2-3 % slower.
+      int pg_next = page_ahead(a, b, tr, 0);
       long long issued = 0;
       for (int k = 0; k < tr.ntiles && !*abort_flag; ++k) {
         int pg = pg_next;
-        const int pf = pf_next;
         pg_next = page_ahead(a, b, tr, k + 1);   // in flight during this tile's copies
-        pf_next = page_ahead(a, b, tr, k + 1 + kPrefetch);
-        prefetch_page(pf, k + kPrefetch);
         if (!page_valid(a, pg)) {
           report(st, PALU_ERR_DEVICE_BOUNDS, 2000000 + b);
           pg = 0;   // keep the pipeline fed from a valid page; the status says the result is void
@@ -509,7 +503,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_expect_tx(bar(BAR_ZK_FULL + stage), kZkBytes);
           bulk_load(base + L.zk + stage * kZkBytes, src + (size_t)c * kZkBytes, kZkBytes, bar(BAR_ZK_FULL + stage));
           ++issued;
-          if (c == 0) trace(6, k);
           if (++stage == kNZK) { stage = 0; phase ^= 1; }
         }
       }
@@ -536,6 +529,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_expect_tx(bar(BAR_ZV_FULL + stage), kZvBytes);
           bulk_load(base + L.zv + stage * kZvBytes, src + (size_t)cb * a.P * 128, kZvBytes,
                     bar(BAR_ZV_FULL + stage));
+          if (cb == 0) trace(6, k);
           ++issued;
           if (++stage == kNVS) { stage = 0; phase ^= 1; }
         }
@@ -554,15 +548,37 @@ __global__ void __launch_bounds__(kThreads, 1)
       // timeout-path test hook: first wait on a phase nothing completes before the teardown commit
       bool ok = a.stall_test == 0 || mbar_wait(bar(BAR_TEARDOWN), 0, abort_flag, st, 26);
       ok = ok && mbar_wait(bar(BAR_B), 0, abort_flag, st, 20);
-      int pv_pending = -1;   // tile whose value MMA (aᵀ[r_v × 16] = z_vᵀ · Pᵀ) is not yet issued
+      const int nv_tiles = tr.ntiles - (tr.ragged_last ? 1 : 0);   // tiles whose value sums run here
+      int pv_next = 0;       // next tile whose value MMA is not issued yet
       int pv_mb = 0;         // next 128-entry block of that value MMA
+      int zv_seen = -1;      // last tile whose value latents were seen in shared memory (trace)
 
-      // aᵀ[128 entries × 16] of block pv_mb for tile pv_pending = z_vᵀ · Pᵀ into
-      // the tile's (drained) D slot; its P and both ring stages are in
+      // The value MMA of tile j, aᵀ[128 entries × 16] per block = z_vᵀ · Pᵀ, goes into
+      // columns [32·mb, +16) of the TMEM slot of tile j + 1: columns whose keys that
+      // tile's epilogue has read by the middle of its score pass (BAR_MID), so the value
+      // round trip never holds a slot back from the next key MMA.  The last tile's value
+      // MMA goes into the other slot once it is free.  Its gate (besides P and z_v):
+      auto pv_gate = [&](int j) -> bool {
+        if (j + 1 < tr.ntiles) return mbar_test_wait(bar(BAR_MID), (uint32_t)((j + 1) & 1));
+        const int u = j + 1;
+        return mbar_test_wait(bar(BAR_D_EMPTY + (u & 1)), (uint32_t)(((u >> 1) & 1) ^ 1));
+      };
+      // The next block of the pending value MMA can go?  (Phases cannot alias: the
+      // epilogue cannot pass tile j + 1 before the value sums of tile j are folded.)
+      auto pv_ready = [&]() -> bool {
+        if (pv_next >= nv_tiles) return false;
+        if (!(mbar_test_wait(bar(BAR_ZV_FULL + 0), vph) && mbar_test_wait(bar(BAR_ZV_FULL + 1), vph))) return false;
+        if (pv_mb == 0 && zv_seen != pv_next) {
+          zv_seen = pv_next;
+          trace(7, pv_next);
+        }
+        return pv_mb > 0 || (mbar_test_wait(bar(BAR_P_FULL + (pv_next & 1)), (uint32_t)((pv_next >> 1) & 1)) &&
+                             pv_gate(pv_next));
+      };
       auto issue_pv_block = [&]() {
-        const int j = pv_pending;
+        const int j = pv_next;
         tc_fence_after();
-        const uint32_t a_tmem = tmem + (uint32_t)(j & 1) * 256;
+        const uint32_t a_tmem = tmem + (uint32_t)((j + 1) & 1) * 256 + (uint32_t)pv_mb * 32;
         const uint32_t p_base = base + L.p + (uint32_t)(j & 1) * kPBytes;
         static_assert(kNVS == 2, "one value MMA operand = the two ring stages");
 #pragma unroll
@@ -570,7 +586,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // rows = latent entries (two 64-entry blocks, one per stage), K = tokens
           const uint64_t ad = sdesc(base + L.zv + kk * 16 * 128, kZvBytes, 1024, kSw128);
           const uint64_t bd = sdesc(p_base + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024, kSw128);
-          umma_f16(a_tmem + pv_mb * 16, ad, bd, idesc_pv, kk != 0);
+          umma_f16(a_tmem, ad, bd, idesc_pv, kk != 0);
         }
         umma_commit(bar(BAR_ZV_EMPTY + 0));
         umma_commit(bar(BAR_ZV_EMPTY + 1));
@@ -578,56 +594,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (++pv_mb == NRV) {
           umma_commit(bar(BAR_AT_FULL));
           trace(2, j);
-          pv_pending = -1;
+          ++pv_next;
           pv_mb = 0;
         }
       };
-      // The next block of the pending value MMA can go (its P and z_v are in)?
-      auto pv_ready = [&]() -> bool {
-        return pv_pending >= 0 &&
-               (pv_mb > 0 || mbar_test_wait(bar(BAR_P_FULL + (pv_pending & 1)), (pv_pending >> 1) & 1)) &&
-               mbar_test_wait(bar(BAR_ZV_FULL + 0), vph) && mbar_test_wait(bar(BAR_ZV_FULL + 1), vph);
-      };
-      // Wait for z_k data; meanwhile issue each block of the pending value MMA
-      // as soon as its P and z_v are in (never blocking on them, so key chunks
-      // keep flowing while the value operand is still being filled).  Bounded.
-      auto wait_zk = [&]() -> bool {
+      // Wait for a barrier phase; meanwhile issue every value-MMA block whose operands
+      // and gate are in (the epilogue's slot releases depend on them).  Bounded.
+      auto poll_wait = [&](uint32_t b, uint32_t parity, int where) -> bool {
         const long long t0 = clock64();
         while (true) {
-          if (mbar_test_wait(bar(BAR_ZK_FULL + zs), zph)) return true;
-          if (pv_ready()) issue_pv_block();
+          if (mbar_test_wait(b, parity)) return true;
+          if (pv_ready()) {
+            issue_pv_block();
+            continue;
+          }
           if (*abort_flag) return false;
           __nanosleep(64);   // leave the issue slots of this SM partition to the epilogue warps
           if (clock64() - t0 > wait_limit(abort_flag)) {
-            report(st, PALU_ERR_DEVICE_TIMEOUT, 24);
+            report(st, PALU_ERR_DEVICE_TIMEOUT, where);
             *abort_flag = 1;
             return false;
           }
         }
       };
-      // Issue what is left of the pending value MMA, waiting for its operands.  Bounded.
-      auto flush_pv = [&]() -> bool {
-        while (pv_pending >= 0) {
-          if (pv_mb == 0 &&
-              !mbar_wait(bar(BAR_P_FULL + (pv_pending & 1)), (pv_pending >> 1) & 1, abort_flag, st, 21))
-            return false;
-          for (int cb = 0; cb < 2; ++cb)
-            if (!mbar_wait(bar(BAR_ZV_FULL + cb), vph, abort_flag, st, 22)) return false;
-          issue_pv_block();
-        }
-        return true;
-      };
 
       for (int k = 0; k < tr.ntiles && ok; ++k) {
         const int slot = k & 1;
-        if (!mbar_wait(bar(BAR_D_EMPTY + slot), ((k >> 1) & 1) ^ 1, abort_flag, st, 23)) { ok = false; break; }
+        if (!poll_wait(bar(BAR_D_EMPTY + slot), ((k >> 1) & 1) ^ 1, 23)) { ok = false; break; }
         tc_fence_after();
         trace(0, k);
         const uint32_t d_tmem = tmem + (uint32_t)slot * 256;
         for (int c = 0; c < nkc; ++c) {
-          if (!wait_zk()) { ok = false; break; }
+          if (!poll_wait(bar(BAR_ZK_FULL + zs), zph, 24)) { ok = false; break; }
           tc_fence_after();
-          if (c == 0) trace(7, k);
           const uint32_t zk_addr = base + L.zk + zs * kZkBytes;
           const uint32_t b_addr = base + L.b + (uint32_t)c * kChunk * 128;
 #pragma unroll
@@ -642,11 +641,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         umma_commit(bar(BAR_D_FULL + slot));
         trace(1, k);
-        // the previous tile's value MMA must be out before this one queues
-        if (!flush_pv()) { ok = false; break; }
-        if (!(tr.ragged_last && k == tr.ntiles - 1)) pv_pending = k;
       }
-      if (ok) ok = flush_pv();
+      // the value MMAs still pending (the last tiles'), each once its operands are in
+      if (ok) {
+        const long long t0 = clock64();
+        while (pv_next < nv_tiles) {
+          if (pv_ready()) {
+            issue_pv_block();
+            continue;
+          }
+          if (*abort_flag) break;
+          __nanosleep(64);
+          if (clock64() - t0 > wait_limit(abort_flag)) {
+            report(st, PALU_ERR_DEVICE_TIMEOUT, 21);
+            *abort_flag = 1;
+            break;
+          }
+        }
+      }
       // drain, also after an abort: every MMA issued above has completed before
       // TMEM is released, and the B_k load has landed before the CTA exits
       umma_commit(bar(BAR_TEARDOWN));
@@ -730,7 +742,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int hh = 0; hh < 2; ++hh) acc[hh][0] = acc[hh][1] = 0ull;
 #pragma unroll
       for (int jj = 0; jj < kNB; ++jj) {
-        mid(jj);   // the previous tile's latent sums, folded as soon as they are in
+        mid(jj);   // halfway: signal that the first batches' columns are read
         const int i0 = wg * 32 + jj * kBatch;
         const uint32_t col = tmem + lane_addr + (uint32_t)slot * 256 + i0;
         // both heads' keys of these kBatch frequency pairs in one TMEM round trip
@@ -813,21 +825,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int mb = 0; mb < NRV; ++mb) acc[mb] = 0.f;
       float* red = reinterpret_cast<float*>(sbase + L.red);
 
+      // The value sums of tile j sit in the TMEM slot of tile j + 1 (columns [32·mb, +16),
+      // column hw of each block for this head); fold them into the running sums.
       auto fold_at = [&](int j, float scale) -> bool {
         if (!mbar_wait(bar(BAR_AT_FULL), j & 1, abort_flag, st, 30)) return false;
         tc_fence_after();
+        const uint32_t sb = (uint32_t)((j + 1) & 1) * 256;
 #pragma unroll
         for (int mb = 0; mb < NRV; ++mb) {
-          const float v = tmem_ld1(tmem + lane_addr + (uint32_t)(j & 1) * 256 + mb * 16 + hw);
+          const float v = tmem_ld1(tmem + lane_addr + sb + mb * 32 + hw);
           tmem_wait_ld();
           acc[mb] = fmaf(acc[mb], scale, v);
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(BAR_D_EMPTY + (j & 1)));
         return true;
       };
 
+      const int nv_tiles = tr.ntiles - (tr.ragged_last ? 1 : 0);   // tiles whose value sums are MMAs
       // causal bound (several queries per step): tokens after the query's position are masked
       const int qlim = a.causal ? a.q_pos[(size_t)b * a.qpos_bstride] : 0;
       for (int k = 0; k < tr.ntiles && ok; ++k) {
@@ -843,28 +856,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         if (row == 0 && wg == 0) trace(3, k);
         float part[2];
-        // The previous tile's latent sums are folded halfway through this tile's
-        // scores: its value MMA has had that long to finish, and its TMEM slot
-        // (where the next key MMA goes) is released early enough for that MMA
-        // to finish before the next tile's scores start.
-        // Fold the previous tile's latent sums before the first score batch that
-        // finds them complete (lane 0 tests, the warp follows), and at the latest
-        // halfway through: that releases its TMEM slot for the next key MMA.
-        bool folded = k == 0, fold_ok = true;
+        // Halfway through the pass (score batches 0 and 1 read) the columns where the
+        // previous tile's value MMA writes are dead: tell the MMA thread.
         half_scores(slot, t0, pos, part, [&](int jj) {
-          if (folded) return;
-          int ready = 1;
-          if (jj < kNB / 2) {
-            if (lane == 0) ready = mbar_test_wait(bar(BAR_AT_FULL), (k - 1) & 1) ? 1 : 0;
-            ready = __shfl_sync(0xffffffffu, ready, 0);
-          }
-          if (ready) {
-            fold_ok = fold_at(k - 1, prev_scale);
-            folded = true;
-          }
+          if (jj != kNB / 2) return;
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(BAR_MID));
         });
-        if (!fold_ok) { ok = false; break; }
-        tc_fence_before();
         psc[(slot * 2 + (1 - hw)) * 128 + row] = part[1 - hw];
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(BAR_XCH + slot));
@@ -891,7 +890,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(BAR_P_FULL + slot));
         if (row == 0 && wg == 0) trace(5, k);
+        // the previous tile's value sums (written into this slot), then release the slot
+        if (k >= 1 && k - 1 < nv_tiles && !fold_at(k - 1, prev_scale)) { ok = false; break; }
         prev_scale = scale;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(BAR_D_EMPTY + slot));
       }
 
       if (ok && tr.ntiles > 0) {

@@ -130,14 +130,11 @@ WORKLOADS = {
            batch=1, context=256, act_dtype="f32", latent_dtype="f32", d_model=256, seed=0),
         _w("7b_f16_r256_b1_t4k", num_heads=32, head_dim=128, group_size=4, rank_k=256,
            rank_v=256, batch=1, context=4096, act_dtype="f16", latent_dtype="f16", seed=2),
-        _w("7b_bf16_r256v128_b1_t4k", num_heads=32, head_dim=128, group_size=4, rank_k=256,
-           rank_v=128, batch=1, context=4096, act_dtype="bf16", latent_dtype="bf16", seed=3),
-        _w("7b_bf16_r256v128_b8_t16k", num_heads=32, head_dim=128, group_size=4, rank_k=256,
-           rank_v=128, batch=8, context=16384, act_dtype="bf16", latent_dtype="bf16", seed=3),
-        _w("7b_bf16_r256v128_b16_t16k", num_heads=32, head_dim=128, group_size=4, rank_k=256,
-           rank_v=128, batch=16, context=16384, act_dtype="bf16", latent_dtype="bf16", seed=3),
-        _w("7b_bf16_r256v128_b16_t64k", num_heads=32, head_dim=128, group_size=4, rank_k=256,
-           rank_v=128, batch=16, context=65536, act_dtype="bf16", latent_dtype="bf16", seed=3),
+        # the bf16 context sweep: context 4k / 16k / 64k x batch 1 / 8 / 16, key rank 256,
+        # value rank 128
+        *[_w(f"7b_bf16_r256v128_b{b}_t{t // 1024}k", num_heads=32, head_dim=128, group_size=4,
+             rank_k=256, rank_v=128, batch=b, context=t, act_dtype="bf16", latent_dtype="bf16", seed=3)
+          for t in (4096, 16384, 65536) for b in (1, 8, 16)],
         _w("7b_int4_r256_b8_t32k", num_heads=32, head_dim=128, group_size=4, rank_k=256,
            rank_v=256, batch=8, context=32768, act_dtype="f16", latent_dtype="int4", seed=4),
         _w("7b_bf16_r256_b32_t16k", num_heads=32, head_dim=128, group_size=4, rank_k=256,

@@ -45,37 +45,42 @@ using namespace tc;
 constexpr int kTile = 128;         // tokens per tile = page size
 constexpr int kChunk = 64;         // K chunk of z_k (elements) = one 128-byte column block of the page
 constexpr int kNKS = 3;            // z_k ring stages (barrier slots)
-__host__ __device__ constexpr int zk_stages(bool int4) { return int4 ? 2 : kNKS; }  // int4: room for the value-code buffer
 constexpr uint32_t kZkSwz = 2u;    // 128-byte swizzle
 constexpr uint32_t kZkSbo = 1024;  // bytes per 8-row swizzle atom
 constexpr int kNVS = 2;            // z_v ring stages
 constexpr int kPrefetch = 3;       // int4: pages of codes pulled into L2 ahead of the loads
 constexpr int kBatch = 8;          // frequency pairs per TMEM round trip of the score pass
 constexpr int kNB = 32 / kBatch;   // score batches per warpgroup and tile
-constexpr int kThreads = 384;      // 12 warps: producers + MMA (warps 0-3), two epilogue warpgroups
+// 16-bit latents: 12 warps (producers + MMA in warps 0-3, two epilogue warpgroups).
+// int4 latents: 16 warps; the codes are converted to the compute dtype by warps 0, 2, 3
+// (values) and 12-15 (keys), so the conversion keeps up with the tensor cores.
+__host__ __device__ constexpr int threads_of(bool int4) { return int4 ? 512 : 384; }
+// int4 register split (setmaxnreg): launched at 128 per thread (65,536 / 512), the two
+// epilogue warpgroups take 168, warpgroup 0 (value conversion and the MMA thread) 104,
+// the key converters 72: 2·168 + 104 + 72 = 4·128 (no spills in any role).
+constexpr uint32_t kRegsLaunch = 128, kRegsEpi = 168, kRegsW0 = 104, kRegsKey = 72;
+static_assert(2 * kRegsEpi + kRegsW0 + kRegsKey == 4 * kRegsLaunch, "register split");
 constexpr int kZkBytes = kTile * kChunk * 2;   // bytes per z_k stage
 constexpr int kZvBytes = 128 * 64 * 2;         // 16 KB: one 64-entry column block of a page (128 tokens)
 constexpr int kPBytes = 16 * kTile * 2;        // 4 KB: 16 rows (heads, padded) × 128 tokens
 
 struct Smem {
   // offsets in bytes from a 1024-aligned base
-  uint32_t b, zk, zv, vraw, p, qr, psc, tb, omega, red, lred, bars, tmem_slot, abort, total;
+  uint32_t b, zk, zv, p, qr, psc, tb, omega, red, lred, bars, tmem_slot, abort, total;
 };
-
-constexpr int kVRawBytes = 128 * 128 + 128 * 16;   // int4: one page of value codes + its scale rows
 
 // Every region but B_k (whose size follows the key rank) sits at a fixed offset,
 // so the kernel's offsets are compile-time constants; B_k comes last.
 __host__ __device__ inline Smem smem_layout(int r_k, bool int4) {
   Smem s{};
+  (void)int4;   // int4 codes are converted straight from global memory into the same rings
   uint32_t o = 0;
-  s.zk = o;     o += zk_stages(int4) * kZkBytes;
+  s.zk = o;     o += kNKS * kZkBytes;
   s.zv = o;     o += kNVS * kZvBytes;
-  s.vraw = o;   o += int4 ? kVRawBytes : 0;
   s.p = o;      o += 2 * kPBytes;
   s.qr = o;     o += 3 * 128 * 4;                        // q'_i, q'_{i+64}, -q'_i per head pair row
   s.psc = o;    o += 2 * 2 * 128 * 4;
-  s.tb = o;     o += 8 * 3 * 32 * 4;                     // per epilogue warp: cos, sin, -sin at t0
+  s.tb = o;     o += 2 * 2 * 2 * 3 * 32 * 4;             // [warpgroup][tile parity][head][A|B|-A][32 freq]
   s.omega = o;  o += 64 * 8;
   s.red = o;    o += 2 * 4 * 2 * 4;
   s.lred = o;   o += 4 * 2 * 4;
@@ -103,8 +108,7 @@ enum {
   BAR_EPI = BAR_TEARDOWN + 1,        // 2: per-warpgroup sync (4 warps), bounded
   BAR_QR = BAR_EPI + 2,              // rotated query staged
   BAR_XCH = BAR_QR + 1,              // 2: both warpgroups posted their cross-head partial scores
-  BAR_VRAW = BAR_XCH + 2,            // int4: a page of value codes landed in the staging buffer
-  BAR_MID = BAR_VRAW + 1,            // the epilogue is halfway through a tile's score pass (one phase per tile)
+  BAR_MID = BAR_XCH + 2,             // the epilogue is halfway through a tile's score pass (one phase per tile)
   BAR_COUNT
 };
 static_assert(BAR_COUNT <= 32, "barrier space");
@@ -255,7 +259,7 @@ __device__ __forceinline__ void trace_record(const DecodeArgs& a, int ev, int k,
 // instantiation keeps the per-token sincos path of explicit positions out of
 // the score loop's instruction footprint.
 template <int ACT, int NRV, int LAT, bool CONTIG>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(threads_of(LAT == PALU_INT4), 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tm_bk, const __grid_constant__ DecodeArgs a) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -267,7 +271,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const Smem L = smem_layout(r_k, LAT == PALU_INT4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr bool kInt4 = LAT == PALU_INT4;
-  constexpr int kNZK = zk_stages(kInt4);
+  constexpr int kNZK = kNKS;
+  constexpr int kThreads = threads_of(kInt4);
   static_assert(!kInt4 || NRV == 2, "int4 latents: r_v = 256");
   DevStatus* st = reinterpret_cast<DevStatus*>(a.status);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sbase + L.abort);
@@ -288,11 +293,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     abort_init(abort_flag, a.wait_cycles);
     mbar_init(bar(BAR_B), 1);
     for (int i = 0; i < kNZK; ++i) {
-      mbar_init(bar(BAR_ZK_FULL + i), kInt4 ? 2 : 1);   // int4: one arrival per dequantising warp
+      mbar_init(bar(BAR_ZK_FULL + i), kInt4 ? 4 : 1);   // int4: one arrival per converting warp
       mbar_init(bar(BAR_ZK_EMPTY + i), 1);
     }
     for (int i = 0; i < kNVS; ++i) {
-      mbar_init(bar(BAR_ZV_FULL + i), 1);
+      mbar_init(bar(BAR_ZV_FULL + i), kInt4 ? 3 : 1);
       mbar_init(bar(BAR_ZV_EMPTY + i), 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -303,7 +308,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(BAR_AT_FULL), 1);
     mbar_init(bar(BAR_TEARDOWN), 1);
     mbar_init(bar(BAR_QR), 4);
-    mbar_init(bar(BAR_VRAW), 1);
     mbar_init(bar(BAR_MID), 8);
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(BAR_EPI + i), 4);
@@ -335,20 +339,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_2d(base + L.b + (uint32_t)nb * r_k * 128 + rb * 128, &tm_bk, hp * 256 + nb * 64,
                     gm.k_row0[gi] + rb, bar(BAR_B));
   }
-  if (kInt4 && (warp == 0 || warp == 3)) {
-    // ============================================================ int4 key codes (warps 0, 3)
+  // Roles.  int4 latents: each warpgroup first sets its share of the register file
+  // (setmaxnreg, see kRegsLaunch), inside the branch whose code uses it.
+  if (kInt4 && warp >= 12) {
+    if constexpr (kInt4) setmaxnreg_dec<kRegsKey>();
+    // ============================================================ int4 key codes (warps 12-15)
     // Chunk c of a tile = entries [64c, 64c + 64) of all 128 tokens, i.e. scale
-    // blocks 2c and 2c+1.  Thread zt takes block 2c + (zt & 1) of tokens
-    // zt/2 + 32i, loaded straight into registers three chunks ahead of the
-    // conversion (four register slots), while later pages are pulled into L2.
-    const int zt = (warp == 3 ? 32 : 0) + lane;
+    // blocks 2c and 2c+1 = 16-byte units 2c and 2c+1 of each token's row of codes.
+    // Thread t takes both units of token t, loaded straight into registers three
+    // chunks ahead of the conversion, while later pages are pulled into L2.
+    const int t = threadIdx.x - 384;
     const int N = tr.ntiles * 4;
     struct Slot {
-      uint4 raw[4];
-      uint16_t sc[4];
+      uint4 raw[2];
+      uint16_t sc[2];
     };
     auto prefetch_page = [&](int ppg) {
-      if (zt != 0 || !page_valid(a, ppg)) return;
+      if (t != 0 || !page_valid(a, ppg)) return;
       prefetch_l2(gm.zk[gi] + (size_t)ppg * gm.k_page, k_blk_bytes);
       prefetch_l2(gm.zks[gi] + (size_t)ppg * gm.ks_page, (uint32_t)(a.P * a.ks_row));
       prefetch_l2(gm.zv[gi] + (size_t)ppg * gm.v_page, (uint32_t)(a.P * a.v_row));
@@ -358,17 +365,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto issue = [&](int n, Slot& sl, int pg) {
       if (n >= N) return;
       if (!page_valid(a, pg)) {
-        if ((n & 3) == 0 && zt == 0) report(st, PALU_ERR_DEVICE_BOUNDS, 2000000 + b);
+        if ((n & 3) == 0 && t == 0) report(st, PALU_ERR_DEVICE_BOUNDS, 2000000 + b);
         pg = 0;   // keep the pipeline fed from a valid page; the status says the result is void
       }
-      const uint8_t* blk = gm.zk[gi] + (size_t)pg * gm.k_page;
-      const uint8_t* sblk = gm.zks[gi] + (size_t)pg * gm.ks_page;
-      const int u = 2 * (n & 3) + (zt & 1);
+      const uint8_t* row = gm.zk[gi] + (size_t)pg * gm.k_page + t * 128;
+      const uint8_t* srow = gm.zks[gi] + (size_t)pg * gm.ks_page + (size_t)t * a.ks_row;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int t = (zt >> 1) + 32 * i;
-        sl.raw[i] = __ldg(reinterpret_cast<const uint4*>(blk + t * 128 + ((u ^ (t & 7)) << 4)));
-        sl.sc[i] = __ldg(reinterpret_cast<const unsigned short*>(sblk + t * a.ks_row + 2 * u));
+      for (int ub = 0; ub < 2; ++ub) {
+        const int u = 2 * (n & 3) + ub;
+        sl.raw[ub] = __ldg(reinterpret_cast<const uint4*>(row + ((u ^ (t & 7)) << 4)));
+        sl.sc[ub] = __ldg(reinterpret_cast<const unsigned short*>(srow + 2 * u));
       }
     };
     int stage = 0;
@@ -376,14 +382,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto consume = [&](int n, const Slot& sl) -> bool {
       if (n >= N) return true;
       if (!mbar_wait(bar(BAR_ZK_EMPTY + stage), phase ^ 1, abort_flag, st, 12)) return false;
-      const uint32_t dst = base + L.zk + stage * kZkBytes;
+      const uint32_t dst = base + L.zk + stage * kZkBytes + t * 128;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int t = (zt >> 1) + 32 * i;
-        const uint32_t w[4] = {sl.raw[i].x, sl.raw[i].y, sl.raw[i].z, sl.raw[i].w};
+      for (int ub = 0; ub < 2; ++ub) {
+        const uint32_t w[4] = {sl.raw[ub].x, sl.raw[ub].y, sl.raw[ub].z, sl.raw[ub].w};
 #pragma unroll
         for (int m = 0; m < 4; ++m)
-          st_shared_v4(dst + t * 128 + (((4 * (zt & 1) + m) ^ (t & 7)) << 4), dequant8<ACT, false>(w[m], sl.sc[i]));
+          st_shared_v4(dst + (((4 * ub + m) ^ (t & 7)) << 4), dequant8<ACT, false>(w[m], sl.sc[ub]));
       }
       fence_proxy_async();
       __syncwarp();
@@ -402,8 +407,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     issue(2, s2, pg_k);
     // One load batch and one conversion per chunk, the register slots shifted
     // down after each: a single copy of the conversion code keeps the kernel's
-    // instruction footprint small (the warps of a sub-partition run different
-    // roles, so an unrolled copy per slot thrashed the instruction cache).
+    // instruction footprint small.
 #pragma unroll 1
     for (int n = 0; n < N && !*abort_flag; ++n) {
       const int c = n & 3;
@@ -422,250 +426,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       s1 = s2;
       s2 = s3;
     }
-  } else if (kInt4 && warp == 2) {
-    // ============================================================ int4 value codes (warp 2)
-    // One page of codes and its scale rows per tile, staged in shared memory by
-    // a bulk copy; ring stage (mb, cb) = the 64 entries [128mb + 64cb, +64) of
-    // all 128 tokens, i.e. scale blocks 4mb + 2cb and 4mb + 2cb + 1.  Lane takes
-    // block 4mb + 2cb + (lane/8 & 1) of tokens lane%8 + 8(2i + lane/16).  Units
-    // are written PAIRED: row r of the value operand holds entry paired_row(r).
-    const int nv_tiles = tr.ntiles - (tr.ragged_last ? 1 : 0);
-    const uint32_t vraw = base + L.vraw;
-    int raw_loads = 0;                // staged pages issued (lane 0); BAR_VRAW phase n completes load n
-    auto load_raw = [&](int pg) {   // pg = raw table entry, read a tile earlier
-      if (!page_valid(a, pg)) pg = 0;   // reported by the key producer
-      ++raw_loads;
-      mbar_expect_tx(bar(BAR_VRAW), kVRawBytes);
-      bulk_load(vraw, gm.zv[gi] + (size_t)pg * gm.v_page, 128 * 128, bar(BAR_VRAW));
-      bulk_load(vraw + 128 * 128, gm.zvs[gi] + (size_t)pg * gm.vs_page, 128 * 16,
-                bar(BAR_VRAW));
-    };
-    if (lane == 0 && nv_tiles > 0) load_raw(page_ahead(a, b, tr, 0));
-    int pg_next = page_ahead(a, b, tr, 1);
-    int stage = 0;
-    uint32_t phase = 0;
-    const int x = lane & 7, ub = (lane >> 3) & 1, tg = lane >> 4;
-    for (int k = 0; k < nv_tiles && !*abort_flag; ++k) {
-      const int pg_after = page_ahead(a, b, tr, k + 2);   // in flight during this tile
-      if (!mbar_wait(bar(BAR_VRAW), k & 1, abort_flag, st, 14)) break;
-      if (lane == 0) trace(6, k);
-      bool ok = true;
-      for (int sidx = 0; sidx < 2 * NRV; ++sidx) {   // column block 2mb + cb of the page
-        if (!mbar_wait(bar(BAR_ZV_EMPTY + stage), phase ^ 1, abort_flag, st, 13)) { ok = false; break; }
-        const uint32_t dst = base + L.zv + stage * kZvBytes;
-        const int u = 2 * sidx + ub;
-#pragma unroll 2
-        for (int i = 0; i < 8; ++i) {
-          const int t = x + 8 * (2 * i + tg);
-          const uint4 raw = ld_shared_v4(vraw + t * 128 + ((u ^ x) << 4));
-          const uint16_t sc = ld_shared_u16(vraw + 128 * 128 + t * 16 + 2 * u);
-          const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-          for (int m = 0; m < 4; ++m)
-            st_shared_v4(dst + t * 128 + (((4 * ub + m) ^ x) << 4), dequant8<ACT, true>(w[m], sc));
-        }
-        fence_proxy_async();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(BAR_ZV_FULL + stage));
-        if (++stage == kNVS) { stage = 0; phase ^= 1; }
-      }
-      if (!ok) break;
-      // every lane has read this page's codes: refill the buffer with the next page
-      fence_proxy_async();
-      __syncwarp();
-      if (lane == 0 && k + 1 < nv_tiles) load_raw(pg_next);
-      pg_next = pg_after;
-    }
-    // the staging buffer may still be filling after an abort: wait for the last page issued
-    if (lane == 0 && raw_loads > 0) mbar_drain(bar(BAR_VRAW), (uint32_t)((raw_loads - 1) & 1), st, 14);
-  } else if (warp == 0) {
-    // ============================================================ z_k producer (bulk copies)
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      // No bulk L2 prefetch of later pages here: with the bulk copies of the two
-      // head-pair CTAs of a group in flight, a prefetch 3 or 6 pages ahead left the
-      // copy latency unchanged and the call 2-3 % slower.
-      int pg_next = page_ahead(a, b, tr, 0);
-      long long issued = 0;
-      for (int k = 0; k < tr.ntiles && !*abort_flag; ++k) {
-        int pg = pg_next;
-        pg_next = page_ahead(a, b, tr, k + 1);   // in flight during this tile's copies
-        if (!page_valid(a, pg)) {
-          report(st, PALU_ERR_DEVICE_BOUNDS, 2000000 + b);
-          pg = 0;   // keep the pipeline fed from a valid page; the status says the result is void
-        }
-        // one (page, group) block is the shared-memory image of the tile: each
-        // 128-byte column block (64 latent entries of all 128 tokens) is one copy
-        const uint8_t* src = gm.zk[gi] + (size_t)pg * gm.k_page;
-        for (int c = 0; c < nkc; ++c) {
-          if (!mbar_wait(bar(BAR_ZK_EMPTY + stage), phase ^ 1, abort_flag, st, 10)) break;
-          mbar_expect_tx(bar(BAR_ZK_FULL + stage), kZkBytes);
-          bulk_load(base + L.zk + stage * kZkBytes, src + (size_t)c * kZkBytes, kZkBytes, bar(BAR_ZK_FULL + stage));
-          ++issued;
-          if (++stage == kNZK) { stage = 0; phase ^= 1; }
-        }
-      }
-      drain_ring(bar(BAR_ZK_FULL), kNZK, issued, st, 10);
-    }
-  } else if (warp == 2) {
-    // ============================================================ z_v producer (bulk copies)
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      int pg_next = page_ahead(a, b, tr, 0);
-      long long issued = 0;
-      for (int k = 0; k < tr.ntiles && !*abort_flag; ++k) {
-        if (tr.ragged_last && k == tr.ntiles - 1) break;    // CUDA-core value sum for a partial page
-        int pg = pg_next;
-        pg_next = page_ahead(a, b, tr, k + 1);   // in flight during this tile's copies
-        if (!page_valid(a, pg)) pg = 0;   // reported by the z_k producer
-        const uint8_t* src = gm.zv[gi] + (size_t)pg * gm.v_page;
-        // one copy per 128-byte column block of the page (64 latent entries of
-        // all 128 tokens); two consecutive blocks are the two MN-blocks of one
-        // value-MMA operand
-        for (int cb = 0; cb < 2 * NRV; ++cb) {
-          if (!mbar_wait(bar(BAR_ZV_EMPTY + stage), phase ^ 1, abort_flag, st, 11)) break;
-          mbar_expect_tx(bar(BAR_ZV_FULL + stage), kZvBytes);
-          bulk_load(base + L.zv + stage * kZvBytes, src + (size_t)cb * a.P * 128, kZvBytes,
-                    bar(BAR_ZV_FULL + stage));
-          if (cb == 0) trace(6, k);
-          ++issued;
-          if (++stage == kNVS) { stage = 0; phase ^= 1; }
-        }
-      }
-      drain_ring(bar(BAR_ZV_FULL), kNVS, issued, st, 11);
-    }
-  } else if (warp == 1) {
-    // ============================================================ MMA issuer
-    if (lane == 0) {
-      constexpr int kBf = ACT == PALU_BF16 ? 1 : 0;
-      const uint32_t idesc_d = idesc_f16(kBf, 0, 1, 256, 128);    // z_k K-major, B_k MN-major
-      const uint32_t idesc_pv = idesc_f16(kBf, 1, 0, 16, 128);    // z_vᵀ MN-major, Pᵀ K-major
-      const uint32_t b_lbo = (uint32_t)r_k * 128;                  // bytes between 64-column blocks of B
-      int zs = 0;
-      uint32_t zph = 0, vph = 0;
-      // timeout-path test hook: first wait on a phase nothing completes before the teardown commit
-      bool ok = a.stall_test == 0 || mbar_wait(bar(BAR_TEARDOWN), 0, abort_flag, st, 26);
-      ok = ok && mbar_wait(bar(BAR_B), 0, abort_flag, st, 20);
-      const int nv_tiles = tr.ntiles - (tr.ragged_last ? 1 : 0);   // tiles whose value sums run here
-      int pv_next = 0;       // next tile whose value MMA is not issued yet
-      int pv_mb = 0;         // next 128-entry block of that value MMA
-      int zv_seen = -1;      // last tile whose value latents were seen in shared memory (trace)
-
-      // The value MMA of tile j, aᵀ[128 entries × 16] per block = z_vᵀ · Pᵀ, goes into
-      // columns [32·mb, +16) of the TMEM slot of tile j + 1: columns whose keys that
-      // tile's epilogue has read by the middle of its score pass (BAR_MID), so the value
-      // round trip never holds a slot back from the next key MMA.  The last tile's value
-      // MMA goes into the other slot once it is free.  Its gate (besides P and z_v):
-      auto pv_gate = [&](int j) -> bool {
-        if (j + 1 < tr.ntiles) return mbar_test_wait(bar(BAR_MID), (uint32_t)((j + 1) & 1));
-        const int u = j + 1;
-        return mbar_test_wait(bar(BAR_D_EMPTY + (u & 1)), (uint32_t)(((u >> 1) & 1) ^ 1));
-      };
-      // The next block of the pending value MMA can go?  (Phases cannot alias: the
-      // epilogue cannot pass tile j + 1 before the value sums of tile j are folded.)
-      auto pv_ready = [&]() -> bool {
-        if (pv_next >= nv_tiles) return false;
-        if (!(mbar_test_wait(bar(BAR_ZV_FULL + 0), vph) && mbar_test_wait(bar(BAR_ZV_FULL + 1), vph))) return false;
-        if (pv_mb == 0 && zv_seen != pv_next) {
-          zv_seen = pv_next;
-          trace(7, pv_next);
-        }
-        return pv_mb > 0 || (mbar_test_wait(bar(BAR_P_FULL + (pv_next & 1)), (uint32_t)((pv_next >> 1) & 1)) &&
-                             pv_gate(pv_next));
-      };
-      auto issue_pv_block = [&]() {
-        const int j = pv_next;
-        tc_fence_after();
-        const uint32_t a_tmem = tmem + (uint32_t)((j + 1) & 1) * 256 + (uint32_t)pv_mb * 32;
-        const uint32_t p_base = base + L.p + (uint32_t)(j & 1) * kPBytes;
-        static_assert(kNVS == 2, "one value MMA operand = the two ring stages");
-#pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk) {
-          // rows = latent entries (two 64-entry blocks, one per stage), K = tokens
-          const uint64_t ad = sdesc(base + L.zv + kk * 16 * 128, kZvBytes, 1024, kSw128);
-          const uint64_t bd = sdesc(p_base + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024, kSw128);
-          umma_f16(a_tmem, ad, bd, idesc_pv, kk != 0);
-        }
-        umma_commit(bar(BAR_ZV_EMPTY + 0));
-        umma_commit(bar(BAR_ZV_EMPTY + 1));
-        vph ^= 1;
-        if (++pv_mb == NRV) {
-          umma_commit(bar(BAR_AT_FULL));
-          trace(2, j);
-          ++pv_next;
-          pv_mb = 0;
-        }
-      };
-      // Wait for a barrier phase; meanwhile issue every value-MMA block whose operands
-      // and gate are in (the epilogue's slot releases depend on them).  Bounded.
-      auto poll_wait = [&](uint32_t b, uint32_t parity, int where) -> bool {
-        const long long t0 = clock64();
-        while (true) {
-          if (mbar_test_wait(b, parity)) return true;
-          if (pv_ready()) {
-            issue_pv_block();
-            continue;
-          }
-          if (*abort_flag) return false;
-          __nanosleep(64);   // leave the issue slots of this SM partition to the epilogue warps
-          if (clock64() - t0 > wait_limit(abort_flag)) {
-            report(st, PALU_ERR_DEVICE_TIMEOUT, where);
-            *abort_flag = 1;
-            return false;
-          }
-        }
-      };
-
-      for (int k = 0; k < tr.ntiles && ok; ++k) {
-        const int slot = k & 1;
-        if (!poll_wait(bar(BAR_D_EMPTY + slot), ((k >> 1) & 1) ^ 1, 23)) { ok = false; break; }
-        tc_fence_after();
-        trace(0, k);
-        const uint32_t d_tmem = tmem + (uint32_t)slot * 256;
-        for (int c = 0; c < nkc; ++c) {
-          if (!poll_wait(bar(BAR_ZK_FULL + zs), zph, 24)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t zk_addr = base + L.zk + zs * kZkBytes;
-          const uint32_t b_addr = base + L.b + (uint32_t)c * kChunk * 128;
-#pragma unroll
-          for (int kk = 0; kk < kChunk / 16; ++kk) {
-            const uint64_t ad = sdesc(zk_addr + kk * 32, 16, kZkSbo, kZkSwz);
-            const uint64_t bd = sdesc(b_addr + kk * 16 * 128, b_lbo, 1024, kSw128);
-            umma_f16(d_tmem, ad, bd, idesc_d, (c | kk) != 0);
-          }
-          umma_commit(bar(BAR_ZK_EMPTY + zs));
-          if (++zs == kNZK) { zs = 0; zph ^= 1; }
-        }
-        if (!ok) break;
-        umma_commit(bar(BAR_D_FULL + slot));
-        trace(1, k);
-      }
-      // the value MMAs still pending (the last tiles'), each once its operands are in
-      if (ok) {
-        const long long t0 = clock64();
-        while (pv_next < nv_tiles) {
-          if (pv_ready()) {
-            issue_pv_block();
-            continue;
-          }
-          if (*abort_flag) break;
-          __nanosleep(64);
-          if (clock64() - t0 > wait_limit(abort_flag)) {
-            report(st, PALU_ERR_DEVICE_TIMEOUT, 21);
-            *abort_flag = 1;
-            break;
-          }
-        }
-      }
-      // drain, also after an abort: every MMA issued above has completed before
-      // TMEM is released, and the B_k load has landed before the CTA exits
-      umma_commit(bar(BAR_TEARDOWN));
-      mbar_drain(bar(BAR_TEARDOWN), 0, st, 25);
-      mbar_drain(bar(BAR_B), 0, st, 20);
-    }
   } else if (warp >= 4) {
+    if constexpr (kInt4) setmaxnreg_inc<kRegsEpi>();
     // ============================================================ epilogue (warps 4-11)
     // Two warpgroups split the 64 RoPE frequency pairs of every key (wg 0:
     // pairs [0, 32), wg 1: [32, 64)) for both heads, then each finishes one head.
@@ -710,12 +472,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Partial scores of both heads over this warpgroup's 32 frequency pairs i:
     //   score += c_i (q'_i k_i + q'_{i+64} k_{i+64}) + s_i (q'_{i+64} k_i - q'_i k_{i+64})
     // which is q'·k' with k' the key rotated by the token's angle (rotate-half).
-    // Contiguous positions (pos = t0 + row): (c, s) at t0 + row come from the
-    // tile base at t0 (one sincos per warp lane per tile) and this thread's
-    // fixed offset `row`, by angle addition; explicit positions take a sincos
-    // per token.  Math runs on packed fp32 pairs (two frequencies at a time).
+    // Explicit positions take a sincos per token.  Contiguous positions (pos = t0 +
+    // row): with (C, S) the cosine and sine at the tile start t0 and (c_r, s_r) those
+    // at this thread's fixed offset `row`, angle addition turns the sum into
+    //   score += c_r (k_i A_i + k_{i+64} B_i) + s_r (k_i B_i - k_{i+64} A_i),
+    //   A_i = C q'_i + S q'_{i+64},  B_i = C q'_{i+64} - S q'_i,
+    // i.e. the query rotated by the tile start, computed once per tile for the whole
+    // warpgroup (double-buffered, published by the tile's softmax sync).  Math runs
+    // on packed fp32 pairs (two frequencies at a time).
     constexpr bool contig = CONTIG;
-    float* tbw = reinterpret_cast<float*>(sbase + L.tb) + (warp - 4) * 96;   // [cos|sin|-sin][32]
+    float* abuf = reinterpret_cast<float*>(sbase + L.tb) + wg * 384;   // [tile parity][head][A|B|-A][32]
     f2 crow[16], srow[16];
     if (contig) {
 #pragma unroll
@@ -727,16 +493,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         srow[v] = f2_pack(s0, s1);
       }
     }
+    // the query rotated by the start t0 of a tile, for this warpgroup's frequencies:
+    // thread row < 64 takes frequency row mod 32 of head row / 32
+    auto post_rotated_query = [&](int t0, int parity) {
+      if (row >= 64) return;
+      const int f = row & 31, hh = row >> 5;
+      float c, sn;
+      rope_cs_fast(t0, om[wg * 32 + f], c, sn);
+      const float qa = qr[hh * 192 + wg * 32 + f], qb = qr[hh * 192 + 64 + wg * 32 + f];
+      const float A = c * qa + sn * qb, B = c * qb - sn * qa;
+      float* o = abuf + parity * 192 + hh * 96 + f;
+      o[0] = A;
+      o[32] = B;
+      o[64] = -A;
+    };
     auto half_scores = [&](int slot, int t0, int pos, float* part, auto&& mid) {
-      if (contig) {
-        float c, sn;
-        rope_cs_fast(t0, om[wg * 32 + lane], c, sn);
-        __syncwarp();
-        tbw[lane] = c;
-        tbw[32 + lane] = sn;
-        tbw[64 + lane] = -sn;
-        __syncwarp();
-      }
+      const float* ab = abuf + ((t0 / kTile) & 1) * 192;
       f2 acc[2][2];
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) acc[hh][0] = acc[hh][1] = 0ull;
@@ -759,27 +531,39 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld8(col + 192, hi[1]);
         }
         tmem_wait_ld();
+        if (contig) {
+#pragma unroll
+          for (int v4 = 0; v4 < kBatch / 4; ++v4) {
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              const float* q = ab + hh * 96 + jj * kBatch + 4 * v4;
+              const float4 A4 = *reinterpret_cast<const float4*>(q);
+              const float4 B4 = *reinterpret_cast<const float4*>(q + 32);
+              const float4 N4 = *reinterpret_cast<const float4*>(q + 64);
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                const int v = v4 * 2 + e, vr = jj * (kBatch / 2) + v;
+                const f2 A2 = e ? f2_pack(A4.z, A4.w) : f2_pack(A4.x, A4.y);
+                const f2 B2 = e ? f2_pack(B4.z, B4.w) : f2_pack(B4.x, B4.y);
+                const f2 N2 = e ? f2_pack(N4.z, N4.w) : f2_pack(N4.x, N4.y);
+                const f2 lo2 = f2_pack(lo[hh][2 * v], lo[hh][2 * v + 1]);
+                const f2 hi2 = f2_pack(hi[hh][2 * v], hi[hh][2 * v + 1]);
+                const f2 u = f2_fma(hi2, B2, f2_mul(lo2, A2));   // k_i A_i + k_{i+64} B_i
+                const f2 w = f2_fma(lo2, B2, f2_mul(hi2, N2));   // k_i B_i - k_{i+64} A_i
+                acc[hh][e] = f2_fma(crow[vr], u, acc[hh][e]);
+                acc[hh][e] = f2_fma(srow[vr], w, acc[hh][e]);
+              }
+            }
+          }
+          continue;
+        }
 #pragma unroll
         for (int v4 = 0; v4 < kBatch / 4; ++v4) {
-          float4 cb4 = make_float4(0.f, 0.f, 0.f, 0.f), sb4 = cb4, nb4 = cb4;
-          if (contig) {
-            cb4 = reinterpret_cast<const float4*>(tbw + jj * kBatch)[v4];
-            sb4 = reinterpret_cast<const float4*>(tbw + 32 + jj * kBatch)[v4];
-            nb4 = reinterpret_cast<const float4*>(tbw + 64 + jj * kBatch)[v4];
-          }
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const int v = v4 * 2 + e;
             f2 cs, sn;
-            if (contig) {
-              const f2 c0 = e ? f2_pack(cb4.z, cb4.w) : f2_pack(cb4.x, cb4.y);
-              const f2 s0 = e ? f2_pack(sb4.z, sb4.w) : f2_pack(sb4.x, sb4.y);
-              const f2 n0 = e ? f2_pack(nb4.z, nb4.w) : f2_pack(nb4.x, nb4.y);
-              // cos(t0+row) = c0 cr - s0 sr ; sin(t0+row) = s0 cr + c0 sr
-              const int vr = jj * (kBatch / 2) + v;
-              cs = f2_fma(c0, crow[vr], f2_mul(n0, srow[vr]));
-              sn = f2_fma(s0, crow[vr], f2_mul(c0, srow[vr]));
-            } else {
+            {
               // explicit positions: a sincos per token
               float c0, s0, c1, s1;
               rope_cs_fast(pos, om[i0 + 2 * v], c0, s0);
@@ -843,6 +627,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int nv_tiles = tr.ntiles - (tr.ragged_last ? 1 : 0);   // tiles whose value sums are MMAs
       // causal bound (several queries per step): tokens after the query's position are masked
       const int qlim = a.causal ? a.q_pos[(size_t)b * a.qpos_bstride] : 0;
+      if (contig && tr.ntiles > 0) {
+        post_rotated_query(tr.t_begin, (tr.t_begin / kTile) & 1);
+        ok = ep_sync(37) && ok;
+      }
       for (int k = 0; k < tr.ntiles && ok; ++k) {
         const int t0 = tr.t_begin + k * kTile;
         int pos = t0 + row;
@@ -864,6 +652,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(bar(BAR_MID));
         });
+        // the next tile's rotated query; the tile-max sync below publishes it
+        if (contig) post_rotated_query(t0 + kTile, ((t0 / kTile) + 1) & 1);
         psc[(slot * 2 + (1 - hw)) * 128 + row] = part[1 - hw];
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(BAR_XCH + slot));
@@ -947,6 +737,272 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int mb = 0; mb < NRV; ++mb) out[2 + mb * 128 + vrow] = acc[mb];
       }
     }
+  } else {
+    // warps 0-3
+    if constexpr (kInt4) setmaxnreg_dec<kRegsW0>();
+    if (kInt4 && warp != 1) {
+      // ============================================================ int4 value codes (warps 0, 2, 3)
+      // Ring stage s of a tile (s = 2mb + cb) = entries [64s, 64s + 64) of all 128
+      // tokens = 16-byte units 2s and 2s+1 of each token's row of codes: 256 (token,
+      // unit) items, dealt to the 96 threads round-robin (item i: token i mod 128, unit
+      // 2s + i / 128) and loaded straight into registers two stages ahead of the
+      // conversion.  Units are written PAIRED: row r of the value operand holds entry
+      // paired_row(r).
+      const int vt = (warp == 0 ? 0 : warp == 2 ? 32 : 64) + lane;
+      const int nv_tiles = tr.ntiles - (tr.ragged_last ? 1 : 0);
+      constexpr int kSPT = 2 * NRV;                      // ring stages per tile
+      const int N = nv_tiles * kSPT;
+      struct Slot {
+        uint4 raw[3];
+        uint16_t sc[3];
+      };
+      // pg = the raw table entry of stage n's tile, read a tile earlier
+      auto issue = [&](int n, Slot& sl, int pg) {
+        if (n >= N) return;
+        if (!page_valid(a, pg)) pg = 0;   // reported by the key converters
+        const uint8_t* blk = gm.zv[gi] + (size_t)pg * gm.v_page;
+        const uint8_t* sblk = gm.zvs[gi] + (size_t)pg * gm.vs_page;
+        const int s = n % kSPT;
+  #pragma unroll
+        for (int j = 0; j < 3; ++j) {
+          const int i = vt + 96 * j;
+          if (i < 256) {
+            const int t = i & 127, u = 2 * s + (i >> 7);
+            sl.raw[j] = __ldg(reinterpret_cast<const uint4*>(blk + t * 128 + ((u ^ (t & 7)) << 4)));
+            sl.sc[j] = __ldg(reinterpret_cast<const unsigned short*>(sblk + (size_t)t * a.vs_row + 2 * u));
+          }
+        }
+      };
+      int stage = 0;
+      uint32_t phase = 0;
+      auto consume = [&](int n, const Slot& sl) -> bool {
+        if (n >= N) return true;
+        if (!mbar_wait(bar(BAR_ZV_EMPTY + stage), phase ^ 1, abort_flag, st, 13)) return false;
+        if (vt == 0 && n % kSPT == 0) trace(6, n / kSPT);
+        const uint32_t dst = base + L.zv + stage * kZvBytes;
+  #pragma unroll
+        for (int j = 0; j < 3; ++j) {
+          const int i = vt + 96 * j;
+          if (i < 256) {
+            const int t = i & 127, ub = i >> 7;
+            const uint32_t w[4] = {sl.raw[j].x, sl.raw[j].y, sl.raw[j].z, sl.raw[j].w};
+  #pragma unroll
+            for (int m = 0; m < 4; ++m)
+              st_shared_v4(dst + t * 128 + (((4 * ub + m) ^ (t & 7)) << 4), dequant8<ACT, true>(w[m], sl.sc[j]));
+          }
+        }
+        fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(BAR_ZV_FULL + stage));
+        if (++stage == kNVS) { stage = 0; phase ^= 1; }
+        return true;
+      };
+      Slot s0, s1, s2;                                   // stages n, n+1; s2 takes n+2
+      int pg_k = page_ahead(a, b, tr, 0);                // tile k of stage n
+      int pg_k1 = page_ahead(a, b, tr, 1);               // tile k+1
+      int pg_k2 = page_ahead(a, b, tr, 2);               // tile k+2, in flight
+      issue(0, s0, pg_k);
+      issue(1, s1, pg_k);
+  #pragma unroll 1
+      for (int n = 0; n < N && !*abort_flag; ++n) {
+        if (n % kSPT == 0 && n > 0) {
+          pg_k = pg_k1;
+          pg_k1 = pg_k2;
+          pg_k2 = page_ahead(a, b, tr, n / kSPT + 2);
+        }
+        issue(n + 2, s2, (n + 2) / kSPT == n / kSPT ? pg_k : pg_k1);
+        if (!consume(n, s0)) break;
+        s0 = s1;
+        s1 = s2;
+      }
+    } else if (warp == 0) {
+      // ============================================================ z_k producer (bulk copies)
+      if (lane == 0) {
+        int stage = 0;
+        uint32_t phase = 0;
+        // No bulk L2 prefetch of later pages here: with the bulk copies of the two
+        // head-pair CTAs of a group in flight, a prefetch 3 or 6 pages ahead left the
+        // copy latency unchanged and the call 2-3 % slower.
+        int pg_next = page_ahead(a, b, tr, 0);
+        long long issued = 0;
+        for (int k = 0; k < tr.ntiles && !*abort_flag; ++k) {
+          int pg = pg_next;
+          pg_next = page_ahead(a, b, tr, k + 1);   // in flight during this tile's copies
+          if (!page_valid(a, pg)) {
+            report(st, PALU_ERR_DEVICE_BOUNDS, 2000000 + b);
+            pg = 0;   // keep the pipeline fed from a valid page; the status says the result is void
+          }
+          // one (page, group) block is the shared-memory image of the tile: each
+          // 128-byte column block (64 latent entries of all 128 tokens) is one copy
+          const uint8_t* src = gm.zk[gi] + (size_t)pg * gm.k_page;
+          for (int c = 0; c < nkc; ++c) {
+            if (!mbar_wait(bar(BAR_ZK_EMPTY + stage), phase ^ 1, abort_flag, st, 10)) break;
+            mbar_expect_tx(bar(BAR_ZK_FULL + stage), kZkBytes);
+            bulk_load(base + L.zk + stage * kZkBytes, src + (size_t)c * kZkBytes, kZkBytes, bar(BAR_ZK_FULL + stage));
+            ++issued;
+            if (++stage == kNZK) { stage = 0; phase ^= 1; }
+          }
+        }
+        drain_ring(bar(BAR_ZK_FULL), kNZK, issued, st, 10);
+      }
+    } else if (warp == 2) {
+      // ============================================================ z_v producer (bulk copies)
+      if (lane == 0) {
+        int stage = 0;
+        uint32_t phase = 0;
+        int pg_next = page_ahead(a, b, tr, 0);
+        long long issued = 0;
+        for (int k = 0; k < tr.ntiles && !*abort_flag; ++k) {
+          if (tr.ragged_last && k == tr.ntiles - 1) break;    // CUDA-core value sum for a partial page
+          int pg = pg_next;
+          pg_next = page_ahead(a, b, tr, k + 1);   // in flight during this tile's copies
+          if (!page_valid(a, pg)) pg = 0;   // reported by the z_k producer
+          const uint8_t* src = gm.zv[gi] + (size_t)pg * gm.v_page;
+          // one copy per 128-byte column block of the page (64 latent entries of
+          // all 128 tokens); two consecutive blocks are the two MN-blocks of one
+          // value-MMA operand
+          for (int cb = 0; cb < 2 * NRV; ++cb) {
+            if (!mbar_wait(bar(BAR_ZV_EMPTY + stage), phase ^ 1, abort_flag, st, 11)) break;
+            mbar_expect_tx(bar(BAR_ZV_FULL + stage), kZvBytes);
+            bulk_load(base + L.zv + stage * kZvBytes, src + (size_t)cb * a.P * 128, kZvBytes,
+                      bar(BAR_ZV_FULL + stage));
+            if (cb == 0) trace(6, k);
+            ++issued;
+            if (++stage == kNVS) { stage = 0; phase ^= 1; }
+          }
+        }
+        drain_ring(bar(BAR_ZV_FULL), kNVS, issued, st, 11);
+      }
+    } else if (warp == 1) {
+      // ============================================================ MMA issuer
+      if (lane == 0) {
+        constexpr int kBf = ACT == PALU_BF16 ? 1 : 0;
+        const uint32_t idesc_d = idesc_f16(kBf, 0, 1, 256, 128);    // z_k K-major, B_k MN-major
+        const uint32_t idesc_pv = idesc_f16(kBf, 1, 0, 16, 128);    // z_vᵀ MN-major, Pᵀ K-major
+        const uint32_t b_lbo = (uint32_t)r_k * 128;                  // bytes between 64-column blocks of B
+        int zs = 0;
+        uint32_t zph = 0, vph = 0;
+        // timeout-path test hook: first wait on a phase nothing completes before the teardown commit
+        bool ok = a.stall_test == 0 || mbar_wait(bar(BAR_TEARDOWN), 0, abort_flag, st, 26);
+        ok = ok && mbar_wait(bar(BAR_B), 0, abort_flag, st, 20);
+        const int nv_tiles = tr.ntiles - (tr.ragged_last ? 1 : 0);   // tiles whose value sums run here
+        int pv_next = 0;       // next tile whose value MMA is not issued yet
+        int pv_mb = 0;         // next 128-entry block of that value MMA
+        int zv_seen = -1;      // last tile whose value latents were seen in shared memory (trace)
+
+        // The value MMA of tile j, aᵀ[128 entries × 16] per block = z_vᵀ · Pᵀ, goes into
+        // columns [32·mb, +16) of the TMEM slot of tile j + 1: columns whose keys that
+        // tile's epilogue has read by the middle of its score pass (BAR_MID), so the value
+        // round trip never holds a slot back from the next key MMA.  The last tile's value
+        // MMA goes into the other slot once it is free.  Its gate (besides P and z_v):
+        auto pv_gate = [&](int j) -> bool {
+          if (j + 1 < tr.ntiles) return mbar_test_wait(bar(BAR_MID), (uint32_t)((j + 1) & 1));
+          const int u = j + 1;
+          return mbar_test_wait(bar(BAR_D_EMPTY + (u & 1)), (uint32_t)(((u >> 1) & 1) ^ 1));
+        };
+        // The next block of the pending value MMA can go?  (Phases cannot alias: the
+        // epilogue cannot pass tile j + 1 before the value sums of tile j are folded.)
+        auto pv_ready = [&]() -> bool {
+          if (pv_next >= nv_tiles) return false;
+          if (!(mbar_test_wait(bar(BAR_ZV_FULL + 0), vph) && mbar_test_wait(bar(BAR_ZV_FULL + 1), vph))) return false;
+          if (pv_mb == 0 && zv_seen != pv_next) {
+            zv_seen = pv_next;
+            trace(7, pv_next);
+          }
+          return pv_mb > 0 || (mbar_test_wait(bar(BAR_P_FULL + (pv_next & 1)), (uint32_t)((pv_next >> 1) & 1)) &&
+                               pv_gate(pv_next));
+        };
+        auto issue_pv_block = [&]() {
+          const int j = pv_next;
+          tc_fence_after();
+          const uint32_t a_tmem = tmem + (uint32_t)((j + 1) & 1) * 256 + (uint32_t)pv_mb * 32;
+          const uint32_t p_base = base + L.p + (uint32_t)(j & 1) * kPBytes;
+          static_assert(kNVS == 2, "one value MMA operand = the two ring stages");
+  #pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk) {
+            // rows = latent entries (two 64-entry blocks, one per stage), K = tokens
+            const uint64_t ad = sdesc(base + L.zv + kk * 16 * 128, kZvBytes, 1024, kSw128);
+            const uint64_t bd = sdesc(p_base + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024, kSw128);
+            umma_f16(a_tmem, ad, bd, idesc_pv, kk != 0);
+          }
+          umma_commit(bar(BAR_ZV_EMPTY + 0));
+          umma_commit(bar(BAR_ZV_EMPTY + 1));
+          vph ^= 1;
+          if (++pv_mb == NRV) {
+            umma_commit(bar(BAR_AT_FULL));
+            trace(2, j);
+            ++pv_next;
+            pv_mb = 0;
+          }
+        };
+        // Wait for a barrier phase; meanwhile issue every value-MMA block whose operands
+        // and gate are in (the epilogue's slot releases depend on them).  Bounded.
+        auto poll_wait = [&](uint32_t b, uint32_t parity, int where) -> bool {
+          const long long t0 = clock64();
+          while (true) {
+            if (mbar_test_wait(b, parity)) return true;
+            if (pv_ready()) {
+              issue_pv_block();
+              continue;
+            }
+            if (*abort_flag) return false;
+            __nanosleep(64);   // leave the issue slots of this SM partition to the epilogue warps
+            if (clock64() - t0 > wait_limit(abort_flag)) {
+              report(st, PALU_ERR_DEVICE_TIMEOUT, where);
+              *abort_flag = 1;
+              return false;
+            }
+          }
+        };
+
+        for (int k = 0; k < tr.ntiles && ok; ++k) {
+          const int slot = k & 1;
+          if (!poll_wait(bar(BAR_D_EMPTY + slot), ((k >> 1) & 1) ^ 1, 23)) { ok = false; break; }
+          tc_fence_after();
+          trace(0, k);
+          const uint32_t d_tmem = tmem + (uint32_t)slot * 256;
+          for (int c = 0; c < nkc; ++c) {
+            if (!poll_wait(bar(BAR_ZK_FULL + zs), zph, 24)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t zk_addr = base + L.zk + zs * kZkBytes;
+            const uint32_t b_addr = base + L.b + (uint32_t)c * kChunk * 128;
+  #pragma unroll
+            for (int kk = 0; kk < kChunk / 16; ++kk) {
+              const uint64_t ad = sdesc(zk_addr + kk * 32, 16, kZkSbo, kZkSwz);
+              const uint64_t bd = sdesc(b_addr + kk * 16 * 128, b_lbo, 1024, kSw128);
+              umma_f16(d_tmem, ad, bd, idesc_d, (c | kk) != 0);
+            }
+            umma_commit(bar(BAR_ZK_EMPTY + zs));
+            if (++zs == kNZK) { zs = 0; zph ^= 1; }
+          }
+          if (!ok) break;
+          umma_commit(bar(BAR_D_FULL + slot));
+          trace(1, k);
+        }
+        // the value MMAs still pending (the last tiles'), each once its operands are in
+        if (ok) {
+          const long long t0 = clock64();
+          while (pv_next < nv_tiles) {
+            if (pv_ready()) {
+              issue_pv_block();
+              continue;
+            }
+            if (*abort_flag) break;
+            __nanosleep(64);
+            if (clock64() - t0 > wait_limit(abort_flag)) {
+              report(st, PALU_ERR_DEVICE_TIMEOUT, 21);
+              *abort_flag = 1;
+              break;
+            }
+          }
+        }
+        // drain, also after an abort: every MMA issued above has completed before
+        // TMEM is released, and the B_k load has landed before the CTA exits
+        umma_commit(bar(BAR_TEARDOWN));
+        mbar_drain(bar(BAR_TEARDOWN), 0, st, 25);
+        mbar_drain(bar(BAR_B), 0, st, 20);
+      }
+    }
   }
 
   // ---------------------------------------------------------------- teardown
@@ -1009,8 +1065,17 @@ cudaError_t launch_t(const DecodeArgs& a, cudaStream_t st) {
   }
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
+  if constexpr (LAT == PALU_INT4) {
+    // The warpgroups' setmaxnreg split adds up to exactly the registers of a launch at
+    // kRegsLaunch per thread; launched with fewer, the epilogue's increase could never
+    // be granted.  Refuse to launch a build whose kernel is not at that count.
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, kern);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs != (int)kRegsLaunch) return cudaErrorInvalidConfiguration;
+  }
   dim3 grid(a.S, a.gm.n * (a.gs / 2), a.batch);
-  kern<<<grid, kThreads, smem, st>>>(tm_bk, args);
+  kern<<<grid, threads_of(LAT == PALU_INT4), smem, st>>>(tm_bk, args);
   count_launch();
   return cudaGetLastError();
 }

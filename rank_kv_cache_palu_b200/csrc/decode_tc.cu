@@ -44,10 +44,15 @@ using namespace tc;
 
 constexpr int kTile = 128;         // tokens per tile = page size
 constexpr int kChunk = 64;         // K chunk of z_k (elements) = one 128-byte column block of the page
-constexpr int kNKS = 3;            // z_k ring stages (barrier slots)
+constexpr int kNKS = 3;            // barrier slots of each ring (the most stages either ring has)
 constexpr uint32_t kZkSwz = 2u;    // 128-byte swizzle
 constexpr uint32_t kZkSbo = 1024;  // bytes per 8-row swizzle atom
-constexpr int kNVS = 2;            // z_v ring stages
+// Ring depths.  A z_v stage is one value-MMA operand of 128 latent entries × 64 tokens (two
+// 64-entry column blocks of a token half), so stages are independent.  16-bit latents: 3 z_k
+// stages, 2 z_v stages.  int4 latents convert codes locally, so the key ring needs less depth
+// and the value ring gets a third stage: the value operand is converted ahead of its MMAs.
+__host__ __device__ constexpr int zk_stages(bool int4) { return int4 ? 2 : 3; }
+__host__ __device__ constexpr int zv_stages(bool int4) { return int4 ? 3 : 2; }
 constexpr int kPrefetch = 3;       // int4: pages of codes pulled into L2 ahead of the loads
 constexpr int kBatch = 8;          // frequency pairs per TMEM round trip of the score pass
 constexpr int kNB = 32 / kBatch;   // score batches per warpgroup and tile
@@ -73,10 +78,9 @@ struct Smem {
 // so the kernel's offsets are compile-time constants; B_k comes last.
 __host__ __device__ inline Smem smem_layout(int r_k, bool int4) {
   Smem s{};
-  (void)int4;   // int4 codes are converted straight from global memory into the same rings
   uint32_t o = 0;
-  s.zk = o;     o += kNKS * kZkBytes;
-  s.zv = o;     o += kNVS * kZvBytes;
+  s.zk = o;     o += zk_stages(int4) * kZkBytes;
+  s.zv = o;     o += zv_stages(int4) * kZvBytes;
   s.p = o;      o += 2 * kPBytes;
   s.qr = o;     o += 3 * 128 * 4;                        // q'_i, q'_{i+64}, -q'_i per head pair row
   s.psc = o;    o += 2 * 2 * 128 * 4;
@@ -96,11 +100,11 @@ __host__ __device__ inline Smem smem_layout(int r_k, bool int4) {
 // barrier indices
 enum {
   BAR_B = 0,
-  BAR_ZK_FULL = 1,                   // kNKS
+  BAR_ZK_FULL = 1,                   // kNKS slots
   BAR_ZK_EMPTY = BAR_ZK_FULL + kNKS,
-  BAR_ZV_FULL = BAR_ZK_EMPTY + kNKS,  // kNVS
-  BAR_ZV_EMPTY = BAR_ZV_FULL + kNVS,
-  BAR_D_FULL = BAR_ZV_EMPTY + kNVS,  // 2
+  BAR_ZV_FULL = BAR_ZK_EMPTY + kNKS,  // kNKS slots
+  BAR_ZV_EMPTY = BAR_ZV_FULL + kNKS,
+  BAR_D_FULL = BAR_ZV_EMPTY + kNKS,  // 2
   BAR_D_EMPTY = BAR_D_FULL + 2,      // 2
   BAR_P_FULL = BAR_D_EMPTY + 2,      // 2
   BAR_AT_FULL = BAR_P_FULL + 2,      // 1
@@ -271,7 +275,9 @@ __global__ void __launch_bounds__(threads_of(LAT == PALU_INT4), 1)
   const Smem L = smem_layout(r_k, LAT == PALU_INT4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr bool kInt4 = LAT == PALU_INT4;
-  constexpr int kNZK = kNKS;
+  constexpr int kNZK = zk_stages(kInt4);
+  constexpr int kNVS = zv_stages(kInt4);
+  static_assert(kNZK <= kNKS && kNVS <= kNKS, "barrier slots");
   constexpr int kThreads = threads_of(kInt4);
   static_assert(!kInt4 || NRV == 2, "int4 latents: r_v = 256");
   DevStatus* st = reinterpret_cast<DevStatus*>(a.status);
@@ -742,12 +748,13 @@ __global__ void __launch_bounds__(threads_of(LAT == PALU_INT4), 1)
     if constexpr (kInt4) setmaxnreg_dec<kRegsW0>();
     if (kInt4 && warp != 1) {
       // ============================================================ int4 value codes (warps 0, 2, 3)
-      // Ring stage s of a tile (s = 2mb + cb) = entries [64s, 64s + 64) of all 128
-      // tokens = 16-byte units 2s and 2s+1 of each token's row of codes: 256 (token,
-      // unit) items, dealt to the 96 threads round-robin (item i: token i mod 128, unit
-      // 2s + i / 128) and loaded straight into registers two stages ahead of the
-      // conversion.  Units are written PAIRED: row r of the value operand holds entry
-      // paired_row(r).
+      // Ring stage s of a tile (s = 2mb + th) = entries [128mb, +128) of tokens
+      // [64th, +64) = 16-byte units 4mb .. 4mb+3 of those tokens' rows of codes: 256
+      // (token, unit) items, dealt to the 96 threads round-robin (item i: token
+      // 64th + i mod 64, unit 4mb + i / 64) and loaded straight into registers two
+      // stages ahead of the conversion.  Unit j = i / 64 lands in the stage's 64-entry
+      // block j / 2 (8 KB apart), its 32 entries written PAIRED: row r of the value
+      // operand holds entry paired_row(r).
       const int vt = (warp == 0 ? 0 : warp == 2 ? 32 : 64) + lane;
       const int nv_tiles = tr.ntiles - (tr.ragged_last ? 1 : 0);
       constexpr int kSPT = 2 * NRV;                      // ring stages per tile
@@ -762,12 +769,12 @@ __global__ void __launch_bounds__(threads_of(LAT == PALU_INT4), 1)
         if (!page_valid(a, pg)) pg = 0;   // reported by the key converters
         const uint8_t* blk = gm.zv[gi] + (size_t)pg * gm.v_page;
         const uint8_t* sblk = gm.zvs[gi] + (size_t)pg * gm.vs_page;
-        const int s = n % kSPT;
+        const int s = n % kSPT, mb = s >> 1, th = s & 1;
   #pragma unroll
         for (int j = 0; j < 3; ++j) {
           const int i = vt + 96 * j;
           if (i < 256) {
-            const int t = i & 127, u = 2 * s + (i >> 7);
+            const int t = 64 * th + (i & 63), u = 4 * mb + (i >> 6);
             sl.raw[j] = __ldg(reinterpret_cast<const uint4*>(blk + t * 128 + ((u ^ (t & 7)) << 4)));
             sl.sc[j] = __ldg(reinterpret_cast<const unsigned short*>(sblk + (size_t)t * a.vs_row + 2 * u));
           }
@@ -784,11 +791,12 @@ __global__ void __launch_bounds__(threads_of(LAT == PALU_INT4), 1)
         for (int j = 0; j < 3; ++j) {
           const int i = vt + 96 * j;
           if (i < 256) {
-            const int t = i & 127, ub = i >> 7;
+            const int tr64 = i & 63, blk = (i >> 7), ub = (i >> 6) & 1;   // token row, entry block, unit
             const uint32_t w[4] = {sl.raw[j].x, sl.raw[j].y, sl.raw[j].z, sl.raw[j].w};
+            const uint32_t row = dst + blk * (kZvBytes / 2) + tr64 * 128;
   #pragma unroll
             for (int m = 0; m < 4; ++m)
-              st_shared_v4(dst + t * 128 + (((4 * ub + m) ^ (t & 7)) << 4), dequant8<ACT, true>(w[m], sl.sc[j]));
+              st_shared_v4(row + (((4 * ub + m) ^ (tr64 & 7)) << 4), dequant8<ACT, true>(w[m], sl.sc[j]));
           }
         }
         fence_proxy_async();
@@ -858,9 +866,9 @@ __global__ void __launch_bounds__(threads_of(LAT == PALU_INT4), 1)
           pg_next = page_ahead(a, b, tr, k + 1);   // in flight during this tile's copies
           if (!page_valid(a, pg)) pg = 0;   // reported by the z_k producer
           const uint8_t* src = gm.zv[gi] + (size_t)pg * gm.v_page;
-          // one copy per 128-byte column block of the page (64 latent entries of
-          // all 128 tokens); two consecutive blocks are the two MN-blocks of one
-          // value-MMA operand
+          // one 16 KB copy per 128-byte column block of the page (64 latent entries of all
+          // 128 tokens); the two stages of the ring are the two 64-entry halves of one
+          // value-MMA operand (whole blocks copied faster than token halves of 8 KB)
           for (int cb = 0; cb < 2 * NRV; ++cb) {
             if (!mbar_wait(bar(BAR_ZV_EMPTY + stage), phase ^ 1, abort_flag, st, 11)) break;
             mbar_expect_tx(bar(BAR_ZV_FULL + stage), kZvBytes);
@@ -887,10 +895,11 @@ __global__ void __launch_bounds__(threads_of(LAT == PALU_INT4), 1)
         ok = ok && mbar_wait(bar(BAR_B), 0, abort_flag, st, 20);
         const int nv_tiles = tr.ntiles - (tr.ragged_last ? 1 : 0);   // tiles whose value sums run here
         int pv_next = 0;       // next tile whose value MMA is not issued yet
-        int pv_mb = 0;         // next 128-entry block of that value MMA
+        int pv_s = 0;          // next operand of that value MMA: block mb = pv_s / 2 (int4: token half pv_s % 2)
+        int vs = 0;            // int4: z_v ring stage of that operand
         int zv_seen = -1;      // last tile whose value latents were seen in shared memory (trace)
 
-        // The value MMA of tile j, aᵀ[128 entries × 16] per block = z_vᵀ · Pᵀ, goes into
+        // The value MMA of tile j, aᵀ[128 entries × 16] per block mb = z_vᵀ · Pᵀ, goes into
         // columns [32·mb, +16) of the TMEM slot of tile j + 1: columns whose keys that
         // tile's epilogue has read by the middle of its score pass (BAR_MID), so the value
         // round trip never holds a slot back from the next key MMA.  The last tile's value
@@ -900,39 +909,67 @@ __global__ void __launch_bounds__(threads_of(LAT == PALU_INT4), 1)
           const int u = j + 1;
           return mbar_test_wait(bar(BAR_D_EMPTY + (u & 1)), (uint32_t)(((u >> 1) & 1) ^ 1));
         };
-        // The next block of the pending value MMA can go?  (Phases cannot alias: the
+        // The next stage of the pending value MMA can go?  (Phases cannot alias: the
         // epilogue cannot pass tile j + 1 before the value sums of tile j are folded.)
+        // int4: one ring stage per operand (mb, th); 16-bit latents: the two stages of the
+        // ring hold the two 64-entry halves of operand mb over all 128 tokens.
         auto pv_ready = [&]() -> bool {
           if (pv_next >= nv_tiles) return false;
-          if (!(mbar_test_wait(bar(BAR_ZV_FULL + 0), vph) && mbar_test_wait(bar(BAR_ZV_FULL + 1), vph))) return false;
-          if (pv_mb == 0 && zv_seen != pv_next) {
+          if constexpr (kInt4) {
+            if (!mbar_test_wait(bar(BAR_ZV_FULL + vs), vph)) return false;
+          } else {
+            if (!(mbar_test_wait(bar(BAR_ZV_FULL + 0), vph) && mbar_test_wait(bar(BAR_ZV_FULL + 1), vph)))
+              return false;
+          }
+          if (pv_s == 0 && zv_seen != pv_next) {
             zv_seen = pv_next;
             trace(7, pv_next);
           }
-          return pv_mb > 0 || (mbar_test_wait(bar(BAR_P_FULL + (pv_next & 1)), (uint32_t)((pv_next >> 1) & 1)) &&
-                               pv_gate(pv_next));
+          return pv_s > 0 || (mbar_test_wait(bar(BAR_P_FULL + (pv_next & 1)), (uint32_t)((pv_next >> 1) & 1)) &&
+                              pv_gate(pv_next));
         };
+        // One value-MMA operand into block mb of the value sums.  int4: stage (mb, th) =
+        // latent entries [128mb, +128) (two 64-entry blocks 8 KB apart) × tokens [64th, +64),
+        // against the matching half of Pᵀ.  16-bit latents: the two ring stages (64 entries
+        // of all 128 tokens each) against all of Pᵀ.
         auto issue_pv_block = [&]() {
           const int j = pv_next;
           tc_fence_after();
-          const uint32_t a_tmem = tmem + (uint32_t)((j + 1) & 1) * 256 + (uint32_t)pv_mb * 32;
           const uint32_t p_base = base + L.p + (uint32_t)(j & 1) * kPBytes;
-          static_assert(kNVS == 2, "one value MMA operand = the two ring stages");
+          if constexpr (kInt4) {
+            const int mb = pv_s >> 1, th = pv_s & 1;
+            const uint32_t a_tmem = tmem + (uint32_t)((j + 1) & 1) * 256 + (uint32_t)mb * 32;
+            const uint32_t z_base = base + L.zv + (uint32_t)vs * kZvBytes;
   #pragma unroll
-          for (int kk = 0; kk < kTile / 16; ++kk) {
-            // rows = latent entries (two 64-entry blocks, one per stage), K = tokens
-            const uint64_t ad = sdesc(base + L.zv + kk * 16 * 128, kZvBytes, 1024, kSw128);
-            const uint64_t bd = sdesc(p_base + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024, kSw128);
-            umma_f16(a_tmem, ad, bd, idesc_pv, kk != 0);
+            for (int kk = 0; kk < 4; ++kk) {
+              // rows = latent entries, K = 16 tokens of the half
+              const uint64_t ad = sdesc(z_base + kk * 16 * 128, kZvBytes / 2, 1024, kSw128);
+              const uint64_t bd = sdesc(p_base + th * 2048 + kk * 32, 16, 1024, kSw128);
+              umma_f16(a_tmem, ad, bd, idesc_pv, (th | kk) != 0);
+            }
+            umma_commit(bar(BAR_ZV_EMPTY + vs));
+            if (++vs == kNVS) { vs = 0; vph ^= 1; }
+            ++pv_s;
+          } else {
+            static_assert(kInt4 || zv_stages(false) == 2, "one value MMA operand = the two ring stages");
+            const uint32_t a_tmem = tmem + (uint32_t)((j + 1) & 1) * 256 + (uint32_t)(pv_s >> 1) * 32;
+  #pragma unroll
+            for (int kk = 0; kk < kTile / 16; ++kk) {
+              // rows = latent entries (two 64-entry blocks, one per stage), K = tokens
+              const uint64_t ad = sdesc(base + L.zv + kk * 16 * 128, kZvBytes, 1024, kSw128);
+              const uint64_t bd = sdesc(p_base + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024, kSw128);
+              umma_f16(a_tmem, ad, bd, idesc_pv, kk != 0);
+            }
+            umma_commit(bar(BAR_ZV_EMPTY + 0));
+            umma_commit(bar(BAR_ZV_EMPTY + 1));
+            vph ^= 1;
+            pv_s += 2;
           }
-          umma_commit(bar(BAR_ZV_EMPTY + 0));
-          umma_commit(bar(BAR_ZV_EMPTY + 1));
-          vph ^= 1;
-          if (++pv_mb == NRV) {
+          if (pv_s == 2 * NRV) {
             umma_commit(bar(BAR_AT_FULL));
             trace(2, j);
             ++pv_next;
-            pv_mb = 0;
+            pv_s = 0;
           }
         };
         // Wait for a barrier phase; meanwhile issue every value-MMA block whose operands

@@ -102,9 +102,11 @@ int auto_splits(const palu_config* c, int batch, int max_pages, int kind, int qn
   // (pages per split + a start-up of ~2 pages); with several queries per pass the
   // combine adds about a page per split and query (measured: 4 queries per pass at
   // 16 x 16k ran best at 4 splits, one query at 8).  Take the split count that minimises that (the
-  // smallest on ties), sized for the longest possible sequence (max_pages).  At
-  // least one full round of CTAs when the pages allow.
+  // smallest on ties), sized for the longest possible sequence (max_pages), from one full round
+  // of CTAs up -- or from the largest count that fits one round when that keeps >= 90 % of the
+  // SMs busy (a round a few SMs short beats two rounds when the units do not divide the SM count).
   long long S0 = (sms + units - 1) / units;
+  if (units * (sms / units) * 10 >= 9LL * sms) S0 = sms / units;
   if (S0 > max_pages) S0 = max_pages;
   if (S0 < 1) S0 = 1;
   long long best_S = S0, best_t = -1;

@@ -243,10 +243,14 @@ def test_ranked_workspace_covers_every_decode_set():
 
 
 def test_split_count_model():
-    # tensor-core launches: the split count minimises ceil(units·S / 148) · (pages/S + 2) over at
-    # least one full round of CTAs (smallest on ties); a pass of several fused queries adds S·Q
+    # tensor-core launches: the split count minimises ceil(units·S / 148) · (pages/S + 2) from one
+    # full round of CTAs up, or from the largest count fitting one round when that keeps >= 90 % of
+    # the SMs busy (smallest on ties); a pass of several fused queries adds S·Q
     def model(units, pages, qn=1):
-        s0 = max(1, min(pages, -(-148 // units)))
+        s0 = -(-148 // units)
+        if units * (148 // units) * 10 >= 9 * 148:
+            s0 = 148 // units
+        s0 = max(1, min(pages, s0))
         best = None
         for S in range(s0, min(pages, 64) + 1):
             t = -(-units * S // 148) * (-(-pages // S) + 2) + (S * qn if qn > 1 else 0)

@@ -80,7 +80,7 @@ def measured_peaks() -> dict:
 # The sources the decode kernels are built from (their own files and the headers of
 # the package they include; from include/palu.h they take only the ABI-fixed dtype
 # and status codes); a committed traffic figure is used only while these are unchanged.
-DECODE_SOURCES = ["decode_tc.cu", "decode_fused.cu", "decode_simt.cu", "palu_common.cuh", "palu_internal.h",
+DECODE_SOURCES = ["decode_tc.cu", "decode_tc_int4.cu", "decode_tc_kernel.cuh", "decode_fused.cu", "decode_simt.cu", "palu_common.cuh", "palu_internal.h",
                   "palu_tc.h", "tc_ptx.cuh"]
 
 

@@ -88,39 +88,69 @@ __device__ __forceinline__ int a_column(const GroupMap& gm, const uint16_t* cols
   return row0[e] + (lc - cols[e]);
 }
 
-// Write latent entry j of one token into its (page, group) block.
-template <int LAT>
-__device__ __forceinline__ void store_latent(const CompressArgs& a, uint8_t* blk, int j, int slot, float v) {
-  using TL = typename Dt<LAT>::T;
-  *reinterpret_cast<TL*>(blk + swz_offset(slot % a.P, (long long)j * sizeof(TL), a.P)) = Dt<LAT>::from_f(v);
+// Where the tokens of a tile go: page (slot / P, or -1 for a token that is not
+// stored) and row (slot % P) of every token, filled once per tile into shared
+// memory by the epilogue threads, so the per-token stores never wait on a
+// dependent load of the slot mapping.  An out-of-range slot is reported.
+__device__ __forceinline__ void fill_token_table(const CompressArgs& a, int t0, int ntok, int2* tab, int tid,
+                                                 int nthr, DevStatus* st) {
+  const long long cap = (long long)a.num_pages * a.P;
+  for (int i = tid; i < ntok; i += nthr) {
+    const int slot = a.slots[t0 + i];
+    int2 d = make_int2(-1, 0);
+    if (slot >= cap) report(st, PALU_ERR_DEVICE_BOUNDS, 3000000 + t0 + i);
+    else if (slot >= 0) d = make_int2(slot / a.P, slot % a.P);
+    tab[i] = d;
+  }
 }
 
-// Write 16 tokens (t0 + j0 .. t0 + j0 + 15, fewer at the end) of latent column gc
-// (this thread's; its warp holds 32 consecutive columns) into the paged cache:
+// The fixed part of this thread's latent column in the paged cache: its group's
+// pool, the column block and 16-byte unit of its entry (before the token's
+// swizzle), and for int4 the scale pool.  Latent entry j of token row t sits at
+// block (j·es / 128)·P·128 + t·128 + (((j·es / 16) mod 8) xor (t mod 8))·16 + j·es mod 16.
+struct ColDst {
+  uint8_t* col;          // pool + page-independent part of the offset
+  long long page_bytes;  // stride between pages
+  int unit;              // 16-byte unit before the swizzle
+  bool ok;               // a real column of this launch
+  uint8_t* spool;        // int4: scale pool + this column's scale slot
+  long long spage, srow;
+};
+
+template <int LAT>
+__device__ __forceinline__ ColDst col_dst(const CompressArgs& a, bool is_v, const uint16_t* cols, int ncols, int gc) {
+  ColDst d{};
+  d.ok = gc < ncols;
+  const int e = d.ok ? col_entry(cols, a.gm.n, gc) : 0;   // group entry of this column
+  const int j = d.ok ? gc - cols[e] : 0;                    // latent entry within it
+  long long o = j >> 1;                                     // int4: two entries per byte
+  if constexpr (LAT != PALU_INT4) o = (long long)j * (long long)sizeof(typename Dt<LAT>::T);
+  d.col = const_cast<uint8_t*>(is_v ? a.gm.zv[e] : a.gm.zk[e]) + (o >> 7) * (long long)a.P * 128 + (o & 15);
+  d.page_bytes = is_v ? a.gm.v_page : a.gm.k_page;
+  d.unit = (int)((o >> 4) & 7);
+  if constexpr (LAT == PALU_INT4) {
+    d.spool = const_cast<uint8_t*>(is_v ? a.gm.zvs[e] : a.gm.zks[e]) + 2 * (j >> 5);
+    d.spage = is_v ? a.gm.vs_page : a.gm.ks_page;
+    d.srow = int4_scale_row(cols[e + 1] - cols[e]);
+  }
+  return d;
+}
+
+// Write 16 tokens (tile rows j0 .. j0 + 15, fewer at the end) of this thread's
+// latent column (its warp holds 32 consecutive columns) into the paged cache:
 // rounded to the latent dtype, or int4-quantised per 32-column block.
 template <int LAT>
-__device__ __forceinline__ void store_tokens(const CompressArgs& a, bool is_v, const uint16_t* cols, int ncols, int gc,
-                                             int t0, int j0, int ntok, const float* v, DevStatus* st) {
+__device__ __forceinline__ void store_tokens(const ColDst& cd, const int2* tab, int j0, int ntok, const float* v) {
   const int lane = threadIdx.x & 31;
-  const long long cap = (long long)a.num_pages * a.P;
-  const bool col_ok = gc < ncols;
-  const int e = col_ok ? col_entry(cols, a.gm.n, gc) : 0;   // group entry of this column
-  const int j = gc - cols[e];                                 // latent entry within it
-  uint8_t* pool = const_cast<uint8_t*>(is_v ? a.gm.zv[e] : a.gm.zk[e]);
-  const long long page_bytes = is_v ? a.gm.v_page : a.gm.k_page;
-#pragma unroll 1
+#pragma unroll
   for (int u = 0; u < 16; ++u) {
-    const int ti = t0 + j0 + u;
     if (j0 + u >= ntok) break;
-    const int slot = a.slots[ti];
-    if (slot < 0) continue;
-    if (slot >= cap) {
-      if (col_ok && (gc & 127) == 0) report(st, PALU_ERR_DEVICE_BOUNDS, 3000000 + ti);
-      continue;
-    }
+    const int2 d = tab[j0 + u];   // the same entry in every lane: warp-uniform branches
+    if (d.x < 0) continue;
+    uint8_t* dst = cd.col + (long long)d.x * cd.page_bytes + d.y * 128 + ((cd.unit ^ (d.y & 7)) << 4);
     if constexpr (LAT == PALU_INT4) {
       // the warp's 32 columns are one quantisation block of this token
-      float amax = col_ok ? fabsf(v[u]) : 0.f;
+      float amax = cd.ok ? fabsf(v[u]) : 0.f;
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
       const __half s16 = __float2half_rn(__fdiv_rn(amax, 7.0f));
@@ -128,18 +158,11 @@ __device__ __forceinline__ void store_tokens(const CompressArgs& a, bool is_v, c
       int code = 0;
       if (s != 0.f) code = (int)fminf(fmaxf(rintf(__fdiv_rn(v[u], s)), -7.f), 7.f);
       const int hi = __shfl_down_sync(0xffffffffu, code, 1);
-      if (col_ok && (lane & 1) == 0)
-        pool[(long long)(slot / a.P) * page_bytes + swz_offset(slot % a.P, j >> 1, a.P)] =
-            (uint8_t)((code & 0xF) | ((hi & 0xF) << 4));
-      if (col_ok && lane == 0) {
-        const uint8_t* spool = is_v ? a.gm.zvs[e] : a.gm.zks[e];
-        const long long srow = int4_scale_row(cols[e + 1] - cols[e]);
-        const long long spage = is_v ? a.gm.vs_page : a.gm.ks_page;
-        reinterpret_cast<__half*>(const_cast<uint8_t*>(spool) + (long long)(slot / a.P) * spage +
-                                  (slot % a.P) * srow)[j >> 5] = s16;
-      }
+      if (cd.ok && (lane & 1) == 0) *dst = (uint8_t)((code & 0xF) | ((hi & 0xF) << 4));
+      if (cd.ok && lane == 0)
+        *reinterpret_cast<__half*>(cd.spool + (long long)d.x * cd.spage + d.y * cd.srow) = s16;
     } else {
-      if (col_ok) store_latent<LAT>(a, pool + (long long)(slot / a.P) * page_bytes, j, slot, v[u]);
+      if (cd.ok) *reinterpret_cast<typename Dt<LAT>::T*>(dst) = Dt<LAT>::from_f(v[u]);
     }
   }
 }
@@ -160,6 +183,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 16);
   int* last_flag = reinterpret_cast<int*>(misc + 32);
+  int2* tok_tab = reinterpret_cast<int2*>(misc + 64);   // NT entries
   auto full = [&](int s) { return bars + 8u * s; };
   auto empty = [&](int s) { return bars + 8u * (p.stages + s); };
   const uint32_t d_full = bars + 8u * (2 * p.stages);
@@ -292,9 +316,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       finalize = *last_flag != 0;
       if (finalize) __threadfence();
     }
+    const int ntok = min(p.NT, a.n - t0);
     if (ok && finalize) {
-      const long long cap = (long long)a.num_pages * a.P;
-      const int ntok = min(p.NT, a.n - t0);
+      fill_token_table(a, t0, ntok, tok_tab, threadIdx.x - 64, kThreads - 64, st);
+      ok = ep_sync(57);
+    }
+    if (ok && finalize) {
+      const ColDst cd = col_dst<LAT>(a, is_v, cols, ncols, gc);
       for (int j0 = 0; j0 < ntok; j0 += 16) {
         float v[16];
         if (p.KS == 1) {
@@ -315,13 +343,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        store_tokens<LAT>(a, is_v, cols, ncols, gc, t0, j0, ntok, v, st);
+        store_tokens<LAT>(cd, tok_tab, j0, ntok, v);
       }
       // positions, once per token
       if (!is_v && ctile == 0 && a.positions != nullptr && a.pos_pool != nullptr) {
         for (int i = c; i < ntok; i += kM) {
-          const int slot = a.slots[t0 + i];
-          if (slot >= 0 && slot < cap) a.pos_pool[slot] = a.positions[t0 + i];
+          const int2 d = tok_tab[i];
+          if (d.x >= 0) a.pos_pool[(long long)d.x * a.P + d.y] = a.positions[t0 + i];
         }
       }
       if (p.KS > 1 && threadIdx.x == 64) t.counters[tile_id] = 0;   // reusable for the next call
@@ -353,15 +381,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* sbase = smem_raw + (base - raw);
   const int stage_bytes = kABytes + p.NT * 128;
-  const uint32_t bars = base + (uint32_t)p.stages * stage_bytes;      // 2·stages + 4 barriers
+  const uint32_t bars = base + (uint32_t)p.stages * stage_bytes;      // 2·stages + 6 barriers
   uint8_t* misc = sbase + (uint32_t)p.stages * stage_bytes + 256;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 16);
+  int2* tok_tab = reinterpret_cast<int2*>(misc + 64);   // 2 × NT entries, by tile parity
   auto full = [&](int s) { return bars + 8u * s; };
   auto empty = [&](int s) { return bars + 8u * (p.stages + s); };
   auto acc_full = [&](int b) { return bars + 8u * (2 * p.stages + b); };
   auto acc_empty = [&](int b) { return bars + 8u * (2 * p.stages + 2 + b); };
   const uint32_t td_bar = bars + 8u * (2 * p.stages + 4);   // teardown: every MMA has completed
+  const uint32_t epi_bar = bars + 8u * (2 * p.stages + 5);  // the 4 epilogue warps: token table written
   DevStatus* st = reinterpret_cast<DevStatus*>(a.status);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ctiles = p.tk + p.tv;
@@ -389,6 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(acc_empty(b), 4);
     }
     mbar_init(td_bar, 1);
+    mbar_init(epi_bar, 4);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -476,26 +507,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       int ctile, c0, t0;
       bool is_v;
       tile_of(i, ctile, is_v, c0, t0);
-      if (!mbar_wait(acc_full(b), (i >> 1) & 1, abort_flag, st, 64)) break;
-      tc_fence_after();
+      const int ntok = min(p.NT, a.n - t0);
+      // the token table of tile i (its parity's half; the other half may still be read
+      // for tile i - 1 by a slower warp, which has passed this sync only after it)
+      int2* tab = tok_tab + b * p.NT;
+      fill_token_table(a, t0, ntok, tab, threadIdx.x - 64, kThreads - 64, st);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(epi_bar);
+      if (!mbar_wait(epi_bar, (uint32_t)(i & 1), abort_flag, st, 66)) break;
       const uint16_t* cols = is_v ? a.vcol : a.kcol;
       const int ncols = is_v ? a.ncols_v : a.ncols_k;
-      const int ntok = min(p.NT, a.n - t0);
+      const ColDst cd = col_dst<LAT>(a, is_v, cols, ncols, c0 + c);
+      if (!mbar_wait(acc_full(b), (i >> 1) & 1, abort_flag, st, 64)) break;
+      tc_fence_after();
       for (int j0 = 0; j0 < ntok; j0 += 16) {
         float v[16];
         tmem_ld16(tmem + lane_addr + 256u * b + j0, v);
         tmem_wait_ld();
-        store_tokens<LAT>(a, is_v, cols, ncols, c0 + c, t0, j0, ntok, v, st);
+        store_tokens<LAT>(cd, tab, j0, ntok, v);
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_empty(b));
       // positions, once per token
       if (!is_v && ctile == 0 && a.positions != nullptr && a.pos_pool != nullptr) {
-        const long long cap = (long long)a.num_pages * a.P;
         for (int k = c; k < ntok; k += kM) {
-          const int slot = a.slots[t0 + k];
-          if (slot >= 0 && slot < cap) a.pos_pool[slot] = a.positions[t0 + k];
+          const int2 d = tab[k];
+          if (d.x >= 0) a.pos_pool[(long long)d.x * a.P + d.y] = a.positions[t0 + k];
         }
       }
     }
@@ -551,7 +589,8 @@ cudaError_t launch_t(const CompressArgs& a, cudaStream_t st) {
   uint8_t* scratch = reinterpret_cast<uint8_t*>(a.scratch);
   t.counters = reinterpret_cast<int*>(scratch);
   t.partials = reinterpret_cast<float*>(scratch + p.counter_bytes);
-  const size_t smem = (size_t)p.stages * (kABytes + p.NT * 128) + 256 + 64 + 1024;
+  // stages, barriers (256), flags (64), token tables (2 × NT), alignment
+  const size_t smem = (size_t)p.stages * (kABytes + p.NT * 128) + 256 + 64 + 2 * (size_t)p.NT * sizeof(int2) + 1024;
   if (p.ntt >= 2 && p.KS == 1) {
     // prefill: persistent, one CTA per SM over every tile
     auto kern = compress_tc_persistent_kernel<ACT, LAT>;

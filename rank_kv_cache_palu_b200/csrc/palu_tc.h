@@ -12,6 +12,8 @@ bool tc_decode_supported(const palu_config* c);
 // Head blocks per group the split kernel's grid uses (heads per CTA = 2).
 int tc_head_blocks(const palu_config* c);
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st);
+// The int4-latent instantiations (own translation unit); launch_decode_tc calls it.
+cudaError_t launch_decode_tc_int4(const DecodeArgs& a, cudaStream_t st);
 
 // Decode without RoPE: the key up-projection folded into the query, scores
 // taken on the cached latents (no key is rebuilt).  Its workspace adds the

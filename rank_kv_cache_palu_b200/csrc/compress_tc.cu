@@ -288,6 +288,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       epi_phase ^= 1;
       return rr;
     };
+    // the tokens' destinations, while the MMAs run; published by the syncs below
+    const int ntok = min(p.NT, a.n - t0);
+    fill_token_table(a, t0, ntok, tok_tab, threadIdx.x - 64, kThreads - 64, st);
     bool ok = mbar_wait(d_full, 0, abort_flag, st, 52);
     tc_fence_after();
     const int tile_id = blockIdx.x * p.ntt + blockIdx.y;
@@ -316,11 +319,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       finalize = *last_flag != 0;
       if (finalize) __threadfence();
     }
-    const int ntok = min(p.NT, a.n - t0);
-    if (ok && finalize) {
-      fill_token_table(a, t0, ntok, tok_tab, threadIdx.x - 64, kThreads - 64, st);
-      ok = ep_sync(57);
-    }
+    if (p.KS == 1) ok = ep_sync(57) && ok;
     if (ok && finalize) {
       const ColDst cd = col_dst<LAT>(a, is_v, cols, ncols, gc);
       for (int j0 = 0; j0 < ntok; j0 += 16) {

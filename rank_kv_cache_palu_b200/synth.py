@@ -139,6 +139,10 @@ WORKLOADS = {
            rank_v=256, batch=8, context=32768, act_dtype="f16", latent_dtype="int4", seed=4),
         _w("7b_bf16_r256_b32_t16k", num_heads=32, head_dim=128, group_size=4, rank_k=256,
            rank_v=256, batch=32, context=16384, act_dtype="bf16", latent_dtype="bf16", seed=5),
+        # the same layer with one short sequence: a small case whose prefill (bench --prefill)
+        # is the batch-32 workload's GEMM, for captures that must stay small on the device
+        _w("7b_bf16_r256_b1_t4k", num_heads=32, head_dim=128, group_size=4, rank_k=256,
+           rank_v=256, batch=1, context=4096, act_dtype="bf16", latent_dtype="bf16", seed=5),
         # attention without RoPE: the key up-projection folds into the query
         # (the fused, latent-space path)
         _w("7b_bf16_r256v128_b16_t16k_norope", num_heads=32, head_dim=128, group_size=4,

@@ -408,21 +408,26 @@ __global__ void __launch_bounds__(threads_of(LAT == PALU_INT4), 1)
       if (++stage == kNZK) { stage = 0; phase ^= 1; }
       return true;
     };
-    Slot s0, s1, s2, s3;                               // chunks n, n+1, n+2; s3 takes n+3
+    Slot s0, s1, s2, s3;                               // after the shift: chunks n, n+1, n+2; s3 takes n+3
     for (int kk = 1; kk <= kPrefetch; ++kk) prefetch_page(page_ahead(a, b, tr, kk));
     int pg_k = page_ahead(a, b, tr, 0);                // tile k of chunk n
     int pg_k1 = page_ahead(a, b, tr, 1);               // tile k+1
     int pg_k2 = page_ahead(a, b, tr, 2);               // tile k+2, in flight
     int pf = page_ahead(a, b, tr, 1 + kPrefetch);      // tile k+1+kPrefetch, pulled into L2
-    issue(0, s0, pg_k);
-    issue(1, s1, pg_k);
-    issue(2, s2, pg_k);
-    // One load batch and one conversion per chunk, the register slots shifted
-    // down after each: a single copy of the conversion code keeps the kernel's
-    // instruction footprint small.
+    issue(0, s1, pg_k);
+    issue(1, s2, pg_k);
+    issue(2, s3, pg_k);
+    // One load batch and one conversion per chunk: a single copy of the conversion
+    // code keeps the kernel's instruction footprint small.  The register slots shift
+    // down at the top of each iteration, before the next loads are issued, so a shift
+    // never copies a slot whose loads went out in the same iteration (the copy would
+    // wait for them).
 #pragma unroll 1
     for (int n = 0; n < N && !*abort_flag; ++n) {
       const int c = n & 3;
+      s0 = s1;
+      s1 = s2;
+      s2 = s3;
       if (c == 0 && n > 0) {
         pg_k = pg_k1;
         pg_k1 = pg_k2;
@@ -434,9 +439,6 @@ __global__ void __launch_bounds__(threads_of(LAT == PALU_INT4), 1)
         prefetch_page(pf);
         pf = page_ahead(a, b, tr, (n >> 2) + 2 + kPrefetch);
       }
-      s0 = s1;
-      s1 = s2;
-      s2 = s3;
     }
   } else if (warp >= 4) {
     if constexpr (kInt4) setmaxnreg_inc<kRegsEpi>();
@@ -811,14 +813,17 @@ __global__ void __launch_bounds__(threads_of(LAT == PALU_INT4), 1)
         if (++stage == kNVS) { stage = 0; phase ^= 1; }
         return true;
       };
-      Slot s0, s1, s2;                                   // stages n, n+1; s2 takes n+2
+      Slot s0, s1, s2;                                   // after the shift: stages n, n+1; s2 takes n+2
       int pg_k = page_ahead(a, b, tr, 0);                // tile k of stage n
       int pg_k1 = page_ahead(a, b, tr, 1);               // tile k+1
       int pg_k2 = page_ahead(a, b, tr, 2);               // tile k+2, in flight
-      issue(0, s0, pg_k);
-      issue(1, s1, pg_k);
+      issue(0, s1, pg_k);
+      issue(1, s2, pg_k);
+      // as for the keys: the slots shift before the next loads go out
   #pragma unroll 1
       for (int n = 0; n < N && !*abort_flag; ++n) {
+        s0 = s1;
+        s1 = s2;
         if (n % kSPT == 0 && n > 0) {
           pg_k = pg_k1;
           pg_k1 = pg_k2;
@@ -826,8 +831,6 @@ __global__ void __launch_bounds__(threads_of(LAT == PALU_INT4), 1)
         }
         issue(n + 2, s2, (n + 2) / kSPT == n / kSPT ? pg_k : pg_k1);
         if (!consume(n, s0)) break;
-        s0 = s1;
-        s1 = s2;
       }
     } else if (warp == 0) {
       // ============================================================ z_k producer (bulk copies)

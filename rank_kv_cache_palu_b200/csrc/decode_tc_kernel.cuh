@@ -346,10 +346,17 @@ __global__ void __launch_bounds__(threads_of(LAT == PALU_INT4), 1)
   if (warp == 0 && lane == 0) {
     mbar_expect_tx(bar(BAR_B), (uint32_t)r_k * 256 * 2);
     // 64-column blocks of B_k (MN-major, 128-byte swizzle), each in boxes of bk_box rows
+    // int4 latents: the rows (latent entries) in the key converters' paired order, row
+    // 8g + 2a + b of shared memory = row 8g + 4b + a of B_k (a 4-D view of B_k, see the launcher)
     for (int nb = 0; nb < 4; ++nb)
-      for (int rb = 0; rb < r_k; rb += a.bk_box)
-        tma_load_2d(base + L.b + (uint32_t)nb * r_k * 128 + rb * 128, &tm_bk, hp * 256 + nb * 64,
-                    gm.k_row0[gi] + rb, bar(BAR_B));
+      for (int rb = 0; rb < r_k; rb += a.bk_box) {
+        if constexpr (kInt4)
+          tma_load_4d(base + L.b + (uint32_t)nb * r_k * 128 + rb * 128, &tm_bk, hp * 256 + nb * 64, 0, 0,
+                      (gm.k_row0[gi] + rb) / 8, bar(BAR_B));
+        else
+          tma_load_2d(base + L.b + (uint32_t)nb * r_k * 128 + rb * 128, &tm_bk, hp * 256 + nb * 64,
+                      gm.k_row0[gi] + rb, bar(BAR_B));
+      }
   }
   // Roles.  int4 latents: each warpgroup first sets its share of the register file
   // (setmaxnreg, see kRegsLaunch), inside the branch whose code uses it.
@@ -359,7 +366,10 @@ __global__ void __launch_bounds__(threads_of(LAT == PALU_INT4), 1)
     // Chunk c of a tile = entries [64c, 64c + 64) of all 128 tokens, i.e. scale
     // blocks 2c and 2c+1 = 16-byte units 2c and 2c+1 of each token's row of codes.
     // Thread t takes both units of token t, loaded straight into registers three
-    // chunks ahead of the conversion, while later pages are pulled into L2.
+    // chunks ahead of the conversion, while later pages are pulled into L2.  Entries
+    // are written PAIRED (K position p of the operand holds entry paired_row(p)), which
+    // saves byte permutes; B_k's rows are loaded in the same order, so the key MMA sums
+    // the same products.
     const int t = threadIdx.x - 384;
     const int N = tr.ntiles * 4;
     struct Slot {
@@ -400,7 +410,7 @@ __global__ void __launch_bounds__(threads_of(LAT == PALU_INT4), 1)
         const uint32_t w[4] = {sl.raw[ub].x, sl.raw[ub].y, sl.raw[ub].z, sl.raw[ub].w};
 #pragma unroll
         for (int m = 0; m < 4; ++m)
-          st_shared_v4(dst + (((4 * ub + m) ^ (t & 7)) << 4), dequant8<ACT, false>(w[m], sl.sc[ub]));
+          st_shared_v4(dst + (((4 * ub + m) ^ (t & 7)) << 4), dequant8<ACT, true>(w[m], sl.sc[ub]));
       }
       fence_proxy_async();
       __syncwarp();
@@ -1091,14 +1101,38 @@ bool make_map_2d(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, int el
   return r == CUDA_SUCCESS;
 }
 
+// B_k (row-major [rows][W], 16-bit) as a 4-D map for the paired row order: dims (innermost
+// first) columns, b (stride 4 rows), a (stride 1 row), g (stride 8 rows); boxes of 64
+// columns × 2 × 4 × box_rows/8.
+bool make_map_bk_paired(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, uint64_t W, uint64_t rows,
+                        uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  const uint64_t rb = W * 2;   // bytes per row
+  cuuint64_t dims[4] = {W, 2, 4, rows / 8};
+  cuuint64_t strides[3] = {4 * rb, rb, 8 * rb};
+  cuuint32_t box[4] = {64, 2, 4, box_rows / 8};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(m, dt, 4, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 template <int ACT, int NRV, int LAT>
 cudaError_t launch_t(const DecodeArgs& a, cudaStream_t st) {
   const CUtensorMapDataType dt = ACT == PALU_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   CUtensorMap tm_bk;
   if (a.bk_box <= 0 || a.bk_box > 256 || a.bk_box % 64 != 0) return cudaErrorInvalidValue;
-  if (!make_map_2d(&tm_bk, a.Bk, dt, 2, a.W, (uint64_t)a.bk_rows, (uint64_t)a.W * 2, 64, a.bk_box,
-                   CU_TENSOR_MAP_SWIZZLE_128B))
+  if constexpr (LAT == PALU_INT4) {
+    // B_k viewed as [rows / 8][a: 4][b: 2][W] with the b dimension traversed before a, so a
+    // box lands row 8g + 4b + a of B_k at row 8g + 2a + b of shared memory: the paired
+    // order the key converters write the latent entries in
+    if (a.bk_rows % 8 != 0 || !make_map_bk_paired(&tm_bk, a.Bk, dt, a.W, (uint64_t)a.bk_rows, a.bk_box))
+      return cudaErrorInvalidValue;
+  } else if (!make_map_2d(&tm_bk, a.Bk, dt, 2, a.W, (uint64_t)a.bk_rows, (uint64_t)a.W * 2, 64, a.bk_box,
+                          CU_TENSOR_MAP_SWIZZLE_128B)) {
     return cudaErrorInvalidValue;
+  }
   const Smem L = smem_layout(a.r_k, LAT == PALU_INT4);
   const size_t smem = L.total + 1024;
   auto kern = a.pos_pool == nullptr ? decode_tc_kernel<ACT, NRV, LAT, true> : decode_tc_kernel<ACT, NRV, LAT, false>;

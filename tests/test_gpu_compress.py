@@ -256,3 +256,35 @@ def test_compress_int4_prefill_bit_exact(act):
         np.testing.assert_array_equal(got_s[keep], sc[keep])
     pos = cache.pos.cpu().numpy()
     np.testing.assert_array_equal(pos[slots[keep]], positions[keep])
+
+
+@pytest.mark.parametrize("n", [16, 600])
+def test_compress_tc_bad_slot_and_holes(n):
+    # Tensor-core compress, both forms: 16 tokens (one token tile, K split across CTAs) and
+    # 600 (the persistent prefill, several tiles and a ragged one).  Each tile looks its
+    # tokens' slots up once; an out-of-pool slot is reported (PALU_ERR_DEVICE_BOUNDS) and,
+    # like a skipped one (-1), writes nothing, while every other token lands in its slot
+    # with its position.
+    dt = "bf16"
+    w = dataclasses.replace(WORKLOADS["7b_bf16_r256v128_b1_t4k"], num_heads=8, d_model=512)
+    x = normal_tensor(31, "x", (n, w.d_model), dt)
+    A_k = normal_tensor(31, "A_k", (w.d_model, w.groups * w.rank_k), dt, 1 / math.sqrt(w.d_model))
+    A_v = normal_tensor(31, "A_v", (w.d_model, w.groups * w.rank_v), dt, 1 / math.sqrt(w.d_model))
+    num_pages = 8
+    cap = num_pages * w.page_size
+    slots = make_slots(n, num_pages, w.page_size, seed=31)
+    valid = np.flatnonzero(slots >= 0)
+    slots[valid[len(valid) // 2]] = cap + 5
+    positions = (np.arange(n) * 5 + 1).astype(np.int32)
+    cache, st, _ = run_compress(w, x, A_k, A_v, slots, positions, num_pages)
+    assert st == 7
+    keep = (slots >= 0) & (slots < cap)
+    rows = np.flatnonzero(keep)
+    _check_rows(w, x, A_k, cache.zk, slots, rows, w.rank_k, dt)
+    _check_rows(w, x, A_v, cache.zv, slots, rows, w.rank_v, dt)
+    others = np.setdiff1d(np.arange(cap, dtype=np.int32), slots[keep])
+    for pool, r in ((cache.zk, w.rank_k), (cache.zv, w.rank_v)):
+        assert np.all(gather_rows(pool, w, others, r, r * 2) == SENTINEL)
+    pos = cache.pos.cpu().numpy()
+    np.testing.assert_array_equal(pos[slots[keep]], positions[keep])
+    assert np.all(pos[others] == 0)

@@ -423,16 +423,17 @@ class Setup:
         self.out = torch.empty(self.qshape, dtype=act, device=dev)
         self.stream = torch.cuda.current_stream(dev)
 
-    def decode(self, q, qpos, lens):
+    def decode(self, q, qpos, lens, out=None):
         w, P, c = self.w, self.P, self.cache
+        out = self.out if out is None else out
         if w.ranked:
             P.palu_decode_attn_ranked(self.cfg, self.rks, self.rvs, q, qpos, c.zk, c.zv, c.zks, c.zvs, None,
-                                      self.page_table, lens, self.num_pages, self.B_k, self.B_v, self.out, None,
+                                      self.page_table, lens, self.num_pages, self.B_k, self.B_v, out, None,
                                       self.ws_d, self.S, self.stream)
             return
         fn = P.palu_decode_attn if self.Q == 1 else P.palu_decode_attn_multi
         fn(self.cfg, q, qpos, c.zk, c.zv, c.zks, c.zvs, None, self.page_table, lens, self.num_pages, self.B_k,
-           self.B_v, self.out, None, self.ws_d, self.S, self.stream)
+           self.B_v, out, None, self.ws_d, self.S, self.stream)
 
     def compress(self, x, slots):
         w, P, c = self.w, self.P, self.cache
@@ -622,38 +623,92 @@ def run_ours(args):
     units = sum(su.step_units(s) for s in range(first_step, first_step + args.steps))
     value = D.sum_over_ranks(units, dev) / (el_ms / 1e3)
 
-    # ---- end to end through the public API: pinned host inputs -> H2D -> step -> D2H
-    xh = [t.cpu().pin_memory() for t in su.xs]
-    qh = [t.cpu().pin_memory() for t in su.qs]
-    meta_h = [tuple(m.cpu().pin_memory() for m in su.metas[s]) for s in range(steps_total)]
-    outh = torch.empty(su.out.shape, dtype=su.out.dtype).pin_memory()
-    x_d, q_d = torch.empty_like(su.xs[0]), torch.empty_like(su.qs[0])
-    m_d = tuple(torch.empty_like(m) for m in su.metas[0])
-    h2d = su.xs[0].numel() * su.xs[0].element_size() + su.qs[0].numel() * su.qs[0].element_size() + \
-        sum(m.numel() * m.element_size() for m in su.metas[0])
+    # ---- end to end through the public API: pinned host inputs -> H2D -> step -> D2H.
+    # A step's inputs (x, q, slots, query positions, lengths) travel as one copy from one
+    # pinned buffer, and its output comes back as one copy.  Two device input and output
+    # buffers alternate, so that on copy streams the upload of step s + 1 and the read-back
+    # of step s run while step s computes; events order every copy against the steps that
+    # produce or consume its buffer, and all copies lie inside the timed region.
+    def packed(ts):
+        offs, n = [], 0
+        for t in ts:
+            n = (n + 255) // 256 * 256
+            offs.append(n)
+            n += t.numel() * t.element_size()
+        return offs, n
+    in_parts = [su.xs[0], su.qs[0], *su.metas[0]]
+    in_offs, in_bytes = packed(in_parts)
+
+    def host_inputs(s):
+        buf = torch.zeros(in_bytes, dtype=torch.uint8).pin_memory()
+        for t, o in zip([su.xs[s % su.ring], su.qs[s % su.ring], *su.metas[s]], in_offs):
+            flat = t.detach().cpu().contiguous().view(torch.uint8).reshape(-1)
+            buf[o:o + flat.numel()].copy_(flat)
+        return buf
+    host_in = [host_inputs(s) for s in range(steps_total)]
+    dev_in = [torch.empty(in_bytes, dtype=torch.uint8, device=dev) for _ in range(2)]
+
+    def views(buf):
+        return [buf[o:o + t.numel() * t.element_size()].view(t.dtype).view(t.shape) for t, o in zip(in_parts, in_offs)]
+    dev_views = [views(d) for d in dev_in]
+    out_d = [torch.empty_like(su.out) for _ in range(2)]
+    out_h = [torch.empty(su.out.shape, dtype=su.out.dtype).pin_memory() for _ in range(2)]
+    h2d = in_bytes
     d2h = su.out.numel() * su.out.element_size()
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in_ready = [torch.cuda.Event() for _ in range(2)]
+    ev_in_free = [torch.cuda.Event() for _ in range(2)]
+    ev_out_ready = [torch.cuda.Event() for _ in range(2)]
+    ev_out_free = [torch.cuda.Event() for _ in range(2)]
+    used = [False, False]
 
-    def e2e_step(s):
-        x_d.copy_(xh[s % su.ring], non_blocking=True)
-        q_d.copy_(qh[s % su.ring], non_blocking=True)
-        for dst, src in zip(m_d, meta_h[s]):
-            dst.copy_(src, non_blocking=True)
-        su.compress(x_d, m_d[0])
-        su.decode(q_d, m_d[1], m_d[2])
-        outh.copy_(su.out, non_blocking=True)
+    def upload(s, j):
+        with torch.cuda.stream(up):
+            if used[j]:
+                up.wait_event(ev_in_free[j])      # the step that read this buffer is done
+            dev_in[j].copy_(host_in[s], non_blocking=True)
+            ev_in_ready[j].record(up)
 
-    for _ in range(min(args.warmup, 3)):
-        e2e_step(s_idx)
-        s_idx += 1
+    def compute(s, j):
+        stream.wait_event(ev_in_ready[j])
+        if used[j]:
+            stream.wait_event(ev_out_free[j])     # the previous result in this buffer is back
+        x_d, q_d, slots_d, qpos_d, lens_d = dev_views[j]
+        su.compress(x_d, slots_d)
+        su.decode(q_d, qpos_d, lens_d, out=out_d[j])
+        ev_in_free[j].record(stream)
+        ev_out_ready[j].record(stream)
+        used[j] = True
+
+    def download(j):
+        with torch.cuda.stream(down):
+            down.wait_event(ev_out_ready[j])
+            out_h[j].copy_(out_d[j], non_blocking=True)
+            ev_out_free[j].record(down)
+
+    def run_steps(first, count, start_ev=None):
+        if start_ev is not None:
+            up.wait_event(start_ev)
+            down.wait_event(start_ev)
+        upload(first, 0)
+        for i in range(count):
+            j = i % 2
+            if i + 1 < count:
+                upload(first + i + 1, (i + 1) % 2)
+            compute(first + i, j)
+            download(j)
+        for j in range(min(count, 2)):
+            stream.wait_event(ev_out_free[j])     # every read-back is in before the end event
+
+    run_steps(s_idx, min(args.warmup, 3))
+    s_idx += min(args.warmup, 3)
     torch.cuda.synchronize(dev)
     D.barrier(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e2e_units = 0
     e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step(s_idx)
-        e2e_units += su.step_units(s_idx)
-        s_idx += 1
+    run_steps(s_idx, args.steps, start_ev=e0)
+    e2e_units = sum(su.step_units(s) for s in range(s_idx, s_idx + args.steps))
+    s_idx += args.steps
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = D.max_over_ranks(e0.elapsed_time(e1), dev)
